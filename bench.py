@@ -1,0 +1,438 @@
+#!/usr/bin/env python
+"""Benchmark of routed block-sparse attention (forward) on B200.
+
+One step = the whole hot path on one synthetic attention call: (optional
+Hilbert gather +) block-mean pooling, proxy scoring + Top-p routing + CSR,
+routed attention with residual pseudo-keys, output (scatter).  Inputs are
+resident in HBM when the timed region starts; the L2 is flushed (a 256 MiB
+write) between timed steps, outside the timed events.
+
+value = FLOPs actually computed by the attention (4 d per exact query-key
+pair plus 4 d per query-pseudo-key pair) / device time of the whole step.
+The line also carries the dense-equivalent rate, the fraction of the
+measured bf16 tensor peak, and the speedup over the same library's dense
+(tau = 1) path on the same inputs.
+
+  python bench.py [--gpus N --steps K --warmup W] [--workload medium]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "block-sparse attn fwd: effective TFLOP/s, % of B200 BF16 peak, speedup vs dense"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 5  # pool, route, scan, compact, attend
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="medium",
+                    choices=["tiny", "medium", "wan", "hunyuan", "stress"])
+    ap.add_argument("--tau", type=float, default=None)
+    ap.add_argument("--residual", type=int, default=None)
+    ap.add_argument("--no-dense", action="store_true", help="skip the tau = 1 comparison run")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="CPU time budget of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_from_args(args, rank=0):
+    from workloads import get_config
+    ov = {}
+    if args.tau is not None:
+        ov["tau"] = args.tau
+    if args.residual is not None:
+        ov["residual"] = args.residual
+    w = get_config(args.workload, **ov)
+    if rank:
+        w = w.with_(seed=w.seed + 1000 * rank)   # independent replica per rank
+    return w
+
+
+def attention_flops(row_ptr, col_idx, w, nb):
+    """(exact, residual) FLOPs: 4 d per query-key pair, from the CSR."""
+    b, N, d = w.b, w.N, w.d
+    n_last = N - (nb - 1) * b
+    rows = len(row_ptr) - 1
+    k = np.diff(row_ptr).astype(np.int64)
+    row_id = np.repeat(np.arange(rows), k)
+    has_last = np.bincount(row_id[col_idx[: row_ptr[-1]] == nb - 1], minlength=rows)
+    keys_per_row = b * k - (b - n_last) * has_last
+    n_i = np.full(rows, b, np.int64)
+    n_i[np.arange(rows) % nb == nb - 1] = n_last
+    exact = 4 * d * int(np.sum(n_i * keys_per_row))
+    res = 4 * d * int(np.sum(n_i * (nb - k))) if w.residual else 0
+    return exact, res
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [x.get("num_threads", 1) for x in threadpool_info() if x.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(w, seconds, Q=None, K=None, V=None, perm=None):
+    """Time the fp64 oracle on a bounded sample of the workload.
+
+    Sample: head (0, 0) -- decode, gather, block means, proxy, routing of all
+    its query blocks -- then routed attention of successive query blocks of
+    that head until `seconds` of wall time have passed.  Returns
+    (TFLOP/s of the sampled attention, description).
+    """
+    from oracle import spattn_ref as R
+    from workloads import make_qkv
+    if Q is None:
+        Q, K, V = make_qkv(w.with_(H=1, B=1))
+    t0 = time.perf_counter()
+    q = R.gather_tokens(R.decode_bf16(Q[0, 0]), perm)
+    k = R.gather_tokens(R.decode_bf16(K[0, 0]), perm)
+    v = R.gather_tokens(R.decode_bf16(V[0, 0]), perm)
+    n = R.block_sizes(w.N, w.b)
+    Qb, Kb, Vb = R.block_means(q, w.b), R.block_means(k, w.b), R.block_means(v, w.b)
+    route = R.route_rows(R.block_softmax(R.proxy_logits(Qb, Kb, n)), w.tau, w.kmin, w.kmax)
+    flops = 0
+    blocks = 0
+    order = np.random.default_rng(0).permutation(len(n))
+    for i in order:
+        rows = np.arange(i * w.b, i * w.b + n[i])
+        R.attention(q, k, v, route["kept"], w.b, bool(w.residual), Kb, Vb, rows=rows)
+        nk = int(n[route["kept"][i]].sum())
+        flops += 4 * w.d * int(n[i]) * (nk + (len(n) - len(route["kept"][i]) if w.residual else 0))
+        blocks += 1
+        if time.perf_counter() - t0 > seconds:
+            break
+    dt = time.perf_counter() - t0
+    desc = (f"head 0 of {w.name}: pooling + routing of all {len(n)} query blocks, then routed "
+            f"attention of {blocks} random query blocks ({blocks * w.b} query tokens); "
+            f"{dt:.1f} s wall; TFLOP/s = sampled attention FLOPs / total wall time")
+    return flops / dt / 1e12, desc, dt
+
+
+def run_reference(args):
+    """The oracle (fp64, CPU) timed on the host cores on the same config."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = workload_from_args(args)
+    from workloads import make_qkv
+    Q, K, V = make_qkv(w.with_(H=1, B=1))
+    perm = None
+    if w.hilbert:
+        import oracle
+        perm = oracle.hilbert_perm(w.grid)
+    per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, per_step, Q, K, V, perm)
+    vals, times, desc = [], [], ""
+    for _ in range(args.steps):
+        v, desc, dt = oracle_sample(w, per_step, Q, K, V, perm)
+        vals.append(v)
+        times.append(dt)
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * float(np.mean(times)), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, "cpu"),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": "each step: " + desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, l2):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "b": w.b,
+            "nb": w.nb, "tau": w.tau, "kmin": w.kmin, "kmax": w.kmax, "residual": w.residual,
+            "hilbert": w.hilbert, "grid": list(w.grid), "global_batch": w.B, "seq_len": w.N,
+            "parallelism": "replicas", "l2": l2}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    import block_sparse_attention_33_b200 as sp
+    from block_sparse_attention_33_b200 import build
+    if rank == 0 and not build.up_to_date():
+        build.build()
+    if world > 1:
+        dist.barrier()
+    sp.lib()
+    from workloads import make_qkv
+
+    w = workload_from_args(args, rank)
+    Qh, Kh, Vh = make_qkv(w)
+    perm = sp.spattn_hilbert_perm(*w.grid) if w.hilbert else None
+    B, H, N, d = Qh.shape
+
+    def dev_bf16(x):
+        return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v = dev_bf16(Qh), dev_bf16(Kh), dev_bf16(Vh)
+    o = torch.empty_like(q)
+    plan = sp.Plan(B, H, N, d, w.b, w.tau, w.kmin, w.kmax, w.residual, perm, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn_list, steps, warmup):
+        """Per step: flush L2, then events around each fn; returns [steps][len(fns)] ms."""
+        for _ in range(warmup):
+            flush.zero_()
+            for fn in fn_list:
+                fn()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(fn_list) + 1)]
+               for _ in range(steps)]
+        for s in range(steps):
+            flush.zero_()
+            evs[s][0].record(stream)
+            for i, fn in enumerate(fn_list):
+                fn()
+                evs[s][i + 1].record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        return [[evs[s][i].elapsed_time(evs[s][i + 1]) for i in range(len(fn_list))]
+                for s in range(steps)]
+
+    row_ptr = torch.zeros(B * H * plan.nb + 1, dtype=torch.int32, device=dev)
+    col_idx = torch.zeros(max(plan.col_capacity, 1), dtype=torch.int32, device=dev)
+    # routing once to count FLOPs (deterministic: same every step)
+    plan.route(q, k, v, row_ptr, col_idx)
+    torch.cuda.synchronize(dev)
+    rp, ci = row_ptr.cpu().numpy(), col_idx.cpu().numpy()
+    exact, resid = attention_flops(rp, ci, w, plan.nb)
+    step_flops = exact + resid
+    kept_frac = float(np.diff(rp).sum()) / (B * H * plan.nb * plan.nb)
+    dense_flops = 4 * N * N * d * B * H
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    t = timed([lambda: plan.route(q, k, v), lambda: plan.attend(q, k, v, o)], args.steps,
+              args.warmup)
+    clk = clocks.stop()
+    route_ms = float(np.mean([x[0] for x in t]))
+    attend_ms = float(np.mean([x[1] for x in t]))
+    step_ms = route_ms + attend_ms
+
+    status = plan.check()
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {sp.spattn_last_error()}")
+
+    # max over ranks of the step time (device-timed)
+    if world > 1:
+        tt = torch.tensor([step_ms, attend_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        step_ms, attend_ms = tt.tolist()
+        ff = torch.tensor([float(step_flops)], device=dev, dtype=torch.float64)
+        dist.all_reduce(ff)
+        total_flops = ff.item()
+    else:
+        total_flops = float(step_flops)
+
+    value = total_flops / (step_ms * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    attn_tflops = step_flops / (attend_ms * 1e-3) / 1e12
+
+    # the same library's dense path (tau = 1) on the same inputs
+    dense_ms = None
+    if not args.no_dense:
+        dplan = sp.Plan(B, H, N, d, w.b, 1.0, 1, 1 << 30, w.residual, perm, device=dev)
+        td = timed([lambda: dplan.forward(q, k, v, o)], max(3, args.steps // 3), 2)
+        dense_ms = float(np.mean([x[0] for x in td]))
+        if world > 1:
+            tt = torch.tensor([dense_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            dense_ms = tt.item()
+        dplan.close()
+
+    # kernel breakdown: the pooling kernel alone (HBM-bound)
+    tp = timed([lambda: plan.pool(q, k, v)], max(3, args.steps // 3), 2)
+    pool_ms = float(np.mean([x[0] for x in tp]))
+    tok_bytes = B * H * N * d * 2
+    pool_bytes = 3 * tok_bytes + B * H * plan.nb * d * (3 * 4 + 2 * 2)
+    if perm is not None:
+        pool_bytes += 3 * tok_bytes
+
+    # end to end through the public call with host buffers
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+                      for x in (Qh, Kh, Vh))
+        oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+
+        def e2e_step():
+            q.copy_(qh, non_blocking=True)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            plan.forward(q, k, v, o)
+            oh.copy_(o, non_blocking=True)
+
+        te = timed([e2e_step], max(3, args.steps // 3), 2)
+        e2e_ms = float(np.mean([x[0] for x in te]))
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = tt.item()
+        e2e = {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * tok_bytes,
+               "d2h_bytes_per_step": tok_bytes}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, desc, _ = oracle_sample(w, args.cpu_seconds, perm=perm)
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc}
+
+    plan.close()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": config_of(w, "flushed (256 MiB write between timed steps)"),
+            "dense_equiv_tflops": dense_flops * world / (step_ms * 1e-3) / 1e12,
+            "attn_tflops": attn_tflops,
+            "pct_of_bf16_peak": 100.0 * attn_tflops / bf16_peak,
+            "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None,
+            "dense_ms_per_step": dense_ms,
+            "kept_fraction": kept_frac,
+            "flops_exact": exact, "flops_residual": resid,
+            "kernels_ms": {"route_total": route_ms, "attend": attend_ms, "pool": pool_ms},
+            "roofline": {"bound": "tensor", "kernel": "attention", "achieved": attn_tflops,
+                         "peak": bf16_peak, "unit": "TFLOP/s", "frac": attn_tflops / bf16_peak,
+                         "peak_kind": f"{peak_kind} bf16 dense (burst)", "traffic": None},
+            "roofline_pool": {"bound": "hbm", "kernel": "pool", "achieved": pool_bytes / (pool_ms * 1e-3) / 1e9,
+                              "peak": hbm_peak, "unit": "GB/s",
+                              "frac": pool_bytes / (pool_ms * 1e-3) / 1e9 / hbm_peak,
+                              "peak_kind": f"{peak_kind} copy bandwidth", "traffic": None},
+            "clocks": clk,
+            "e2e": e2e,
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,196 @@
+"""Python binding of libspattn (routed block-sparse attention for B200).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``libspattn.so``.  Tensors may be passed as torch tensors (their device
+pointer is used) or as raw integer addresses.  There is no fallback: if the
+library is missing, importing a function raises.
+
+The functions carry the names of the C entry points in ``include/spattn.h``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libspattn.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(7)
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA",
+                5: "TIMEOUT", 6: "DEVICE"}
+
+EXPORTS = ("spattn_plan", "spattn_plan_destroy", "spattn_plan_info", "spattn_pool",
+           "spattn_route", "spattn_attend", "spattn_forward", "spattn_means", "spattn_check",
+           "spattn_hilbert_perm", "spattn_last_error")
+
+
+class SpAttnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"spattn status {STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """Load libspattn.so (built in-tree by build.build()); raise if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -c 'import __graft_entry__ as g; g.build()'`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, F, S, I32P, SZP = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t,
+                             ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_size_t))
+    sig = {
+        "spattn_plan": [ctypes.POINTER(P), I, I, I, I, I, F, I, I, I, P, SZP],
+        "spattn_plan_destroy": [P],
+        "spattn_plan_info": [P, ctypes.POINTER(I), ctypes.POINTER(ctypes.c_int64)],
+        "spattn_pool": [P, P, P, P, P, P],
+        "spattn_route": [P, P, P, P, P, P, P, P],
+        "spattn_attend": [P, P, P, P, P, P, P, P, P],
+        "spattn_forward": [P, P, P, P, P, P, P],
+        "spattn_means": [P, P, P, P, P, P],
+        "spattn_check": [P, P, P],
+        "spattn_hilbert_perm": [I, I, I, P],
+    }
+    for name, args in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    L.spattn_last_error.argtypes = []
+    L.spattn_last_error.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if hasattr(x, "ctypes"):
+        return x.ctypes.data
+    raise TypeError(f"cannot take a pointer of {type(x)}")
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(st: int):
+    if st != OK:
+        raise SpAttnError(st, lib().spattn_last_error().decode())
+
+
+def spattn_last_error() -> str:
+    return lib().spattn_last_error().decode()
+
+
+def spattn_plan(B, H, N, d, b, tau, kmin, kmax, residual, perm=None):
+    """Create a plan; returns (handle, workspace_bytes).  perm: host int32 array or None."""
+    import numpy as np
+    h = ctypes.c_void_p()
+    ws = ctypes.c_size_t()
+    pp = None
+    if perm is not None:
+        perm = np.ascontiguousarray(perm, dtype=np.int32)
+        pp = perm.ctypes.data
+    _check(lib().spattn_plan(ctypes.byref(h), B, H, N, d, b, float(tau), kmin, kmax, residual,
+                             pp, ctypes.byref(ws)))
+    return h.value, ws.value
+
+
+def spattn_plan_destroy(plan):
+    _check(lib().spattn_plan_destroy(plan))
+
+
+def spattn_plan_info(plan):
+    nb = ctypes.c_int()
+    cap = ctypes.c_int64()
+    _check(lib().spattn_plan_info(plan, ctypes.byref(nb), ctypes.byref(cap)))
+    return nb.value, cap.value
+
+
+def spattn_pool(plan, Q, K, V, workspace, stream=None):
+    _check(lib().spattn_pool(plan, _ptr(Q), _ptr(K), _ptr(V), _ptr(workspace), _stream(stream)))
+
+
+def spattn_route(plan, Q, K, V, workspace, row_ptr=None, col_idx=None, stream=None):
+    _check(lib().spattn_route(plan, _ptr(Q), _ptr(K), _ptr(V), _ptr(workspace), _ptr(row_ptr),
+                              _ptr(col_idx), _stream(stream)))
+
+
+def spattn_attend(plan, Q, K, V, O, workspace, row_ptr=None, col_idx=None, stream=None):
+    _check(lib().spattn_attend(plan, _ptr(Q), _ptr(K), _ptr(V), _ptr(row_ptr), _ptr(col_idx),
+                               _ptr(O), _ptr(workspace), _stream(stream)))
+
+
+def spattn_forward(plan, Q, K, V, O, workspace, stream=None):
+    _check(lib().spattn_forward(plan, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(workspace),
+                                _stream(stream)))
+
+
+def spattn_means(plan, workspace, Qbar=None, Kbar=None, Vbar=None, stream=None):
+    _check(lib().spattn_means(plan, _ptr(workspace), _ptr(Qbar), _ptr(Kbar), _ptr(Vbar),
+                              _stream(stream)))
+
+
+def spattn_check(plan, workspace, stream=None) -> int:
+    """Synchronise and return the device status code (does not raise)."""
+    return lib().spattn_check(plan, _ptr(workspace), _stream(stream))
+
+
+def spattn_hilbert_perm(T, Hs, W):
+    """perm[new] = old for a T x Hs x W grid along the library's 3D Hilbert curve."""
+    import numpy as np
+    out = np.empty(T * Hs * W, dtype=np.int32)
+    _check(lib().spattn_hilbert_perm(T, Hs, W, out.ctypes.data))
+    return out
+
+
+class Plan:
+    """Owning wrapper: a plan plus its device workspace (torch allocation)."""
+
+    def __init__(self, B, H, N, d, b, tau, kmin, kmax, residual, perm=None, device="cuda"):
+        import torch
+        self.shape = (B, H, N, d)
+        self.handle, self.ws_bytes = spattn_plan(B, H, N, d, b, tau, kmin, kmax, residual, perm)
+        self.nb, self.col_capacity = spattn_plan_info(self.handle)
+        self.workspace = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=device)
+
+    def forward(self, Q, K, V, O, stream=None):
+        spattn_forward(self.handle, Q, K, V, O, self.workspace, stream)
+
+    def route(self, Q, K, V, row_ptr=None, col_idx=None, stream=None):
+        spattn_route(self.handle, Q, K, V, self.workspace, row_ptr, col_idx, stream)
+
+    def attend(self, Q, K, V, O, row_ptr=None, col_idx=None, stream=None):
+        spattn_attend(self.handle, Q, K, V, O, self.workspace, row_ptr, col_idx, stream)
+
+    def pool(self, Q, K, V, stream=None):
+        spattn_pool(self.handle, Q, K, V, self.workspace, stream)
+
+    def check(self, stream=None) -> int:
+        return spattn_check(self.handle, self.workspace, stream)
+
+    def close(self):
+        if self.handle:
+            spattn_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

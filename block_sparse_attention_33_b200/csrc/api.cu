@@ -1,0 +1,335 @@
+// C ABI of libspattn: plans, workspace layout, argument checks, dispatch.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <new>
+#include <numeric>
+#include <vector>
+
+#include "../../include/spattn.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace spattn {
+cudaError_t launch_attend_mma(const Problem& p, const void* Q, const void* K, const void* V,
+                              const int32_t* row_ptr, const int32_t* col_idx, void* O,
+                              const Work& w, cudaStream_t s);
+}  // namespace spattn
+
+using spattn::Problem;
+using spattn::Work;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+spattn_status_t fail(spattn_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+spattn_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(SPATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr size_t ALIGN = 256;
+inline size_t up(size_t x) { return (x + ALIGN - 1) / ALIGN * ALIGN; }
+
+// Byte offsets of the workspace regions.
+struct Layout {
+  size_t qp, kp, vp, qbar, kbar, vbar, kbar16, vbar16, counts, lists, row_ptr, col_idx, order,
+      ctrl, total;
+};
+
+Layout make_layout(const Problem& p) {
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += up(bytes); return o; };
+  const size_t tok = (size_t)p.BH * p.N * p.d;
+  const size_t cen = (size_t)p.BH * p.nb * p.d;
+  const size_t rows = (size_t)p.BH * p.nb;
+  const bool perm = p.perm != nullptr;
+  L.qp = perm ? take(tok * 2) : 0;
+  L.kp = perm ? take(tok * 2) : 0;
+  L.vp = perm ? take(tok * 2) : 0;
+  L.qbar = take(cen * 4);
+  L.kbar = take(cen * 4);
+  L.vbar = take(cen * 4);
+  L.kbar16 = take(cen * 2);
+  L.vbar16 = take(cen * 2);
+  L.counts = take(rows * 4);
+  L.lists = take(rows * p.kcap * 4);
+  L.row_ptr = take((rows + 1) * 4);
+  L.col_idx = take(rows * p.kcap * 4);
+  L.order = take(rows * 4);
+  L.ctrl = take(spattn::CTRL_WORDS * 4);
+  L.total = off;
+  return L;
+}
+
+Work bind(const Problem& p, const Layout& L, void* ws) {
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  Work w;
+  const bool perm = p.perm != nullptr;
+  w.qp = perm ? reinterpret_cast<__nv_bfloat16*>(b + L.qp) : nullptr;
+  w.kp = perm ? reinterpret_cast<__nv_bfloat16*>(b + L.kp) : nullptr;
+  w.vp = perm ? reinterpret_cast<__nv_bfloat16*>(b + L.vp) : nullptr;
+  w.qbar = reinterpret_cast<float*>(b + L.qbar);
+  w.kbar = reinterpret_cast<float*>(b + L.kbar);
+  w.vbar = reinterpret_cast<float*>(b + L.vbar);
+  w.kbar16 = reinterpret_cast<__nv_bfloat16*>(b + L.kbar16);
+  w.vbar16 = reinterpret_cast<__nv_bfloat16*>(b + L.vbar16);
+  w.counts = reinterpret_cast<int32_t*>(b + L.counts);
+  w.lists = reinterpret_cast<int32_t*>(b + L.lists);
+  w.row_ptr = reinterpret_cast<int32_t*>(b + L.row_ptr);
+  w.col_idx = reinterpret_cast<int32_t*>(b + L.col_idx);
+  w.order = reinterpret_cast<int32_t*>(b + L.order);
+  w.ctrl = reinterpret_cast<int32_t*>(b + L.ctrl);
+  return w;
+}
+
+}  // namespace
+
+struct spattn_plan_s {
+  Problem p;
+  Layout L;
+  int32_t* perm_dev = nullptr;
+};
+
+namespace {
+
+spattn_status_t check_plan(spattn_plan_t plan) {
+  if (!plan) return fail(SPATTN_ERR_INVALID_ARG, "plan is NULL");
+  return SPATTN_OK;
+}
+
+spattn_status_t check_inputs(spattn_plan_t plan, const void* Q, const void* K, const void* V,
+                             const void* ws) {
+  if (spattn_status_t st = check_plan(plan)) return st;
+  if (!Q || !K || !V) return fail(SPATTN_ERR_INVALID_ARG, "Q, K and V must be non-NULL");
+  if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K) |
+       reinterpret_cast<uintptr_t>(V)) & 15)
+    return fail(SPATTN_ERR_INVALID_ARG, "Q, K and V must be 16-byte aligned");
+  if (!ws) return fail(SPATTN_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) & (ALIGN - 1))
+    return fail(SPATTN_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  return SPATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* spattn_last_error(void) { return g_err; }
+
+spattn_status_t spattn_plan(spattn_plan_t* out, int B, int H, int N, int d, int b, float tau,
+                            int kmin, int kmax, int residual, const int32_t* perm_host,
+                            size_t* workspace_bytes) {
+  g_err[0] = 0;
+  if (!out) return fail(SPATTN_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (B < 1 || H < 1 || N < 1) return fail(SPATTN_ERR_INVALID_ARG, "need B, H, N >= 1 (got %d, %d, %d)", B, H, N);
+  if (d != 64 && d != 128) return fail(SPATTN_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
+  if (b != 64 && b != 128) return fail(SPATTN_ERR_UNSUPPORTED, "b must be 64 or 128 (got %d)", b);
+  if (!isfinite(tau)) return fail(SPATTN_ERR_INVALID_ARG, "tau must be finite");
+  if (kmin < 1 || kmax < kmin) return fail(SPATTN_ERR_INVALID_ARG, "need 1 <= kmin <= kmax (got %d, %d)", kmin, kmax);
+  if (residual != 0 && residual != 1) return fail(SPATTN_ERR_INVALID_ARG, "residual must be 0 or 1");
+  const long long nb = (N + (long long)b - 1) / b;
+  if (nb > 2048) return fail(SPATTN_ERR_UNSUPPORTED, "nb = %lld blocks exceeds 2048", nb);
+  if ((long long)B * H * nb > (1LL << 30) || (long long)B * H * (long long)N * d > (1LL << 40))
+    return fail(SPATTN_ERR_UNSUPPORTED, "problem too large");
+  if (perm_host) {
+    std::vector<uint8_t> seen(N, 0);
+    for (int n = 0; n < N; ++n) {
+      const int32_t v = perm_host[n];
+      if (v < 0 || v >= N || seen[v]) return fail(SPATTN_ERR_INVALID_ARG, "perm is not a bijection of [0, N) (entry %d)", n);
+      seen[v] = 1;
+    }
+  }
+  spattn_plan_s* P = new (std::nothrow) spattn_plan_s;
+  if (!P) return fail(SPATTN_ERR_INVALID_ARG, "out of host memory");
+  Problem& p = P->p;
+  p.B = B; p.H = H; p.N = N; p.d = d; p.b = b;
+  p.nb = (int)nb;
+  p.n_last = N - (p.nb - 1) * b;
+  p.kcap = std::min(kmax, p.nb);
+  p.BH = B * H;
+  p.tau = tau; p.kmin = kmin; p.kmax = kmax; p.residual = residual;
+  p.perm = nullptr;
+  if (perm_host) {
+    cudaError_t e = cudaMalloc(&P->perm_dev, sizeof(int32_t) * (size_t)N);
+    if (e != cudaSuccess) { delete P; return cuda_fail(e, "cudaMalloc(perm)"); }
+    e = cudaMemcpy(P->perm_dev, perm_host, sizeof(int32_t) * (size_t)N, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { cudaFree(P->perm_dev); delete P; return cuda_fail(e, "cudaMemcpy(perm)"); }
+    p.perm = P->perm_dev;
+  }
+  P->L = make_layout(p);
+  if (workspace_bytes) *workspace_bytes = P->L.total;
+  *out = P;
+  return SPATTN_OK;
+}
+
+spattn_status_t spattn_plan_destroy(spattn_plan_t plan) {
+  if (!plan) return SPATTN_OK;
+  cudaError_t e = cudaSuccess;
+  if (plan->perm_dev) e = cudaFree(plan->perm_dev);
+  delete plan;
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFree(perm)");
+  return SPATTN_OK;
+}
+
+spattn_status_t spattn_plan_info(spattn_plan_t plan, int* nb, int64_t* col_capacity) {
+  if (spattn_status_t st = check_plan(plan)) return st;
+  if (nb) *nb = plan->p.nb;
+  if (col_capacity) *col_capacity = (int64_t)plan->p.BH * plan->p.nb * plan->p.kcap;
+  return SPATTN_OK;
+}
+
+spattn_status_t spattn_pool(spattn_plan_t plan, const void* Q, const void* K, const void* V,
+                            void* workspace, void* stream) {
+  if (spattn_status_t st = check_inputs(plan, Q, K, V, workspace)) return st;
+  const Work w = bind(plan->p, plan->L, workspace);
+  cudaError_t e = spattn::launch_pool(plan->p, Q, K, V, w, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pool kernel");
+  return SPATTN_OK;
+}
+
+spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, const void* V,
+                             void* workspace, int32_t* row_ptr, int32_t* col_idx, void* stream) {
+  if (spattn_status_t st = check_inputs(plan, Q, K, V, workspace)) return st;
+  const Work w = bind(plan->p, plan->L, workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = spattn::launch_pool(plan->p, Q, K, V, w, s);
+  if (e != cudaSuccess) return cuda_fail(e, "pool kernel");
+  e = spattn::launch_route(plan->p, w, row_ptr, col_idx, s);
+  if (e != cudaSuccess) return cuda_fail(e, "route kernels");
+  return SPATTN_OK;
+}
+
+spattn_status_t spattn_attend(spattn_plan_t plan, const void* Q, const void* K, const void* V,
+                              const int32_t* row_ptr, const int32_t* col_idx, void* O,
+                              void* workspace, void* stream) {
+  if (spattn_status_t st = check_inputs(plan, Q, K, V, workspace)) return st;
+  if (!O) return fail(SPATTN_ERR_INVALID_ARG, "O must be non-NULL");
+  if (reinterpret_cast<uintptr_t>(O) & 15) return fail(SPATTN_ERR_INVALID_ARG, "O must be 16-byte aligned");
+  if ((row_ptr == nullptr) != (col_idx == nullptr))
+    return fail(SPATTN_ERR_INVALID_ARG, "row_ptr and col_idx must both be NULL or both be set");
+  const Work w = bind(plan->p, plan->L, workspace);
+  if (!row_ptr) { row_ptr = w.row_ptr; col_idx = w.col_idx; }
+  cudaError_t e = spattn::launch_attend(plan->p, Q, K, V, row_ptr, col_idx, O, w,
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel");
+  return SPATTN_OK;
+}
+
+spattn_status_t spattn_forward(spattn_plan_t plan, const void* Q, const void* K, const void* V,
+                               void* O, void* workspace, void* stream) {
+  if (spattn_status_t st = spattn_route(plan, Q, K, V, workspace, nullptr, nullptr, stream)) return st;
+  return spattn_attend(plan, Q, K, V, nullptr, nullptr, O, workspace, stream);
+}
+
+spattn_status_t spattn_means(spattn_plan_t plan, const void* workspace, float* Qbar, float* Kbar,
+                             float* Vbar, void* stream) {
+  if (spattn_status_t st = check_plan(plan)) return st;
+  if (!workspace) return fail(SPATTN_ERR_WORKSPACE, "workspace is NULL");
+  const Work w = bind(plan->p, plan->L, const_cast<void*>(workspace));
+  const size_t bytes = (size_t)plan->p.BH * plan->p.nb * plan->p.d * sizeof(float);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const float* src[3] = {w.qbar, w.kbar, w.vbar};
+  float* dst[3] = {Qbar, Kbar, Vbar};
+  for (int t = 0; t < 3; ++t) {
+    if (!dst[t]) continue;
+    cudaError_t e = cudaMemcpyAsync(dst[t], src[t], bytes, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(means)");
+  }
+  return SPATTN_OK;
+}
+
+spattn_status_t spattn_check(spattn_plan_t plan, void* workspace, void* stream) {
+  if (spattn_status_t st = check_plan(plan)) return st;
+  if (!workspace) return fail(SPATTN_ERR_WORKSPACE, "workspace is NULL");
+  const Work w = bind(plan->p, plan->L, workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t h[2] = {0, 0};
+  cudaError_t e = cudaMemcpyAsync(h, w.ctrl, sizeof(h), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  e = cudaMemsetAsync(w.ctrl, 0, sizeof(int32_t) * 2, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+  if (h[0] == spattn::DEV_BAD_INDEX)
+    return fail(SPATTN_ERR_DEVICE, "a CSR block index outside [0, nb) was skipped (work item %d)", h[1]);
+  if (h[0] == spattn::DEV_TIMEOUT)
+    return fail(SPATTN_ERR_TIMEOUT, "a device-side wait gave up (site %d)", h[1]);
+  if (h[0] != 0) return fail(SPATTN_ERR_DEVICE, "device error code %d (aux %d)", h[0], h[1]);
+  return SPATTN_OK;
+}
+
+// ---- 3D Hilbert order (host, no CUDA) ----
+// Skilling's transform, one cell at a time: walk the bit levels from the top,
+// at each level either invert the lower bits of axis 0 or swap them with axis
+// i, then Gray-encode across the axes; the index reads the three transformed
+// words level by level, axis 0 most significant.
+static uint64_t hilbert_key3(uint32_t x[3], int bits) {
+  const uint32_t top = 1u << (bits - 1);
+  for (uint32_t q = top; q > 1; q >>= 1) {
+    const uint32_t low = q - 1;
+    for (int i = 0; i < 3; ++i) {
+      if (x[i] & q) {
+        x[0] ^= low;
+      } else {
+        const uint32_t t = (x[0] ^ x[i]) & low;
+        x[0] ^= t;
+        x[i] ^= t;
+      }
+    }
+  }
+  x[1] ^= x[0];
+  x[2] ^= x[1];
+  uint32_t flip = 0;
+  for (uint32_t q = top; q > 1; q >>= 1)
+    if (x[2] & q) flip ^= q - 1;
+  for (int i = 0; i < 3; ++i) x[i] ^= flip;
+  uint64_t key = 0;
+  for (int level = bits - 1; level >= 0; --level)
+    for (int i = 0; i < 3; ++i) key = (key << 1) | ((x[i] >> level) & 1u);
+  return key;
+}
+
+spattn_status_t spattn_hilbert_perm(int T, int Hs, int W, int32_t* perm_host) {
+  if (T < 1 || Hs < 1 || W < 1) return fail(SPATTN_ERR_INVALID_ARG, "grid sides must be >= 1");
+  if (!perm_host) return fail(SPATTN_ERR_INVALID_ARG, "perm_host is NULL");
+  const long long N = (long long)T * Hs * W;
+  if (N > (1LL << 31) - 1) return fail(SPATTN_ERR_UNSUPPORTED, "grid too large");
+  const int side = std::max(T, std::max(Hs, W));
+  int bits = 1;
+  while ((1 << bits) < side) ++bits;
+  std::vector<uint64_t> key((size_t)N);
+  for (int t = 0; t < T; ++t)
+    for (int h = 0; h < Hs; ++h)
+      for (int w = 0; w < W; ++w) {
+        uint32_t x[3] = {(uint32_t)t, (uint32_t)h, (uint32_t)w};
+        key[((size_t)t * Hs + h) * W + w] = hilbert_key3(x, bits);
+      }
+  std::vector<int32_t> idx((size_t)N);
+  std::iota(idx.begin(), idx.end(), 0);
+  std::stable_sort(idx.begin(), idx.end(), [&](int32_t a, int32_t b) { return key[a] < key[b]; });
+  memcpy(perm_host, idx.data(), sizeof(int32_t) * (size_t)N);
+  return SPATTN_OK;
+}
+
+}  // extern "C"
+
+namespace spattn {
+cudaError_t launch_attend(const Problem& p, const void* Q, const void* K, const void* V,
+                          const int32_t* row_ptr, const int32_t* col_idx, void* O,
+                          const Work& w, cudaStream_t s) {
+  return launch_attend_mma(p, Q, K, V, row_ptr, col_idx, O, w, s);
+}
+}  // namespace spattn

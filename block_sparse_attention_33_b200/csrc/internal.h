@@ -1,0 +1,42 @@
+// Internal launch interface shared by the spattn translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace spattn {
+
+// Problem description derived from a plan (all sizes in elements).
+struct Problem {
+  int B, H, N, d, b, nb, n_last, kcap;
+  int BH;
+  float tau;
+  int kmin, kmax;
+  int residual;
+  const int32_t* perm;  // device, NULL if none
+};
+
+// Device buffers of one workspace (pointers into it).
+struct Work {
+  __nv_bfloat16 *qp, *kp, *vp;  // permuted copies (NULL without perm)
+  float *qbar, *kbar, *vbar;    // fp32 means [BH, nb, d]
+  __nv_bfloat16 *kbar16, *vbar16;  // bf16 means for the residual tiles
+  int32_t* counts;   // [BH*nb] kept count per query block
+  int32_t* lists;    // [BH*nb*kcap] kept blocks, ascending, padded rows
+  int32_t* row_ptr;  // [BH*nb + 1]
+  int32_t* col_idx;  // [BH*nb*kcap]
+  int32_t* order;    // [BH*nb] work order for the attention kernel
+  int32_t* ctrl;     // control block (CTRL_WORDS int32)
+};
+
+cudaError_t launch_pool(const Problem& p, const void* Q, const void* K, const void* V,
+                        const Work& w, cudaStream_t s);
+cudaError_t launch_route(const Problem& p, const Work& w, int32_t* row_ptr_out,
+                         int32_t* col_idx_out, cudaStream_t s);
+cudaError_t launch_attend(const Problem& p, const void* Q, const void* K, const void* V,
+                          const int32_t* row_ptr, const int32_t* col_idx, void* O,
+                          const Work& w, cudaStream_t s);
+
+}  // namespace spattn

@@ -1,0 +1,293 @@
+// Steps a3-a5: proxy logits, block softmax, Top-p selection, CSR of kept blocks.
+//
+// Block importance (PARK page 3.2): p_ij = softmax_j(Qbar_i . Kbar_j / sqrt(d)
+// + ln n_j), the centroid estimate of the block log-mass (PARK D.2).  Blocks
+// are taken in descending p until the cumulative mass reaches tau (PARK 3.2
+// "Top-p"), ties to the lower block index, budget clamped to [kmin, kmax]
+// (Sol-Attn abstract: dynamic but controllable budgets).  The proxy map never
+// leaves shared memory.
+//
+// Selection without a sort: with p >= 0 the float bit pattern orders p, and
+// the mass G(u) = sum of p_j whose bits exceed u is monotone in u.  The kept
+// prefix is {p_j > v} plus the first few blocks with p_j == v (ascending j),
+// where v is the smallest value whose strictly-larger mass is < tau; a binary
+// search over the bit patterns finds v with one warp reduction per step.  The
+// same search on the count #{p_j > u} yields the top-k set when the clamp
+// binds.  Kept blocks are then emitted in ascending j with warp ballots.
+//
+// route_kernel: one CTA per (16 query blocks, head); 8 warps; the proxy tile
+// S[16][nb] is computed with fp32 FMAs (no TF32/BF16: a logit error of 1e-2
+// would move cumulative mass by more than the 1e-4 comparison margin).
+#include "common.cuh"
+#include "internal.h"
+
+namespace spattn {
+namespace {
+
+constexpr int RT_ROWS = 16;      // query blocks per CTA
+constexpr int RT_THREADS = 256;
+
+struct RouteArgs {
+  const float* qbar;
+  const float* kbar;
+  int32_t* counts;
+  int32_t* lists;
+  int nb, b, n_last, kcap, kmin;
+  float tau;
+};
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Mass of the blocks whose probability bits exceed u.
+__device__ __forceinline__ float mass_above(const float* p, int nb, uint32_t u) {
+  float s = 0.f;
+  for (int j = threadIdx.x & 31; j < nb; j += 32) {
+    const float x = p[j];
+    if (__float_as_uint(x) > u) s += x;
+  }
+  return warp_sum(s);
+}
+__device__ __forceinline__ int count_above(const float* p, int nb, uint32_t u) {
+  int c = 0;
+  for (int j = threadIdx.x & 31; j < nb; j += 32) c += (__float_as_uint(p[j]) > u) ? 1 : 0;
+  return warp_sum_i(c);
+}
+__device__ __forceinline__ int count_equal(const float* p, int nb, uint32_t u) {
+  int c = 0;
+  for (int j = threadIdx.x & 31; j < nb; j += 32) c += (__float_as_uint(p[j]) == u) ? 1 : 0;
+  return warp_sum_i(c);
+}
+
+template <int D>
+__global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
+  extern __shared__ __align__(16) float sm[];
+  const int nbp = (a.nb + 31) & ~31;
+  float* Qs = sm;                       // [RT_ROWS][D]
+  float* S = sm + RT_ROWS * D;          // [RT_ROWS][nbp]
+  const int bh = blockIdx.y, i0 = blockIdx.x * RT_ROWS;
+  const int rows = min(RT_ROWS, a.nb - i0);
+  const float* qbar = a.qbar + ((size_t)bh * a.nb + i0) * D;
+  const float* kbar = a.kbar + (size_t)bh * a.nb * D;
+
+  for (int e = threadIdx.x; e < RT_ROWS * D; e += RT_THREADS)
+    Qs[e] = (e / D < rows) ? qbar[e] : 0.f;
+  __syncthreads();
+
+  // ---- proxy logits: thread owns key block j, all 16 query rows ----
+  const float inv_sqrt_d = 1.0f / sqrtf((float)D);
+  for (int j = threadIdx.x; j < a.nb; j += RT_THREADS) {
+    float acc[RT_ROWS];
+#pragma unroll
+    for (int r = 0; r < RT_ROWS; ++r) acc[r] = 0.f;
+    const float4* kr = reinterpret_cast<const float4*>(kbar + (size_t)j * D);
+#pragma unroll 4
+    for (int k4 = 0; k4 < D / 4; ++k4) {
+      const float4 kv = __ldg(kr + k4);
+#pragma unroll
+      for (int r = 0; r < RT_ROWS; ++r) {
+        const float4 q = reinterpret_cast<const float4*>(Qs + r * D)[k4];
+        acc[r] = fmaf(q.x, kv.x, acc[r]);
+        acc[r] = fmaf(q.y, kv.y, acc[r]);
+        acc[r] = fmaf(q.z, kv.z, acc[r]);
+        acc[r] = fmaf(q.w, kv.w, acc[r]);
+      }
+    }
+    const int nj = (j == a.nb - 1) ? a.n_last : a.b;
+    const float lnn = logf((float)nj);
+#pragma unroll
+    for (int r = 0; r < RT_ROWS; ++r) S[r * nbp + j] = fmaf(acc[r], inv_sqrt_d, lnn);
+  }
+  __syncthreads();
+
+  // ---- per query block: softmax, selection, emission (one warp per row) ----
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int r = warp; r < rows; r += RT_THREADS / 32) {
+    float* p = S + r * nbp;
+    float mx = -INFINITY;
+    for (int j = lane; j < a.nb; j += 32) mx = fmaxf(mx, p[j]);
+    mx = warp_max(mx);
+    float sum = 0.f;
+    for (int j = lane; j < a.nb; j += 32) {
+      const float e = expf(p[j] - mx);
+      p[j] = e;
+      sum += e;
+    }
+    sum = warp_sum(sum);
+    for (int j = lane; j < a.nb; j += 32) p[j] = p[j] / sum;
+    __syncwarp();
+
+    // kept set = {bits(p) > thr} + first `ties` blocks with bits(p) == thr
+    uint32_t thr = 0;
+    int ties = 0, kstar = 0;
+    bool by_mass = false;
+    if (a.tau >= 1.0f) {
+      kstar = a.nb;               // tau >= 1 keeps every block
+    } else if (a.tau > 0.0f) {
+      uint32_t lo = 0, hi = 0x3F800000u;  // p <= 1, so nothing is above hi
+      while (lo < hi) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (mass_above(p, a.nb, mid) < a.tau) hi = mid; else lo = mid + 1;
+      }
+      thr = lo;
+      const float g = mass_above(p, a.nb, thr);
+      const int gt = count_above(p, a.nb, thr);
+      const int eq = count_equal(p, a.nb, thr);
+      const float v = __uint_as_float(thr);
+      float e = g;
+      int keep = 0;
+      while (keep < eq && e < a.tau) { e += v; ++keep; }
+      ties = keep;
+      kstar = gt + keep;
+      by_mass = true;
+    }
+    const int k = min(max(kstar, a.kmin), a.kcap);
+    const bool all = (k >= a.nb);
+    if (!all && !(by_mass && k == kstar)) {
+      // the clamp binds (or tau <= 0): top-k in (p desc, j asc) order
+      uint32_t lo = 0, hi = 0x3F800000u;
+      while (lo < hi) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (count_above(p, a.nb, mid) < k) hi = mid; else lo = mid + 1;
+      }
+      thr = lo;
+      ties = k - count_above(p, a.nb, thr);
+    }
+    const int row = bh * a.nb + i0 + r;
+    int32_t* out = a.lists + (size_t)row * a.kcap;
+    int base = 0, seen_eq = 0;
+    for (int j0 = 0; j0 < a.nb; j0 += 32) {
+      const int j = j0 + lane;
+      const bool valid = j < a.nb;
+      const uint32_t u = valid ? __float_as_uint(p[j]) : 0u;
+      const bool eq = valid && !all && u == thr;
+      const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+      const int eq_rank = seen_eq + __popc(eqm & ((1u << lane) - 1u));
+      seen_eq += __popc(eqm);
+      const bool keep = valid && (all || u > thr || (eq && eq_rank < ties));
+      const unsigned km = __ballot_sync(0xffffffffu, keep);
+      if (keep) out[base + __popc(km & ((1u << lane) - 1u))] = j;
+      base += __popc(km);
+    }
+    if (lane == 0) a.counts[row] = k;
+  }
+}
+
+// Exclusive scan of the per-row counts into row_ptr (single CTA), total in
+// ctrl[CTRL_NNZ]; also a counting sort of the rows by descending budget, so
+// that the attention grid starts with the longest rows.
+constexpr int SCAN_THREADS = 1024;
+
+__global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(const int32_t* counts, int rows,
+                                                            int kcap, int32_t* row_ptr,
+                                                            int32_t* order, int32_t* ctrl) {
+  __shared__ int part[SCAN_THREADS];
+  extern __shared__ int hist[];  // [kcap + 1]
+  const int per = (rows + SCAN_THREADS - 1) / SCAN_THREADS;
+  const int lo = threadIdx.x * per, hi = min(rows, lo + per);
+  for (int q = threadIdx.x; q <= kcap; q += SCAN_THREADS) hist[q] = 0;
+  int s = 0;
+  for (int q = lo; q < hi; ++q) s += counts[q];
+  part[threadIdx.x] = s;
+  __syncthreads();
+  for (int q = lo; q < hi; ++q) atomicAdd(&hist[min(counts[q], kcap)], 1);
+  // Hillis-Steele inclusive scan over the thread partials
+  for (int off = 1; off < SCAN_THREADS; off <<= 1) {
+    const int v = threadIdx.x >= off ? part[threadIdx.x - off] : 0;
+    __syncthreads();
+    part[threadIdx.x] += v;
+    __syncthreads();
+  }
+  int run = threadIdx.x ? part[threadIdx.x - 1] : 0;
+  for (int q = lo; q < hi; ++q) {
+    row_ptr[q] = run;
+    run += counts[q];
+  }
+  if (threadIdx.x == SCAN_THREADS - 1) {
+    row_ptr[rows] = part[SCAN_THREADS - 1];
+    ctrl[CTRL_NNZ] = part[SCAN_THREADS - 1];
+  }
+  __syncthreads();
+  // descending-budget start offsets (serial over at most kcap+1 bins)
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int q = kcap; q >= 0; --q) {
+      const int c = hist[q];
+      hist[q] = acc;
+      acc += c;
+    }
+  }
+  __syncthreads();
+  for (int q = lo; q < hi; ++q) order[atomicAdd(&hist[min(counts[q], kcap)], 1)] = q;
+}
+
+// Copy the padded per-row lists into the compact CSR (one warp per row).
+__global__ void __launch_bounds__(256) compact_kernel(const int32_t* counts, const int32_t* lists,
+                                                      const int32_t* row_ptr, int rows, int kcap,
+                                                      int32_t* col_idx, int32_t* row_ptr_out,
+                                                      int32_t* col_idx_out) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row < rows) {
+    const int c = counts[row], o = row_ptr[row];
+    const int32_t* src = lists + (size_t)row * kcap;
+    for (int q = lane; q < c; q += 32) {
+      const int32_t v = src[q];
+      col_idx[o + q] = v;
+      if (col_idx_out) col_idx_out[o + q] = v;
+    }
+    if (row_ptr_out && lane == 0) {
+      row_ptr_out[row] = o;
+      if (row == rows - 1) row_ptr_out[rows] = o + c;
+    }
+  }
+}
+
+}  // namespace
+
+size_t route_smem_bytes(int d, int nb) {
+  const int nbp = (nb + 31) & ~31;
+  return (size_t)RT_ROWS * (d + nbp) * sizeof(float);
+}
+
+cudaError_t launch_route(const Problem& p, const Work& w, int32_t* row_ptr_out,
+                         int32_t* col_idx_out, cudaStream_t s) {
+  RouteArgs a;
+  a.qbar = w.qbar; a.kbar = w.kbar; a.counts = w.counts; a.lists = w.lists;
+  a.nb = p.nb; a.b = p.b; a.n_last = p.n_last; a.kcap = p.kcap; a.kmin = p.kmin;
+  a.tau = p.tau;
+  const size_t smem = route_smem_bytes(p.d, p.nb);
+  dim3 grid((p.nb + RT_ROWS - 1) / RT_ROWS, p.BH);
+  cudaError_t e;
+  if (p.d == 128) {
+    e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    route_kernel<128><<<grid, RT_THREADS, smem, s>>>(a);
+  } else {
+    e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    route_kernel<64><<<grid, RT_THREADS, smem, s>>>(a);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int rows = p.BH * p.nb;
+  scan_kernel<<<1, SCAN_THREADS, (p.kcap + 1) * sizeof(int), s>>>(w.counts, rows, p.kcap,
+                                                                  w.row_ptr, w.order, w.ctrl);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  compact_kernel<<<(rows + 7) / 8, 256, 0, s>>>(w.counts, w.lists, w.row_ptr, rows, p.kcap,
+                                                w.col_idx, row_ptr_out, col_idx_out);
+  return cudaGetLastError();
+}
+
+}  // namespace spattn

@@ -1,0 +1,148 @@
+/*
+ * spattn -- routed block-sparse attention with proxy residual, for NVIDIA
+ * B200 (sm_100a).  C ABI.
+ *
+ * What the library computes (one attention call; pages: PARK "Accurate
+ * Block Retrieval for Sparse Attention in Video Diffusion Transformers",
+ * sections 3.1-3.2 and D.2; Sol-Attn abstract; DFSAttn abstract):
+ *
+ *   Q, K, V: bf16 [B, H, N, d] (row-major, d contiguous).  With a token
+ *   permutation perm, tokens are first gathered, Xp[n] = X[perm[n]].
+ *   Tokens are cut into nb = ceil(N / b) blocks; block j holds n_j tokens
+ *   (b, except a possibly partial last block).  Query blocks use the same
+ *   partition.
+ *
+ *   1. block means Qbar_i, Kbar_j, Vbar_j in fp32;
+ *   2. proxy logits s_ij = Qbar_i . Kbar_j / sqrt(d) + ln n_j and
+ *      p_ij = softmax_j(s_ij) (PARK 3.2 block importance; the ln n_j term
+ *      makes s_ij the Jensen lower bound of PARK D.2);
+ *   3. per query block i, blocks in descending p (ties: lower j) and the
+ *      shortest prefix whose cumulative mass reaches tau is kept, budget
+ *      clamped to [kmin, min(kmax, nb)]; tau >= 1 keeps every block
+ *      (PARK 3.2 "Top-p"; Sol-Attn dynamic budgets);
+ *   4. each query token q of block i runs one softmax over the exact tokens
+ *      of its kept blocks; with residual != 0 every dropped block j adds one
+ *      pseudo-key with logit q . Kbar_j / sqrt(d) + ln n_j and value Vbar_j
+ *      (Sol-Attn: reuse the proxy scores of unselected blocks);
+ *   5. the output is scattered back, O[perm[n]] = Op[n], bf16.
+ *
+ * Conventions for every call:
+ *   - Pointers named *_host are host memory; every other data pointer is
+ *     device memory of the current CUDA device.  The caller owns all of
+ *     them; the library keeps no pointer past the call that received it.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Device
+ *     work is enqueued on it and the call returns without waiting;
+ *     argument errors are reported synchronously before anything is
+ *     enqueued.
+ *   - Every call returns a spattn_status_t; spattn_last_error() gives a
+ *     human-readable message for the calling thread's last failure.  No
+ *     C++ exception crosses this boundary.
+ *   - Supported: d in {64, 128}; b in {64, 128}; 1 <= N; nb <= 2048;
+ *     1 <= kmin <= kmax (kmax > nb is clamped to nb); tau finite.
+ */
+#ifndef SPATTN_H_
+#define SPATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SPATTN_OK = 0,
+  SPATTN_ERR_INVALID_ARG = 1,  /* bad shape, knob, pointer or permutation */
+  SPATTN_ERR_UNSUPPORTED = 2,  /* valid but outside the supported range  */
+  SPATTN_ERR_WORKSPACE = 3,    /* workspace missing or too small          */
+  SPATTN_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed       */
+  SPATTN_ERR_TIMEOUT = 5,      /* a device-side bounded wait gave up      */
+  SPATTN_ERR_DEVICE = 6        /* a kernel flagged bad data (e.g. a CSR
+                                  block index out of range); see
+                                  spattn_check                             */
+} spattn_status_t;
+
+typedef struct spattn_plan_s* spattn_plan_t;
+
+/* Create a plan for one problem shape and set of routing knobs.
+ *   B, H, N, d, b       shapes (see above);
+ *   tau, kmin, kmax     Top-p threshold and budget clamp;
+ *   residual            0: dropped blocks are skipped; 1: pseudo-keys;
+ *   perm_host           NULL, or N int32 forming a bijection of [0, N):
+ *                       perm[new] = old.  The plan copies it to device
+ *                       memory it owns (this needs a current CUDA device);
+ *   workspace_bytes     out: bytes of device workspace the route/attend/
+ *                       forward calls need (256-byte aligned base).
+ * Validation happens before any CUDA call.  The plan is immutable and may
+ * be shared by threads; one workspace must not be used by two calls that
+ * overlap on the device. */
+spattn_status_t spattn_plan(spattn_plan_t* out, int B, int H, int N, int d, int b,
+                            float tau, int kmin, int kmax, int residual,
+                            const int32_t* perm_host, size_t* workspace_bytes);
+
+/* Release a plan (and its device copy of the permutation). NULL is a no-op. */
+spattn_status_t spattn_plan_destroy(spattn_plan_t plan);
+
+/* Number of query/key blocks nb and the capacity (B*H*nb*min(kmax, nb)) a
+ * caller-provided col_idx buffer must have. */
+spattn_status_t spattn_plan_info(spattn_plan_t plan, int* nb, int64_t* col_capacity);
+
+/* Steps a1-a2: gather (if the plan has a permutation) and pool.  Writes the
+ * permuted copies and the fp32 block means Qbar, Kbar, Vbar into the
+ * workspace.  Q, K, V: bf16 [B, H, N, d] device. */
+spattn_status_t spattn_pool(spattn_plan_t plan, const void* Q, const void* K, const void* V,
+                            void* workspace, void* stream);
+
+/* Steps a1-a5: spattn_pool, then proxy scoring, Top-p selection and the CSR
+ * of kept blocks.
+ *   row_ptr  NULL or int32 [B*H*nb + 1], rows ordered (batch, head, block i);
+ *   col_idx  NULL or int32 [col capacity], kept block indices j in [0, nb),
+ *            ascending within a row.
+ * The CSR is always also kept in the workspace for a following attend. */
+spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, const void* V,
+                             void* workspace, int32_t* row_ptr, int32_t* col_idx,
+                             void* stream);
+
+/* Steps a6-a8: routed attention (+ residual pseudo-keys) and the scatter
+ * of the output, using the permuted copies and block means that the last
+ * spattn_pool / spattn_route left in this workspace for the same inputs.
+ *   row_ptr, col_idx  NULL to use the workspace CSR of the last route, or a
+ *                     caller CSR in the layout above (device).  Block
+ *                     indices outside [0, nb) are skipped and flagged
+ *                     (SPATTN_ERR_DEVICE from spattn_check).
+ *   O                 bf16 [B, H, N, d] device, written in the original
+ *                     token order. */
+spattn_status_t spattn_attend(spattn_plan_t plan, const void* Q, const void* K, const void* V,
+                              const int32_t* row_ptr, const int32_t* col_idx, void* O,
+                              void* workspace, void* stream);
+
+/* The whole path: spattn_route (CSR in the workspace only) + spattn_attend. */
+spattn_status_t spattn_forward(spattn_plan_t plan, const void* Q, const void* K, const void* V,
+                               void* O, void* workspace, void* stream);
+
+/* Copy the fp32 block means [B, H, nb, d] left in the workspace by the last
+ * pool/route into caller device buffers (any may be NULL). */
+spattn_status_t spattn_means(spattn_plan_t plan, const void* workspace, float* Qbar,
+                             float* Kbar, float* Vbar, void* stream);
+
+/* Synchronise `stream` and report the device error word of this workspace:
+ * SPATTN_OK, SPATTN_ERR_DEVICE or SPATTN_ERR_TIMEOUT.  Clears the word. */
+spattn_status_t spattn_check(spattn_plan_t plan, void* workspace, void* stream);
+
+/* Host helper (no CUDA): perm[new] = old ordering the tokens of a T x Hs x W
+ * latent grid (row-major token order n = (t*Hs + h)*W + w) along a 3D
+ * Hilbert curve (DFSAttn abstract: Hilbert curve-based token reordering).
+ * The curve is J. Skilling's ("Programming the Hilbert curve", AIP Conf.
+ * Proc. 707, 2004) on the smallest power-of-two cube covering the grid,
+ * axes (t, h, w); tokens are stably sorted by curve index.  perm_host must
+ * hold T*Hs*W int32. */
+spattn_status_t spattn_hilbert_perm(int T, int Hs, int W, int32_t* perm_host);
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+const char* spattn_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPATTN_H_ */

@@ -161,12 +161,12 @@ def route_rows(p: np.ndarray, tau: float, kmin: int, kmax: int):
             marg.update(np.nonzero(np.abs(E_rank - tau) < MASS_MARGIN)[0].tolist())
         if 0 < k < nb:
             p_in, p_out = sorted_p[k - 1], sorted_p[k]
-            for r in range(k):          # kept blocks tying with the first dropped
-                if sorted_p[r] - p_out <= TIE_MARGIN * sorted_p[r]:
-                    marg.add(int(order[r]))
-            for r in range(k, nb):      # dropped blocks tying with the last kept
-                if p_in - sorted_p[r] <= TIE_MARGIN * p_in:
-                    marg.add(int(order[r]))
+            # kept blocks tying with the first dropped one
+            r_in = np.nonzero(sorted_p[:k] - p_out <= TIE_MARGIN * sorted_p[:k])[0]
+            # dropped blocks tying with the last kept one
+            r_out = k + np.nonzero(p_in - sorted_p[k:] <= TIE_MARGIN * p_in)[0]
+            marg.update(order[r_in].tolist())
+            marg.update(order[r_out].tolist())
         marginal.append(np.array(sorted(marg), dtype=np.int64))
     return {"kept": kept, "k": ks, "marginal": marginal, "E": E_all}
 

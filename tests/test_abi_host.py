@@ -1,0 +1,113 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol the header declares, validates arguments before touching CUDA,
+sizes workspaces, and builds the same Hilbert order as the oracle."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import block_sparse_attention_33_b200 as sp
+import oracle
+from workloads import get_config
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from block_sparse_attention_33_b200 import build
+    build.build()
+    return sp.lib()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "spattn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(spattn_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = header_functions()
+    assert set(names) == set(sp.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def plan_status(*args, perm=None):
+    h = ctypes.c_void_p()
+    ws = ctypes.c_size_t()
+    p = None
+    if perm is not None:
+        perm = np.ascontiguousarray(perm, dtype=np.int32)
+        p = perm.ctypes.data
+    st = sp.lib().spattn_plan(ctypes.byref(h), *args, p, ctypes.byref(ws))
+    return st, h.value, ws.value
+
+
+@pytest.mark.parametrize("args,code", [
+    ((0, 1, 64, 64, 64, 0.9, 1, 4, 1), sp.ERR_INVALID_ARG),      # B = 0
+    ((1, 1, 0, 64, 64, 0.9, 1, 4, 1), sp.ERR_INVALID_ARG),       # N = 0
+    ((1, 1, 64, 96, 64, 0.9, 1, 4, 1), sp.ERR_UNSUPPORTED),      # d = 96
+    ((1, 1, 64, 64, 32, 0.9, 1, 4, 1), sp.ERR_UNSUPPORTED),      # b = 32
+    ((1, 1, 64, 64, 64, float("nan"), 1, 4, 1), sp.ERR_INVALID_ARG),
+    ((1, 1, 64, 64, 64, float("inf"), 1, 4, 1), sp.ERR_INVALID_ARG),
+    ((1, 1, 64, 64, 64, 0.9, 0, 4, 1), sp.ERR_INVALID_ARG),      # kmin = 0
+    ((1, 1, 64, 64, 64, 0.9, 5, 4, 1), sp.ERR_INVALID_ARG),      # kmin > kmax
+    ((1, 1, 64, 64, 64, 0.9, 1, 4, 2), sp.ERR_INVALID_ARG),      # residual = 2
+    ((1, 1, 2049 * 64, 64, 64, 0.9, 1, 4, 1), sp.ERR_UNSUPPORTED),  # nb > 2048
+])
+def test_plan_rejects_bad_arguments(L, args, code):
+    st, h, _ = plan_status(*args)
+    assert st == code and not h
+    assert L.spattn_last_error().decode()
+
+
+def test_plan_rejects_non_bijective_perm(L):
+    perm = np.arange(100)
+    perm[5] = 6
+    st, h, _ = plan_status(1, 1, 100, 64, 64, 0.9, 1, 4, 1, perm=perm)
+    assert st == sp.ERR_INVALID_ARG and "bijection" in L.spattn_last_error().decode()
+    st, h, _ = plan_status(1, 1, 100, 64, 64, 0.9, 1, 4, 1, perm=np.arange(1, 101))
+    assert st == sp.ERR_INVALID_ARG
+
+
+def test_plan_without_perm_needs_no_cuda_and_sizes_workspace(L):
+    w = get_config("wan")
+    st, h, ws = plan_status(w.B, w.H, w.N, w.d, w.b, w.tau, w.kmin, w.kmax, w.residual)
+    assert st == sp.OK and h
+    nb, cap = sp.spattn_plan_info(h)
+    assert nb == 256 and cap == w.H * 256 * 256
+    # means (3 x fp32 + 2 x bf16) + CSR + lists dominate; no token copies
+    cen = w.H * nb * w.d
+    assert ws >= cen * (3 * 4 + 2 * 2) + 2 * cap * 4
+    assert ws < cen * (3 * 4 + 2 * 2) + 2 * cap * 4 + (1 << 20)
+    assert ws % 256 == 0
+    sp.spattn_plan_destroy(h)
+
+
+def test_calls_reject_null_arguments(L):
+    st, h, ws = plan_status(1, 1, 256, 64, 64, 0.9, 1, 4, 1)
+    assert st == sp.OK
+    f = L.spattn_forward
+    assert f(None, 16, 16, 16, 16, 256, None) == sp.ERR_INVALID_ARG
+    assert f(h, None, 16, 16, 16, 256, None) == sp.ERR_INVALID_ARG
+    assert f(h, 16, 16, 16, 16, None, None) == sp.ERR_WORKSPACE
+    assert f(h, 16, 16, 16, 16, 257, None) == sp.ERR_WORKSPACE      # misaligned workspace
+    assert f(h, 8, 16, 16, 16, 256, None) == sp.ERR_INVALID_ARG     # misaligned Q
+    assert L.spattn_attend(h, 16, 16, 16, 16, None, 16, 256, None) == sp.ERR_INVALID_ARG
+    assert L.spattn_attend(h, 16, 16, 16, None, None, None, 256, None) == sp.ERR_INVALID_ARG
+    sp.spattn_plan_destroy(h)
+    assert L.spattn_plan_destroy(None) == sp.OK
+
+
+@pytest.mark.parametrize("grid", [(4, 16, 16), (21, 30, 52), (1, 1, 5), (3, 1, 7), (8, 8, 8)])
+def test_library_hilbert_matches_oracle(L, grid):
+    assert np.array_equal(sp.spattn_hilbert_perm(*grid), oracle.hilbert_perm(grid))
+
+
+def test_hilbert_rejects_bad_grid(L):
+    buf = np.empty(4, np.int32)
+    assert L.spattn_hilbert_perm(0, 2, 2, buf.ctypes.data) == sp.ERR_INVALID_ARG
+    assert L.spattn_hilbert_perm(2, 2, 1, None) == sp.ERR_INVALID_ARG
