@@ -1,5 +1,6 @@
 // C ABI of libspattn: plans, workspace layout, argument checks, dispatch.
 #include <math.h>
+#include <stdlib.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -17,6 +18,10 @@ namespace spattn {
 cudaError_t launch_attend_mma(const Problem& p, const void* Q, const void* K, const void* V,
                               const int32_t* row_ptr, const int32_t* col_idx, void* O,
                               const Work& w, cudaStream_t s);
+cudaError_t launch_attend_tc(const Problem& p, const void* Q, const void* K, const void* V,
+                             const int32_t* row_ptr, const int32_t* col_idx, void* O,
+                             const Work& w, cudaStream_t s);
+bool attend_tc_supported(const Problem& p);
 }  // namespace spattn
 
 using spattn::Problem;
@@ -162,6 +167,13 @@ spattn_status_t spattn_plan(spattn_plan_t* out, int B, int H, int N, int d, int 
   p.BH = B * H;
   p.tau = tau; p.kmin = kmin; p.kmax = kmax; p.residual = residual;
   p.perm = nullptr;
+  {
+    // tcgen05/TMEM kernel for 128-token blocks; the warp-MMA kernel serves
+    // b = 64 and, with SPATTN_ATTN=mma in the environment when the plan is
+    // made, any shape (used to cross-check the two GPU paths).
+    const char* env = getenv("SPATTN_ATTN");
+    p.use_tc = spattn::attend_tc_supported(p) && !(env && strcmp(env, "mma") == 0);
+  }
   if (perm_host) {
     cudaError_t e = cudaMalloc(&P->perm_dev, sizeof(int32_t) * (size_t)N);
     if (e != cudaSuccess) { delete P; return cuda_fail(e, "cudaMalloc(perm)"); }
@@ -195,7 +207,10 @@ spattn_status_t spattn_pool(spattn_plan_t plan, const void* Q, const void* K, co
                             void* workspace, void* stream) {
   if (spattn_status_t st = check_inputs(plan, Q, K, V, workspace)) return st;
   const Work w = bind(plan->p, plan->L, workspace);
-  cudaError_t e = spattn::launch_pool(plan->p, Q, K, V, w, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(w.ctrl, 0, spattn::CTRL_WORDS * sizeof(int32_t), s);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the control block");
+  e = spattn::launch_pool(plan->p, Q, K, V, w, s);
   if (e != cudaSuccess) return cuda_fail(e, "pool kernel");
   return SPATTN_OK;
 }
@@ -205,7 +220,9 @@ spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, c
   if (spattn_status_t st = check_inputs(plan, Q, K, V, workspace)) return st;
   const Work w = bind(plan->p, plan->L, workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = spattn::launch_pool(plan->p, Q, K, V, w, s);
+  cudaError_t e = cudaMemsetAsync(w.ctrl, 0, spattn::CTRL_WORDS * sizeof(int32_t), s);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the control block");
+  e = spattn::launch_pool(plan->p, Q, K, V, w, s);
   if (e != cudaSuccess) return cuda_fail(e, "pool kernel");
   e = spattn::launch_route(plan->p, w, row_ptr, col_idx, s);
   if (e != cudaSuccess) return cuda_fail(e, "route kernels");
@@ -330,6 +347,7 @@ namespace spattn {
 cudaError_t launch_attend(const Problem& p, const void* Q, const void* K, const void* V,
                           const int32_t* row_ptr, const int32_t* col_idx, void* O,
                           const Work& w, cudaStream_t s) {
+  if (p.use_tc) return launch_attend_tc(p, Q, K, V, row_ptr, col_idx, O, w, s);
   return launch_attend_mma(p, Q, K, V, row_ptr, col_idx, O, w, s);
 }
 }  // namespace spattn

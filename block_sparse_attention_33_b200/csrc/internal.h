@@ -15,6 +15,7 @@ struct Problem {
   float tau;
   int kmin, kmax;
   int residual;
+  int use_tc;           // attention on the tcgen05 kernel (else warp MMA)
   const int32_t* perm;  // device, NULL if none
 };
 
