@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: 
 
 EXPORTS = ("spattn_plan", "spattn_plan_destroy", "spattn_plan_info", "spattn_pool",
            "spattn_route", "spattn_attend", "spattn_forward", "spattn_means", "spattn_check",
-           "spattn_hilbert_perm", "spattn_last_error")
+           "spattn_hilbert_perm", "spattn_route_static", "spattn_last_error")
 
 
 class SpAttnError(RuntimeError):
@@ -56,6 +56,7 @@ def lib():
         "spattn_means": [P, P, P, P, P, P],
         "spattn_check": [P, P, P],
         "spattn_hilbert_perm": [I, I, I, P],
+        "spattn_route_static": [I, I, I, I, I, F, I, I, P, P, P, P, P, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -157,6 +158,15 @@ def spattn_hilbert_perm(T, Hs, W):
     out = np.empty(T * Hs * W, dtype=np.int32)
     _check(lib().spattn_hilbert_perm(T, Hs, W, out.ctypes.data))
     return out
+
+
+def spattn_route_static(B, H, N, d, b, tau, kmin, kmax, Q, K, row_ptr, col_idx, perm=None,
+                        stream=None):
+    """Routing with no device allocation (scratch in the library's static
+    device array); same CSR as spattn_route.  perm: None or a device int32
+    tensor of N entries."""
+    _check(lib().spattn_route_static(B, H, N, d, b, float(tau), kmin, kmax, _ptr(perm), _ptr(Q),
+                                     _ptr(K), _ptr(row_ptr), _ptr(col_idx), _stream(stream)))
 
 
 class Plan:

@@ -101,6 +101,10 @@ Work bind(const Problem& p, const Layout& L, void* ws) {
 
 }  // namespace
 
+namespace spattn {
+void record_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+}  // namespace spattn
+
 struct spattn_plan_s {
   Problem p;
   Layout L;

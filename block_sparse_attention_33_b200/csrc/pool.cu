@@ -1,4 +1,4 @@
-// Steps a1-a2: token gather (optional permutation) fused with block-mean pooling.
+// Token gather (optional permutation) fused with block-mean pooling.
 //
 // Blocks are represented by the mean of their tokens (PARK page, abstract and
 // section 4: "averaged representations of query and key blocks").  With a
@@ -99,6 +99,25 @@ cudaError_t launch_pool(const Problem& p, const void* Q, const void* K, const vo
   a.perm = p.perm;
   a.N = p.N; a.b = p.b; a.nb = p.nb; a.n_last = p.n_last;
   dim3 grid(p.nb, p.BH, 3);
+  if (p.d == 128) pool_kernel<128><<<grid, 256, 0, s>>>(a);
+  else pool_kernel<64><<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+// Means of Q and K only (grid z = 2), no bf16 copies and no permuted copies:
+// what the routing step needs, for callers that keep no other scratch.
+cudaError_t launch_pool_qk(const Problem& p, const void* Q, const void* K, float* qbar,
+                           float* kbar, cudaStream_t s) {
+  PoolArgs a;
+  a.X[0] = static_cast<const __nv_bfloat16*>(Q);
+  a.X[1] = static_cast<const __nv_bfloat16*>(K);
+  a.X[2] = nullptr;
+  a.Xp[0] = a.Xp[1] = a.Xp[2] = nullptr;
+  a.bar[0] = qbar; a.bar[1] = kbar; a.bar[2] = nullptr;
+  a.bar16[0] = a.bar16[1] = a.bar16[2] = nullptr;
+  a.perm = p.perm;
+  a.N = p.N; a.b = p.b; a.nb = p.nb; a.n_last = p.n_last;
+  dim3 grid(p.nb, p.BH, 2);
   if (p.d == 128) pool_kernel<128><<<grid, 256, 0, s>>>(a);
   else pool_kernel<64><<<grid, 256, 0, s>>>(a);
   return cudaGetLastError();

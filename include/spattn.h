@@ -87,13 +87,13 @@ spattn_status_t spattn_plan_destroy(spattn_plan_t plan);
  * caller-provided col_idx buffer must have. */
 spattn_status_t spattn_plan_info(spattn_plan_t plan, int* nb, int64_t* col_capacity);
 
-/* Steps a1-a2: gather (if the plan has a permutation) and pool.  Writes the
+/* Gather (if the plan has a permutation) and pool.  Writes the
  * permuted copies and the fp32 block means Qbar, Kbar, Vbar into the
  * workspace.  Q, K, V: bf16 [B, H, N, d] device. */
 spattn_status_t spattn_pool(spattn_plan_t plan, const void* Q, const void* K, const void* V,
                             void* workspace, void* stream);
 
-/* Steps a1-a5: spattn_pool, then proxy scoring, Top-p selection and the CSR
+/* spattn_pool, then proxy scoring, Top-p selection and the CSR
  * of kept blocks.
  *   row_ptr  NULL or int32 [B*H*nb + 1], rows ordered (batch, head, block i);
  *   col_idx  NULL or int32 [col capacity], kept block indices j in [0, nb),
@@ -103,7 +103,7 @@ spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, c
                              void* workspace, int32_t* row_ptr, int32_t* col_idx,
                              void* stream);
 
-/* Steps a6-a8: routed attention (+ residual pseudo-keys) and the scatter
+/* Routed attention (+ residual pseudo-keys) and the scatter
  * of the output, using the permuted copies and block means that the last
  * spattn_pool / spattn_route left in this workspace for the same inputs.
  *   row_ptr, col_idx  NULL to use the workspace CSR of the last route, or a
@@ -137,6 +137,37 @@ spattn_status_t spattn_check(spattn_plan_t plan, void* workspace, void* stream);
  * axes (t, h, w); tokens are stably sorted by curve index.  perm_host must
  * hold T*Hs*W int32. */
 spattn_status_t spattn_hilbert_perm(int T, int Hs, int W, int32_t* perm_host);
+
+/* Routing without any device allocation (pooling of Q and K, scoring,
+ * selection and CSR; no permuted copies).
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot call cudaMalloc: code whose device memory belongs to another
+ * allocator that forbids side allocations, plug-ins that are handed only
+ * their inputs and outputs, and loops that must not pay cudaMalloc's implicit
+ * device synchronisation.  It computes the same CSR as spattn_route for the
+ * same shape and knobs (same kernels, bit-identical result), without a plan
+ * or workspace:
+ *   B, H, N, d, b, tau, kmin, kmax   as for spattn_plan;
+ *   perm     NULL, or a DEVICE array of N int32 (perm[new] = old), which the
+ *            caller guarantees to be a bijection (it is not checked here);
+ *   Q, K     bf16 [B, H, N, d] device (V is not needed for routing);
+ *   row_ptr  int32 [B*H*nb + 1] device, col_idx int32 [B*H*nb*min(kmax, nb)]
+ *            device: the CSR, as written by spattn_route.
+ * Scratch lives in one file-scope device array of
+ * SPATTN_ROUTE_STATIC_SCRATCH_BYTES, held by every GPU that loads the library
+ * until the process exits.  A problem whose scratch (2*B*H*nb*d*4 bytes of
+ * means + B*H*nb*(min(kmax,nb) + 2)*4 bytes of lists, each rounded up to 256)
+ * exceeds it is rejected with SPATTN_ERR_UNSUPPORTED before anything runs.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  Every call shares the one array: calls that
+ * overlap on the GPU (other streams or host threads) race and must be
+ * serialised by the caller.  No cudaMalloc, cudaFree or allocating library
+ * routine is called. */
+#define SPATTN_ROUTE_STATIC_SCRATCH_BYTES (32u << 20)
+spattn_status_t spattn_route_static(int B, int H, int N, int d, int b, float tau, int kmin,
+                                    int kmax, const int32_t* perm, const void* Q, const void* K,
+                                    int32_t* row_ptr, int32_t* col_idx, void* stream);
 
 /* Message for the calling thread's last non-OK status ("" if none). */
 const char* spattn_last_error(void);
