@@ -47,6 +47,8 @@ def parse_args():
                     choices=["tiny", "medium", "wan", "hunyuan", "stress"])
     ap.add_argument("--tau", type=float, default=None)
     ap.add_argument("--residual", type=int, default=None)
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the number of heads (smaller profiling captures)")
     ap.add_argument("--no-dense", action="store_true", help="skip the tau = 1 comparison run")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -72,6 +74,8 @@ def workload_from_args(args, rank=0):
         ov["tau"] = args.tau
     if args.residual is not None:
         ov["residual"] = args.residual
+    if args.heads is not None:
+        ov["H"] = args.heads
     w = get_config(args.workload, **ov)
     if rank:
         w = w.with_(seed=w.seed + 1000 * rank)   # independent replica per rank

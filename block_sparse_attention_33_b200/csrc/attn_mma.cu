@@ -1,4 +1,4 @@
-// Steps a6-a8 on the legacy warp-MMA path (mma.sync m16n8k16, bf16 -> fp32).
+// Routed attention on the legacy warp-MMA path (mma.sync m16n8k16, bf16 -> fp32).
 //
 // This is the simple, portable form of the routed attention: it is kept as
 // the baseline the tcgen05 kernel is measured against and as a second,

@@ -1,4 +1,4 @@
-// Steps a6-a8 on Blackwell tensor cores: routed block-sparse attention with
+// Routed block-sparse attention on Blackwell tensor cores, with
 // the residual pseudo-keys folded into the same online softmax.
 //
 // One CTA per work item (head bh, query block i of 128 tokens); items are

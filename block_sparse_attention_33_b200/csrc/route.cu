@@ -1,4 +1,4 @@
-// Steps a3-a5: proxy logits, block softmax, Top-p selection, CSR of kept blocks.
+// Proxy logits, block softmax, Top-p selection, CSR of kept blocks.
 //
 // Block importance (PARK page 3.2): p_ij = softmax_j(Qbar_i . Kbar_j / sqrt(d)
 // + ln n_j), the centroid estimate of the block log-mass (PARK D.2).  Blocks
