@@ -36,6 +36,12 @@
 namespace spattn {
 namespace {
 
+// One pair of exponentials in every SPATTN_EXP_EMU pairs runs on the FMA pipe
+// (tc::ex2_fma) instead of the MUFU unit; 0 keeps every exponential on MUFU.
+#ifndef SPATTN_EXP_EMU
+#define SPATTN_EXP_EMU 0
+#endif
+
 constexpr int TC_THREADS = 192;
 constexpr int TILE_ROWS = 128;
 constexpr uint32_t TMEM_COLS = 256;  // S/P: columns [0,128), O: [128, 128+d)
@@ -56,6 +62,8 @@ struct __align__(8) TcCtrl {
   uint32_t tmem_base;
   int abort;
   uint32_t kept[64];  // kept-block bitmap of this query block (nb <= 2048)
+  uint32_t bad[64];   // tasks whose CSR block index is out of range (caller CSR)
+  int tail_task;      // task index of the partial last key block, -1 if none
 };
 
 template <int D>
@@ -94,14 +102,22 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
     tc::tc_fence_before();
   }
   if (warp < 4) {
-    const int nwords = (a.nb + 31) >> 5;
-    for (int q = threadIdx.x; q < nwords; q += 128) cs->kept[q] = 0;
+    for (int q = threadIdx.x; q < 64; q += 128) {
+      cs->kept[q] = 0;
+      cs->bad[q] = 0;
+    }
+    if (threadIdx.x == 0) cs->tail_task = -1;
   }
   __syncthreads();
-  if (warp < 4 && a.residual) {
-    for (int q = r_lo + threadIdx.x; q < r_lo + nkept; q += 128) {
-      const int j = __ldg(a.col_idx + q);
-      if (j >= 0 && j < a.nb) atomicOr(&cs->kept[j >> 5], 1u << (j & 31));
+  if (warp < 4) {
+    for (int t = threadIdx.x; t < nkept; t += 128) {
+      const int j = __ldg(a.col_idx + r_lo + t);
+      if (j >= 0 && j < a.nb) {
+        atomicOr(&cs->kept[j >> 5], 1u << (j & 31));
+        if (j == a.nb - 1 && a.n_last < TILE_ROWS) cs->tail_task = t;
+      } else if (t < 2048) {
+        atomicOr(&cs->bad[t >> 5], 1u << (t & 31));
+      }
     }
   }
   __syncthreads();
@@ -203,15 +219,6 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
     for (int t = 0; t < T; ++t) {
       if (!(ok = tc::mbar_wait(bar(B_SFULL), (uint32_t)t & 1u, abort, a.ctrl, 7))) break;
       tc::tc_fence_after();
-      // column bias for this task (log2 units): 0 / -inf for key tiles,
-      // log2 n_j / -inf for centroid tiles
-      int nvalid = 0, jres = -1;
-      if (t < nkept) {
-        const int j = __ldg(a.col_idx + r_lo + t);
-        nvalid = (j >= 0 && j < a.nb) ? ((j == a.nb - 1) ? a.n_last : TILE_ROWS) : 0;
-      } else {
-        jres = (t - nkept) * TILE_ROWS;
-      }
       uint32_t s[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -219,21 +226,38 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
         tc::tmem_ld32(tS + lane_off + 32 * c, chunk);
       }
       tc::tmem_wait_ld();
-      float rmax = -INFINITY;
+      // Key tiles: the max is taken on the raw scores (the scale is > 0) and
+      // columns past n_j of the partial last block (or a whole tile with a
+      // bad index) are set to -inf.  Centroid tiles: the log2-scaled logit
+      // plus the bias log2 n_j (dropped) / -inf (kept) is formed up front.
+      float scale = a.sl2;
+      if (t < nkept) {
+        const bool bad = t < 2048 && ((cs->bad[t >> 5] >> (t & 31)) & 1u);
+        const int nvalid = bad ? 0 : (t == cs->tail_task ? a.n_last : TILE_ROWS);
+        if (nvalid < TILE_ROWS) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float bias;
-        if (jres < 0) {
-          bias = c < nvalid ? 0.f : -INFINITY;
-        } else {
+          for (int c = 0; c < 128; ++c)
+            if (c >= nvalid) s[c] = __float_as_uint(-INFINITY);
+        }
+      } else {
+        const int jres = (t - nkept) * TILE_ROWS;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
           const int j = jres + c;
           const bool dropped = j < a.nb && !((cs->kept[j >> 5] >> (j & 31)) & 1u);
-          bias = dropped ? (j == a.nb - 1 ? lg_last : lg_b) : -INFINITY;
+          const float bias = dropped ? (j == a.nb - 1 ? lg_last : lg_b) : -INFINITY;
+          s[c] = __float_as_uint(fmaf(__uint_as_float(s[c]), a.sl2, bias));
         }
-        const float x = fmaf(__uint_as_float(s[c]), a.sl2, bias);
-        s[c] = __float_as_uint(x);
-        rmax = fmaxf(rmax, x);
+        scale = 1.f;
       }
+      float mx[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx[e] = __uint_as_float(s[e]);
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(s[c]));
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mx[e] = fmaxf(mx[e], mx[e + 4]);
+      const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale;
       // lazy rescale: a row moves its reference max only when the new max
       // exceeds it by more than 2^8; the TMEM read-modify-write of O is done
       // by the whole warp (tcgen05.ld/st are warp-collective), scale 1 for
@@ -245,20 +269,33 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
         l *= sc;
         m = rmax;
       }
-      const float mu = (m == -INFINITY) ? 0.f : m;
+      const float nmu = (m == -INFINITY) ? 0.f : -m;
+      float ls[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ls[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         // 32 logits -> 16 packed bf16 pairs -> TMEM columns [16c, 16c+16)
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = tc::ex2(__uint_as_float(s[32 * c + 2 * e]) - mu);
-          const float p1 = tc::ex2(__uint_as_float(s[32 * c + 2 * e + 1]) - mu);
-          l += p0 + p1;
+          const float x0 = fmaf(__uint_as_float(s[32 * c + 2 * e]), scale, nmu);
+          const float x1 = fmaf(__uint_as_float(s[32 * c + 2 * e + 1]), scale, nmu);
+          float p0, p1;
+          if (SPATTN_EXP_EMU > 0 && (e % (SPATTN_EXP_EMU > 0 ? SPATTN_EXP_EMU : 1)) == 0) {
+            p0 = tc::ex2_fma(x0);
+            p1 = tc::ex2_fma(x1);
+          } else {
+            p0 = tc::ex2(x0);
+            p1 = tc::ex2(x1);
+          }
+          ls[(2 * e) & 7] += p0;
+          ls[(2 * e + 1) & 7] += p1;
           pk[e] = pack_bf16x2(p0, p1);
         }
         tc::tmem_st16(tS + lane_off + 16 * c, pk);
       }
+      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       if (t > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {

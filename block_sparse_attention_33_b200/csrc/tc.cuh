@@ -178,5 +178,29 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, for x <= 8 (the softmax's exponent range): split
+// x = n + f with n = round(x) (adding and subtracting 1.5 * 2^23 rounds to an
+// integer under round-to-nearest), f in [-1/2, 1/2]; 2^f by a degree-3
+// polynomial whose coefficients are a relative-error minimax (Remez exchange)
+// fit of 2^f on [-1/2, 1/2] made for this file (max relative error 7.5e-5,
+// far below the 2^-9 rounding of the bf16 probabilities it feeds); 2^n is
+// added to the exponent field.  x is clamped at -125 so that the exponent
+// add stays in the normal range (about 2e-38, below every probability that
+// matters next to the row maximum's 1).
+constexpr float kExp2C0 = 0.99992805719375610f;
+constexpr float kExp2C1 = 0.69326096773147583f;
+constexpr float kExp2C2 = 0.24261112511157990f;
+constexpr float kExp2C3 = 0.05517166852951050f;
+
+__device__ __forceinline__ float ex2_fma(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = __fadd_rn(x, 12582912.f);
+  const float n = __fadd_rn(t, -12582912.f);
+  const float f = __fadd_rn(x, -n);
+  const float q = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  const int ni = __float_as_int(t) - 0x4B400000;
+  return __int_as_float(__float_as_int(q) + (ni << 23));
+}
+
 }  // namespace tc
 }  // namespace spattn
