@@ -10,7 +10,7 @@
 #include <numeric>
 #include <vector>
 
-#include "../../include/spattn.h"
+#include "spattn.h"
 #include "common.cuh"
 #include "internal.h"
 

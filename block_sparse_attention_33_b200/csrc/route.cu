@@ -15,8 +15,9 @@
 // same search on the count #{p_j > u} yields the top-k set when the clamp
 // binds.  Kept blocks are then emitted in ascending j with warp ballots.
 //
-// route_kernel: one CTA per (16 query blocks, head); 8 warps; the proxy tile
-// S[16][nb] is computed with fp32 FMAs (no TF32/BF16: a logit error of 1e-2
+// route_kernel: one CTA per (ROWS query blocks, head), ROWS = 4, 8 or 16 by
+// the number of blocks so that small problems still fill the GPU; 8 warps;
+// the proxy tile S[ROWS][nb] is computed with fp32 FMAs (no TF32/BF16: a logit error of 1e-2
 // would move cumulative mass by more than the 1e-4 comparison margin).
 #include "common.cuh"
 #include "internal.h"
@@ -24,8 +25,10 @@
 namespace spattn {
 namespace {
 
-constexpr int RT_ROWS = 16;      // query blocks per CTA
 constexpr int RT_THREADS = 256;
+
+// query blocks per routing CTA
+inline int route_rows_per_cta(int nb) { return nb <= 128 ? 4 : (nb <= 512 ? 8 : 16); }
 
 struct RouteArgs {
   const float* qbar;
@@ -72,7 +75,7 @@ __device__ __forceinline__ int count_equal(const float* p, int nb, uint32_t u) {
   return warp_sum_i(c);
 }
 
-template <int D>
+template <int D, int RT_ROWS>
 __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
   extern __shared__ __align__(16) float sm[];
   const int nbp = (a.nb + 31) & ~31;
@@ -257,9 +260,29 @@ __global__ void __launch_bounds__(256) compact_kernel(const int32_t* counts, con
 
 }  // namespace
 
-size_t route_smem_bytes(int d, int nb) {
+size_t route_smem_bytes(int d, int nb, int rows) {
   const int nbp = (nb + 31) & ~31;
-  return (size_t)RT_ROWS * (d + nbp) * sizeof(float);
+  return (size_t)rows * (d + nbp) * sizeof(float);
+}
+
+template <int D, int ROWS>
+cudaError_t launch_route_rows(const RouteArgs& a, int nb, int BH, cudaStream_t s) {
+  const size_t smem = route_smem_bytes(D, nb, ROWS);
+  cudaError_t e = cudaFuncSetAttribute(route_kernel<D, ROWS>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((nb + ROWS - 1) / ROWS, BH);
+  route_kernel<D, ROWS><<<grid, RT_THREADS, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_route_d(const RouteArgs& a, int nb, int BH, cudaStream_t s) {
+  switch (route_rows_per_cta(nb)) {
+    case 4: return launch_route_rows<D, 4>(a, nb, BH, s);
+    case 8: return launch_route_rows<D, 8>(a, nb, BH, s);
+    default: return launch_route_rows<D, 16>(a, nb, BH, s);
+  }
 }
 
 cudaError_t launch_route(const Problem& p, const Work& w, int32_t* row_ptr_out,
@@ -268,18 +291,8 @@ cudaError_t launch_route(const Problem& p, const Work& w, int32_t* row_ptr_out,
   a.qbar = w.qbar; a.kbar = w.kbar; a.counts = w.counts; a.lists = w.lists;
   a.nb = p.nb; a.b = p.b; a.n_last = p.n_last; a.kcap = p.kcap; a.kmin = p.kmin;
   a.tau = p.tau;
-  const size_t smem = route_smem_bytes(p.d, p.nb);
-  dim3 grid((p.nb + RT_ROWS - 1) / RT_ROWS, p.BH);
-  cudaError_t e;
-  if (p.d == 128) {
-    e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    route_kernel<128><<<grid, RT_THREADS, smem, s>>>(a);
-  } else {
-    e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    route_kernel<64><<<grid, RT_THREADS, smem, s>>>(a);
-  }
+  cudaError_t e = p.d == 128 ? launch_route_d<128>(a, p.nb, p.BH, s)
+                             : launch_route_d<64>(a, p.nb, p.BH, s);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int rows = p.BH * p.nb;
   scan_kernel<<<1, SCAN_THREADS, (p.kcap + 1) * sizeof(int), s>>>(w.counts, rows, p.kcap,

@@ -21,7 +21,7 @@
 #include <stdarg.h>
 #include <stdio.h>
 
-#include "../../include/spattn.h"
+#include "spattn.h"
 #include "common.cuh"
 #include "internal.h"
 

@@ -56,6 +56,13 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
   }
 }
 
+// Inline fast path: a phase that has already completed costs one try_wait.
+__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, volatile int* abort,
+                                               int32_t* ctrl, int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait(bar, parity, abort, ctrl, site);
+}
+
 // Short bounded wait used only while winding down after an abort.
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   const long long t0 = clock64();
@@ -178,6 +185,31 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// ---- paired fp32 arithmetic (one instruction for two lanes of values) ----
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;\n" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // 2^x on the FMA pipe, for x <= 8 (the softmax's exponent range): split
 // x = n + f with n = round(x) (adding and subtracting 1.5 * 2^23 rounds to an
 // integer under round-to-nearest), f in [-1/2, 1/2]; 2^f by a degree-3
@@ -200,6 +232,27 @@ __device__ __forceinline__ float ex2_fma(float x) {
   const float q = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
   const int ni = __float_as_int(t) - 0x4B400000;
   return __int_as_float(__float_as_int(q) + (ni << 23));
+}
+
+// Two lanes of ex2_fma with paired arithmetic: the same steps and constants;
+// the exponent add bits(q) + (bits(t) << 23) equals bits(q) + (n << 23)
+// modulo 2^32 because the low nine bits of bits(1.5 * 2^23) are zero.
+__device__ __forceinline__ uint64_t ex2_fma2(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x2 = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t big = f2_pack(12582912.f, 12582912.f), nbig = f2_pack(-12582912.f, -12582912.f);
+  const uint64_t t = f2_add(x2, big);
+  const uint64_t n = f2_add(t, nbig);
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x2);
+  uint64_t q = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+  q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
+  q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23)),
+                 __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23)));
 }
 
 }  // namespace tc

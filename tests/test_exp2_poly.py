@@ -55,3 +55,13 @@ def test_coefficients_are_a_fit_of_exp2():
     # sanity: at f = 0 the polynomial is ~1, its slope ~ln 2
     c0, c1, _, _ = coeffs()
     assert abs(c0 - 1) < 1e-4 and abs(c1 - np.log(2)) < 2e-3
+
+
+def test_paired_exponent_add_matches_scalar():
+    """The paired form adds bits(t) << 23 instead of n << 23; the two agree
+    modulo 2^32 because the low nine bits of bits(1.5 * 2^23) are zero."""
+    x = np.linspace(-125, 8, 100_001, dtype=np.float32)
+    t = (x + np.float32(12582912.0)).astype(np.float32)
+    n_shift = ((t.view(np.int32) - np.int32(0x4B400000)).astype(np.int64) << 23) & 0xFFFFFFFF
+    t_shift = (t.view(np.uint32).astype(np.int64) << 23) & 0xFFFFFFFF
+    assert np.array_equal(n_shift, t_shift)
