@@ -3,24 +3,33 @@
 //
 // One CTA per work item (head bh, query block i of 128 tokens), one CTA per
 // SM; items are launched longest budget first (the counting sort of the
-// routing step).  TMEM (512 columns) holds two S buffers, the O accumulator
-// and two P buffers, so the MMA of task t+1 runs while the softmax of task t
-// is computed and the tensor core is fed back to back.  Warp roles:
+// routing step).  TMEM (512 columns) holds two S buffers and two O
+// accumulators, one per 64-key half of every key tile, so the MMA of task
+// t+1 runs while the softmax of task t is computed.  Warp roles:
 //
 //   warps 0-7  softmax.  Warp w owns TMEM lane quarter w % 4 (query rows
-//              32(w%4) .. +31) and key-column half w / 4 of every S tile.  Both
-//              warps of a quarter read the whole 128-column row to form the
-//              same row maximum, then each exponentiates its 64 columns and
-//              writes them as packed bf16 into the P buffer.  The running max
-//              moves only when it grows by more than 2^8 (then O and the
-//              partial sums are rescaled).  The epilogue normalises O and
-//              stores each row, scattered through perm.
+//              32(w%4) .. +31) and key half h = w / 4 of every S tile, and runs
+//              its own online softmax over those keys with its own reference
+//              maximum m and sum l; O_h accumulates P_h V_h.  The softmax is
+//              max-free: m is the row maximum of the first tile, after which
+//              p = 2^(s * scale - m) is computed directly and the tile's
+//              partial sum tells when m must move (sum > 2^16: m moves up by
+//              the integer part of log2 of the sum, an exact power-of-two
+//              rescale of l and O_h; sum > 2^60 or not finite: the tile is
+//              recomputed against its own maximum).  Optionally a fixed
+//              share of the exponentials runs on the FMA pipe (tc::ex2_fma2);
+//              measured on B200 the MUFU-only form is faster for this
+//              structure, so the share defaults to zero.  P(t) is written as packed bf16 over the warp's own,
+//              already read, columns of S(t).  The epilogue merges the two
+//              halves of each row, normalises and stores the row, scattered
+//              through perm.
 //   warp 8     producer: TMA loads of the Q tile and of the K and V tiles
 //              (128 tokens x d, 128-byte swizzle, no multicast) through one
 //              ring of shared-memory slots, in the order the MMA consumes them.
 //   warp 9     MMA issuer: S = Q K^T (both operands in shared memory) into
-//              S buffer t & 1, and O += P V (P from TMEM, V from shared memory),
-//              tcgen05.mma with fp32 accumulation in TMEM.
+//              S buffer t & 1, and O_h += P_h V_h for both halves (P from
+//              TMEM, V from shared memory), tcgen05.mma with fp32
+//              accumulation in TMEM.
 //
 // Tasks of an item: its kept key blocks (CSR row; Sol-Attn: "a single
 // online-softmax pass" over the selected blocks), then, in residual mode,
@@ -44,8 +53,9 @@
 namespace spattn {
 namespace {
 
-// One pair of exponentials in every SPATTN_EXP_EMU pairs runs on the FMA pipe
-// (tc::ex2_fma2) instead of the MUFU unit; 0 keeps every exponential on MUFU.
+// SPATTN_EXP_EMU of every 8 pairs of exponentials run on the FMA pipe
+// (tc::ex2_fma2) instead of the MUFU unit (0: all on MUFU, the fastest
+// setting measured for this kernel).
 #ifndef SPATTN_EXP_EMU
 #define SPATTN_EXP_EMU 0
 #endif
@@ -55,9 +65,10 @@ constexpr int WARP_PRODUCER = 8, WARP_MMA = 9;
 constexpr int TC_THREADS = 32 * 10;
 constexpr int TILE_ROWS = 128;
 constexpr uint32_t TMEM_COLS = 512;
-// TMEM column map: S buffers [0,128) and [128,256), O [256, 256+d),
-// P buffers [384, 448) and [448, 512) (bf16 packed two per column).
-constexpr uint32_t COL_O = 256, COL_P = 384;
+// TMEM column map: S buffers [0,128) and [128,256); O_0 [256, 256+d) and
+// O_1 [384, 384+d).  P(t) (bf16, two per column) of key half h lives in
+// columns [64h, 64h+32) of S buffer t & 1.
+constexpr uint32_t COL_O = 256;
 constexpr int MAX_STAGES = 10;
 
 template <int D>
@@ -70,7 +81,6 @@ struct TcCfg {
 enum : int {
   B_QFULL = 0,
   B_SFULL0, B_SFULL1,      // S buffer b holds S(t) (MMA commit)
-  B_SUSED0, B_SUSED1,      // S buffer b has been read by all softmax warps
   B_PREADY,                // P(t) written by all softmax warps (one phase per task)
   B_PVDONE,                // PV(t) complete (one phase per task)
   B_OFULL, B_DRAIN,
@@ -92,7 +102,8 @@ struct __align__(8) TcCtrl {
   uint32_t kept[64];  // kept-block bitmap of this query block (nb <= 2048)
   uint32_t bad[64];   // tasks whose CSR block index is out of range (caller CSR)
   int tail_task;      // task index of the partial last key block, -1 if none
-  float lsum[2][TILE_ROWS];  // partial row sums of the two column halves
+  float xm[2][TILE_ROWS];    // epilogue: reference max of each key half
+  float xl[2][TILE_ROWS];    // epilogue: sum of each key half
 };
 
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
@@ -130,8 +141,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tc::mbar_init(bar(B_QFULL), 1);
     tc::mbar_init(bar(B_SFULL0), 1);
     tc::mbar_init(bar(B_SFULL1), 1);
-    tc::mbar_init(bar(B_SUSED0), NUM_SOFTMAX_WARPS);
-    tc::mbar_init(bar(B_SUSED1), NUM_SOFTMAX_WARPS);
     tc::mbar_init(bar(B_PREADY), NUM_SOFTMAX_WARPS);
     tc::mbar_init(bar(B_PVDONE), 1);
     tc::mbar_init(bar(B_OFULL), 1);
@@ -274,24 +283,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int s = li % STAGES;
         if (!(ok = tc::mbar_wait_fast(full(s), (uint32_t)(li / STAGES) & 1u, abort, a.ctrl, 6))) break;
         tc::tc_fence_after();
-        // O += P V: M = 128 queries, N = d, K = 128 keys in steps of 16; P is
-        // bf16 packed two per TMEM column, V is MN-major (d contiguous)
+        // O_h += P_h V_h for both key halves: M = 128 queries, N = d, K = 64
+        // keys in steps of 16; P is bf16 packed two per TMEM column, V is
+        // MN-major (d contiguous), rows 64h .. 64h+63 of the tile
         const uint64_t slot16 = (uint64_t)(s * TILE_BYTES / 16);
-        const uint32_t tP = tmem + COL_P + 64u * (uint32_t)(t & 1);
+        const uint32_t tP = tmem + 128u * (uint32_t)(t & 1);
 #pragma unroll
-        for (int kk = 0; kk < TILE_ROWS / 16; ++kk)
-          tc::umma_ts(tmem + COL_O, tP + kk * 8, dV + slot16 + (uint64_t)(kk * 2048 / 16), idO,
-                      (t > 0 || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc::umma_ts(tmem + COL_O + 128u * h, tP + 64u * h + 8u * kk,
+                        dV + slot16 + (uint64_t)((64 * h + 16 * kk) * 128 / 16), idO,
+                        (t > 0 || kk > 0) ? 1u : 0u);
         tc::umma_commit(empty(s));
         tc::umma_commit(bar(B_PVDONE));
         ++li;
-        if (t + 2 < T) {
-          // S buffer t & 1 is free once every softmax warp has read S(t)
-          if (!(ok = tc::mbar_wait_fast(bar(B_SUSED0 + (t & 1)), (uint32_t)(t >> 1) & 1u, abort,
-                                        a.ctrl, 9)))
-            break;
-          if (!(ok = issue_s(t + 2))) break;
-        }
+        // S buffer t & 1 (S(t), then P(t)) is free once PV(t) has run; the
+        // tensor core executes in issue order
+        if (t + 2 < T && !(ok = issue_s(t + 2))) break;
       }
       if (ok) {
         tc::umma_commit(bar(B_OFULL));
@@ -306,87 +315,93 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int quarter = warp & 3, half = warp >> 2;
     const int r = quarter * 32 + lane;                 // row / TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tOh = tmem + lane_off + COL_O + 128u * (uint32_t)half;  // this half's O
     const int rows_valid = (i == a.nb - 1) ? a.n_last : TILE_ROWS;
     const float lg_b = log2f((float)TILE_ROWS), lg_last = log2f((float)a.n_last);
-    float m = -INFINITY, l = 0.f;
+    // m: reference maximum of this row's key half (log2 units); l: sum of
+    // p at that reference; owe: factor O_h owes once PV(t-1) is done.
+    float m = -INFINITY, l = 0.f, owe = 1.f;
     bool ok = true;
+
+    auto rescale_o = [&](float f) {
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        tc::tmem_ld32(tOh + 32u * c, ov);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+        tc::tmem_st32(tOh + 32u * c, ov);
+      }
+    };
+
     for (int t = 0; t < T; ++t) {
       const int b = t & 1;
       if (!(ok = tc::mbar_wait_fast(bar(B_SFULL0 + b), (uint32_t)(t >> 1) & 1u, abort, a.ctrl, 7)))
         break;
       tc::tc_fence_after();
-      uint32_t s[128];
+      // this warp's 64 columns of S(t).  Key tiles: columns past n_j of the
+      // partial last block (or a whole tile with a bad index) are set to
+      // -inf.  Centroid tiles: the log2-scaled logit plus the bias log2 n_j
+      // (dropped) / -inf (kept) is formed up front.
+      uint32_t u[64];
+      const uint32_t scol = tmem + lane_off + 128u * (uint32_t)b + 64u * (uint32_t)half;
+      const float scale = t < nkept ? a.sl2 : 1.f;
+      auto load_s = [&]() {
+        tc::tmem_ld32(scol, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+        tc::tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+        tc::tmem_wait_ld();
+        if (t < nkept) {
+          const bool bad = t < 2048 && ((cs->bad[t >> 5] >> (t & 31)) & 1u);
+          const int nvalid = (bad ? 0 : (t == cs->tail_task ? a.n_last : TILE_ROWS)) - 64 * half;
+          if (nvalid < 64) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t (&chunk)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]);
-        tc::tmem_ld32(tmem + lane_off + 128u * b + 32 * c, chunk);
-      }
-      tc::tmem_wait_ld();
-      // S(t) is in registers: the MMA may overwrite the buffer with S(t+2)
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar(B_SUSED0 + b));
-      // Key tiles: the max is taken on the raw scores (the scale is > 0) and
-      // columns past n_j of the partial last block (or a whole tile with a
-      // bad index) are set to -inf.  Centroid tiles: the log2-scaled logit
-      // plus the bias log2 n_j (dropped) / -inf (kept) is formed up front.
-      float scale = a.sl2;
-      if (t < nkept) {
-        const bool bad = t < 2048 && ((cs->bad[t >> 5] >> (t & 31)) & 1u);
-        const int nvalid = bad ? 0 : (t == cs->tail_task ? a.n_last : TILE_ROWS);
-        if (nvalid < TILE_ROWS) {
+            for (int c = 0; c < 64; ++c)
+              if (c >= nvalid) u[c] = __float_as_uint(-INFINITY);
+          }
+        } else {
+          const int jres = res_tile(t - nkept) * TILE_ROWS + 64 * half;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c >= nvalid) s[c] = __float_as_uint(-INFINITY);
+          for (int c = 0; c < 64; ++c) {
+            const int j = jres + c;
+            const bool dropped = j < a.nb && !((cs->kept[j >> 5] >> (j & 31)) & 1u);
+            const float bias = dropped ? (j == a.nb - 1 ? lg_last : lg_b) : -INFINITY;
+            u[c] = __float_as_uint(fmaf(__uint_as_float(u[c]), a.sl2, bias));
+          }
         }
-      } else {
-        const int jres = res_tile(t - nkept) * TILE_ROWS;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int j = jres + c;
-          const bool dropped = j < a.nb && !((cs->kept[j >> 5] >> (j & 31)) & 1u);
-          const float bias = dropped ? (j == a.nb - 1 ? lg_last : lg_b) : -INFINITY;
-          s[c] = __float_as_uint(fmaf(__uint_as_float(s[c]), a.sl2, bias));
-        }
-        scale = 1.f;
-      }
-      // row max over all 128 columns (both halves compute the same value):
-      // 8 independent chains of 3-input max
-      float mx[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mx[e] = __uint_as_float(s[e]);
-#pragma unroll
-      for (int c = 8; c < 128; c += 16) {
+      };
+      load_s();
+      auto tile_max = [&]() {
+        float mx[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          mx[e] = tc::fmax3(mx[e], __uint_as_float(s[c + e]), __uint_as_float(s[c + e + 8]));
+          mx[e] = tc::fmax3(__uint_as_float(u[e]), __uint_as_float(u[e + 8]), __uint_as_float(u[e + 16]));
+#pragma unroll
+        for (int c = 24; c < 64; c += 16)
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            mx[e] = c + 8 + e < 64 ? tc::fmax3(mx[e], __uint_as_float(u[c + e]), __uint_as_float(u[c + e + 8]))
+                                   : fmaxf(mx[e], __uint_as_float(u[c + e]));
+        return tc::fmax3(tc::fmax3(mx[0], mx[1], mx[2]), tc::fmax3(mx[3], mx[4], mx[5]),
+                         fmaxf(mx[6], mx[7])) * scale;
+      };
+      // a row without a reference yet (first tile, or only masked keys so
+      // far) takes this tile's maximum
+      if (__any_sync(0xffffffffu, m == -INFINITY)) {
+        if (m == -INFINITY) m = tile_max();
       }
-      const float rmax = tc::fmax3(tc::fmax3(mx[0], mx[1], mx[2]), tc::fmax3(mx[3], mx[4], mx[5]),
-                                   fmaxf(mx[6], mx[7])) * scale;
-      // lazy rescale: a row moves its reference max only when the new max
-      // exceeds it by more than 2^8
-      const bool grow = rmax > m + 8.0f;
-      float sc = 1.f;
-      if (grow) {
-        sc = tc::ex2(m - rmax);
-        l *= sc;
-        m = rmax;
-      }
-      const float nmu = (m == -INFINITY) ? 0.f : -m;
-      // this warp's 64 columns: p = 2^(s * scale - m), paired arithmetic; the
-      // column half is a template argument so that s[] stays in registers
-      const uint64_t sc2 = tc::f2_pack(scale, scale), nmu2 = tc::f2_pack(nmu, nmu);
-      uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[32];
-      auto exps = [&](auto H) {
-        constexpr int c0 = 64 * decltype(H)::value;
+      float lt;
+      auto exps = [&]() {
+        const float nmu = (m == -INFINITY) ? 0.f : -m;
+        const uint64_t sc2 = tc::f2_pack(scale, scale), nmu2 = tc::f2_pack(nmu, nmu);
+        uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const uint64_t x2 = tc::f2_fma(
-              tc::f2_pack(__uint_as_float(s[c0 + 2 * e]), __uint_as_float(s[c0 + 2 * e + 1])), sc2,
-              nmu2);
+              tc::f2_pack(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1])), sc2, nmu2);
           float p0, p1;
-          if (SPATTN_EXP_EMU > 0 && (e % (SPATTN_EXP_EMU > 0 ? SPATTN_EXP_EMU : 1)) == 0) {
+          if ((e & 7) < SPATTN_EXP_EMU) {
             tc::f2_unpack(tc::ex2_fma2(x2), p0, p1);
           } else {
             float x0, x1;
@@ -397,32 +412,50 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           ls2[e & 3] = tc::f2_add(ls2[e & 3], tc::f2_pack(p0, p1));
           pk[e] = pack_bf16x2(p0, p1);
         }
-      };
-      if (half == 0) exps(std::integral_constant<int, 0>());
-      else exps(std::integral_constant<int, 1>());
-      tc::tmem_st32(tmem + lane_off + COL_P + 64u * b + 32u * half, pk);
-      {
         const uint64_t t2 = tc::f2_add(tc::f2_add(ls2[0], ls2[1]), tc::f2_add(ls2[2], ls2[3]));
         float lo, hi;
         tc::f2_unpack(t2, lo, hi);
-        l += lo + hi;
+        lt = lo + hi;
+      };
+      exps();
+      // A tile far above the reference is recomputed against its own
+      // maximum, so every p stays below 2^60 (bf16 P and fp32 O cannot
+      // overflow); O_h then owes the factor before PV(t).
+      const bool over = !(lt <= 1.152921504606847e18f);   // 2^60; also catches inf / NaN
+      if (__any_sync(0xffffffffu, over)) {
+        load_s();   // S(t) is still in TMEM: reload rather than keep u live
+        if (over) {
+          const float mn = fmaxf(m, tile_max());
+          const float f = tc::ex2(m - mn);
+          l *= f;
+          owe *= f;
+          m = mn;
+        }
+        exps();
       }
-      if (t > 0 && __any_sync(0xffffffffu, grow)) {
-        // O holds PV(0..t-1) once PV(t-1) is done; this warp rescales its half
-        // of the head dimension (scale 1 on rows that keep their max)
+      tc::tmem_st32(scol, pk);   // P(t) over this warp's own, already read, columns
+      l += lt;
+      // O_h owes `owe` once PV(t-1) is done (factor 1 on rows owing nothing).
+      // Every phase of the PV barrier is waited for, so its parity always
+      // names the one PV in question.
+      if (t > 0) {
         if (!(ok = tc::mbar_wait_fast(bar(B_PVDONE), (uint32_t)(t - 1) & 1u, abort, a.ctrl, 10)))
           break;
-        tc::tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t ov[32];
-          const uint32_t col = tmem + lane_off + COL_O + (uint32_t)(half * (D / 2) + 32 * c);
-          tc::tmem_ld32(col, ov);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * sc);
-          tc::tmem_st32(col, ov);
+        if (__any_sync(0xffffffffu, owe != 1.f)) {
+          tc::tc_fence_after();
+          rescale_o(owe);
         }
+      }
+      owe = 1.f;
+      // keep p moderate: when this tile's sum passes 2^16 the reference moves
+      // up by the integer part of log2(sum), an exact power-of-two rescale
+      // (l now; O_h after PV(t), in the next step)
+      if (lt > 65536.f) {
+        const int e = ((int)(__float_as_uint(lt) >> 23) & 0xFF) - 127;
+        const float f = __int_as_float((127 - e) << 23);   // 2^-e
+        l *= f;
+        owe = f;
+        m += (float)e;
       }
       tc::tmem_wait_st();
       tc::tc_fence_before();
@@ -430,37 +463,54 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (lane == 0) tc::mbar_arrive(bar(B_PREADY));
     }
     if (ok && T > 0) ok = tc::mbar_wait(bar(B_OFULL), 0, abort, a.ctrl, 8);
-    // both halves of a row combine their partial sums (named barrier per
-    // lane quarter, 64 threads)
-    cs->lsum[half][r] = l;
+    if (ok && __any_sync(0xffffffffu, owe != 1.f)) {
+      tc::tc_fence_after();
+      rescale_o(owe);
+      tc::tmem_wait_st();
+    }
+    // merge the two key halves of each row (named barrier per lane quarter)
+    cs->xm[half][r] = m;
+    cs->xl[half][r] = l;
+    tc::tc_fence_before();
     named_sync(1 + quarter, 64);
-    const float ltot = cs->lsum[0][r] + cs->lsum[1][r];
+    const float m0 = cs->xm[0][r], m1 = cs->xm[1][r];
+    const float M = fmaxf(m0, m1);
+    const float a0 = m0 == -INFINITY ? 0.f : tc::ex2(m0 - M);
+    const float a1 = m1 == -INFINITY ? 0.f : tc::ex2(m1 - M);
+    const float L = a0 * cs->xl[0][r] + a1 * cs->xl[1][r];
     if (ok) {
       tc::tc_fence_after();
       const int tok = i * TILE_ROWS + r;
       const bool store = r < rows_valid;
       const int dst = store ? (a.perm ? __ldg(a.perm + tok) : tok) : 0;
       uint4* orow = reinterpret_cast<uint4*>(a.o + ((size_t)bh * a.N + dst) * D + half * (D / 2));
-      const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      const float w0 = a0 * inv, w1 = a1 * inv;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
-        uint32_t ov[32];
-        if (T > 0) {  // CTA-uniform: every lane of the warp takes part in the load
-          tc::tmem_ld32(tmem + lane_off + COL_O + (uint32_t)(half * (D / 2) + 32 * c), ov);
+        uint32_t o0[32], o1[32];
+        if (T > 0) {  // CTA-uniform: every lane of the warp takes part in the loads
+          const uint32_t col = (uint32_t)(half * (D / 2) + 32 * c);
+          tc::tmem_ld32(tmem + lane_off + COL_O + col, o0);
+          tc::tmem_ld32(tmem + lane_off + COL_O + 128u + col, o1);
           tc::tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = 0u;
+          for (int e = 0; e < 32; ++e) o0[e] = o1[e] = 0u;
         }
         if (store) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(ov[8 * q + 0]) * inv, __uint_as_float(ov[8 * q + 1]) * inv);
-            v.y = pack_bf16x2(__uint_as_float(ov[8 * q + 2]) * inv, __uint_as_float(ov[8 * q + 3]) * inv);
-            v.z = pack_bf16x2(__uint_as_float(ov[8 * q + 4]) * inv, __uint_as_float(ov[8 * q + 5]) * inv);
-            v.w = pack_bf16x2(__uint_as_float(ov[8 * q + 6]) * inv, __uint_as_float(ov[8 * q + 7]) * inv);
-            orow[c * 4 + q] = v;
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              v[e] = __uint_as_float(o0[8 * q + e]) * w0 + __uint_as_float(o1[8 * q + e]) * w1;
+            uint4 pv;
+            pv.x = pack_bf16x2(v[0], v[1]);
+            pv.y = pack_bf16x2(v[2], v[3]);
+            pv.z = pack_bf16x2(v[4], v[5]);
+            pv.w = pack_bf16x2(v[6], v[7]);
+            orow[c * 4 + q] = pv;
           }
         }
       }
