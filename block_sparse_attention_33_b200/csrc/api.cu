@@ -6,8 +6,11 @@
 #include <string.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
 #include <new>
 #include <numeric>
+#include <utility>
 #include <vector>
 
 #include "spattn.h"
@@ -103,6 +106,21 @@ Work bind(const Problem& p, const Layout& L, void* ws) {
 
 namespace spattn {
 void record_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+
+cudaError_t ensure_dyn_smem(const void* fn, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;  // below the default limit
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, size_t> granted;
+  std::lock_guard<std::mutex> lock(mu);
+  size_t& g = granted[{fn, dev}];
+  if (g >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) g = bytes;
+  return e;
+}
 }  // namespace spattn
 
 struct spattn_plan_s {

@@ -263,8 +263,7 @@ __global__ void __launch_bounds__(BQ * 2, 1) attn_mma_kernel(AttnArgs a) {
 template <int D, int BQ>
 cudaError_t launch_one(const AttnArgs& a, int items, cudaStream_t s) {
   const size_t smem = (size_t)BQ * D * 2 + 4 * KT * D * 2 + (2048 / 32) * 4;
-  cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel<D, BQ>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_dyn_smem((const void*)attn_mma_kernel<D, BQ>, smem);
   if (e != cudaSuccess) return e;
   attn_mma_kernel<D, BQ><<<items, BQ * 2, smem, s>>>(a);
   return cudaGetLastError();

@@ -40,4 +40,9 @@ cudaError_t launch_attend(const Problem& p, const void* Q, const void* K, const 
                           const int32_t* row_ptr, const int32_t* col_idx, void* O,
                           const Work& w, cudaStream_t s);
 
+// Raise kernel `fn`'s dynamic shared-memory limit on the current device to at
+// least `bytes`; the attribute call is made only when a launch needs more
+// than was granted before (thread-safe).
+cudaError_t ensure_dyn_smem(const void* fn, size_t bytes);
+
 }  // namespace spattn

@@ -19,6 +19,9 @@
 // the number of blocks so that small problems still fill the GPU; 8 warps;
 // the proxy tile S[ROWS][nb] is computed with fp32 FMAs (no TF32/BF16: a logit error of 1e-2
 // would move cumulative mass by more than the 1e-4 comparison margin).
+#include <algorithm>
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -190,51 +193,65 @@ __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
 }
 
 // Exclusive scan of the per-row counts into row_ptr (single CTA), total in
-// ctrl[CTRL_NNZ]; also a counting sort of the rows by descending budget, so
-// that the attention grid starts with the longest rows.
+// ctrl[CTRL_NNZ]; also the work order of the attention grid: rows grouped by
+// consecutive heads (group_rows rows per group, sized so one group's K and V
+// stay resident in L2 while its rows run), longest budget first inside a
+// group.  The order is a counting sort on the key
+// group * (kcap + 1) + (kcap - count).
 constexpr int SCAN_THREADS = 1024;
 
-__global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(const int32_t* counts, int rows,
-                                                            int kcap, int32_t* row_ptr,
-                                                            int32_t* order, int32_t* ctrl) {
-  __shared__ int part[SCAN_THREADS];
-  extern __shared__ int hist[];  // [kcap + 1]
-  const int per = (rows + SCAN_THREADS - 1) / SCAN_THREADS;
-  const int lo = threadIdx.x * per, hi = min(rows, lo + per);
-  for (int q = threadIdx.x; q <= kcap; q += SCAN_THREADS) hist[q] = 0;
-  int s = 0;
-  for (int q = lo; q < hi; ++q) s += counts[q];
-  part[threadIdx.x] = s;
+__device__ __forceinline__ int block_exclusive_scan(int v, int* part) {
+  part[threadIdx.x] = v;
   __syncthreads();
-  for (int q = lo; q < hi; ++q) atomicAdd(&hist[min(counts[q], kcap)], 1);
-  // Hillis-Steele inclusive scan over the thread partials
   for (int off = 1; off < SCAN_THREADS; off <<= 1) {
-    const int v = threadIdx.x >= off ? part[threadIdx.x - off] : 0;
+    const int u = threadIdx.x >= off ? part[threadIdx.x - off] : 0;
     __syncthreads();
-    part[threadIdx.x] += v;
+    part[threadIdx.x] += u;
     __syncthreads();
   }
-  int run = threadIdx.x ? part[threadIdx.x - 1] : 0;
+  const int ex = threadIdx.x ? part[threadIdx.x - 1] : 0;
+  return ex;
+}
+
+__global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(const int32_t* counts, int rows,
+                                                            int kcap, int group_rows,
+                                                            int32_t* row_ptr, int32_t* order,
+                                                            int32_t* ctrl) {
+  __shared__ int part[SCAN_THREADS];
+  extern __shared__ int hist[];  // [ngroups * (kcap + 1)]
+  const int ngroups = (rows + group_rows - 1) / group_rows;
+  const int nbins = ngroups * (kcap + 1);
+  auto key = [&](int q) { return (q / group_rows) * (kcap + 1) + (kcap - min(counts[q], kcap)); };
+  const int per = (rows + SCAN_THREADS - 1) / SCAN_THREADS;
+  const int lo = threadIdx.x * per, hi = min(rows, lo + per);
+  for (int q = threadIdx.x; q < nbins; q += SCAN_THREADS) hist[q] = 0;
+  int s = 0;
+  for (int q = lo; q < hi; ++q) s += counts[q];
+  int run = block_exclusive_scan(s, part);
+  if (threadIdx.x == SCAN_THREADS - 1) {
+    row_ptr[rows] = run + s;
+    ctrl[CTRL_NNZ] = run + s;
+  }
   for (int q = lo; q < hi; ++q) {
     row_ptr[q] = run;
     run += counts[q];
   }
-  if (threadIdx.x == SCAN_THREADS - 1) {
-    row_ptr[rows] = part[SCAN_THREADS - 1];
-    ctrl[CTRL_NNZ] = part[SCAN_THREADS - 1];
+  // (the scan's barriers also order the zeroing of hist before the counts)
+  for (int q = lo; q < hi; ++q) atomicAdd(&hist[key(q)], 1);
+  __syncthreads();
+  // exclusive offsets of the bins in ascending key order
+  const int bper = (nbins + SCAN_THREADS - 1) / SCAN_THREADS;
+  const int blo = threadIdx.x * bper, bhi = min(nbins, blo + bper);
+  int bs = 0;
+  for (int q = blo; q < bhi; ++q) bs += hist[q];
+  int acc = block_exclusive_scan(bs, part);
+  for (int q = blo; q < bhi; ++q) {
+    const int c = hist[q];
+    hist[q] = acc;
+    acc += c;
   }
   __syncthreads();
-  // descending-budget start offsets (serial over at most kcap+1 bins)
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int q = kcap; q >= 0; --q) {
-      const int c = hist[q];
-      hist[q] = acc;
-      acc += c;
-    }
-  }
-  __syncthreads();
-  for (int q = lo; q < hi; ++q) order[atomicAdd(&hist[min(counts[q], kcap)], 1)] = q;
+  for (int q = lo; q < hi; ++q) order[atomicAdd(&hist[key(q)], 1)] = q;
 }
 
 // Copy the padded per-row lists into the compact CSR (one warp per row).
@@ -268,8 +285,7 @@ size_t route_smem_bytes(int d, int nb, int rows) {
 template <int D, int ROWS>
 cudaError_t launch_route_rows(const RouteArgs& a, int nb, int BH, cudaStream_t s) {
   const size_t smem = route_smem_bytes(D, nb, ROWS);
-  cudaError_t e = cudaFuncSetAttribute(route_kernel<D, ROWS>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_dyn_smem((const void*)route_kernel<D, ROWS>, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((nb + ROWS - 1) / ROWS, BH);
   route_kernel<D, ROWS><<<grid, RT_THREADS, smem, s>>>(a);
@@ -285,6 +301,32 @@ cudaError_t launch_route_d(const RouteArgs& a, int nb, int BH, cudaStream_t s) {
   }
 }
 
+// Rows per work-order group: whole heads, as many as keep the group's K and V
+// (bf16) within a third of the device's L2, and few enough groups that the
+// scan's histogram fits its shared-memory budget.
+static int scan_group_rows(const Problem& p) {
+  static std::atomic<long long> l2_cache[64];
+  long long l2 = 126ll << 20;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+    long long c = l2_cache[dev].load(std::memory_order_relaxed);
+    if (c == 0) {
+      int v = 0;
+      if (cudaDeviceGetAttribute(&v, cudaDevAttrL2CacheSize, dev) == cudaSuccess && v > 0) c = v;
+      else c = l2;
+      l2_cache[dev].store(c, std::memory_order_relaxed);
+    }
+    l2 = c;
+  }
+  const long long head_bytes = 2ll * p.N * p.d * 2;  // K and V of one head
+  int heads = (int)std::max(1ll, (l2 / 3) / std::max(1ll, head_bytes));
+  heads = std::min(heads, p.BH);
+  constexpr long long HIST_BUDGET = 96 * 1024;
+  const long long max_groups = std::max(1ll, HIST_BUDGET / ((long long)(p.kcap + 1) * 4));
+  while ((p.BH + heads - 1) / heads > max_groups) ++heads;
+  return heads * p.nb;
+}
+
 cudaError_t launch_route(const Problem& p, const Work& w, int32_t* row_ptr_out,
                          int32_t* col_idx_out, cudaStream_t s) {
   RouteArgs a;
@@ -295,8 +337,12 @@ cudaError_t launch_route(const Problem& p, const Work& w, int32_t* row_ptr_out,
                              : launch_route_d<64>(a, p.nb, p.BH, s);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int rows = p.BH * p.nb;
-  scan_kernel<<<1, SCAN_THREADS, (p.kcap + 1) * sizeof(int), s>>>(w.counts, rows, p.kcap,
-                                                                  w.row_ptr, w.order, w.ctrl);
+  const int group_rows = scan_group_rows(p);
+  const size_t hist_bytes =
+      (size_t)((rows + group_rows - 1) / group_rows) * (p.kcap + 1) * sizeof(int);
+  if ((e = ensure_dyn_smem((const void*)scan_kernel, hist_bytes)) != cudaSuccess) return e;
+  scan_kernel<<<1, SCAN_THREADS, hist_bytes, s>>>(w.counts, rows, p.kcap, group_rows, w.row_ptr,
+                                                  w.order, w.ctrl);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   compact_kernel<<<(rows + 7) / 8, 256, 0, s>>>(w.counts, w.lists, w.row_ptr, rows, p.kcap,
                                                 w.col_idx, row_ptr_out, col_idx_out);
