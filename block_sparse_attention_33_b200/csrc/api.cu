@@ -230,9 +230,8 @@ spattn_status_t spattn_pool(spattn_plan_t plan, const void* Q, const void* K, co
   if (spattn_status_t st = check_inputs(plan, Q, K, V, workspace)) return st;
   const Work w = bind(plan->p, plan->L, workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(w.ctrl, 0, spattn::CTRL_WORDS * sizeof(int32_t), s);
-  if (e != cudaSuccess) return cuda_fail(e, "clearing the control block");
-  e = spattn::launch_pool(plan->p, Q, K, V, w, s);
+  // the pooling kernel also clears the control block
+  cudaError_t e = spattn::launch_pool(plan->p, Q, K, V, w, s);
   if (e != cudaSuccess) return cuda_fail(e, "pool kernel");
   return SPATTN_OK;
 }
@@ -242,9 +241,8 @@ spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, c
   if (spattn_status_t st = check_inputs(plan, Q, K, V, workspace)) return st;
   const Work w = bind(plan->p, plan->L, workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(w.ctrl, 0, spattn::CTRL_WORDS * sizeof(int32_t), s);
-  if (e != cudaSuccess) return cuda_fail(e, "clearing the control block");
-  e = spattn::launch_pool(plan->p, Q, K, V, w, s);
+  // the pooling kernel also clears the control block
+  cudaError_t e = spattn::launch_pool(plan->p, Q, K, V, w, s);
   if (e != cudaSuccess) return cuda_fail(e, "pool kernel");
   e = spattn::launch_route(plan->p, w, row_ptr, col_idx, s);
   if (e != cudaSuccess) return cuda_fail(e, "route kernels");

@@ -44,6 +44,7 @@
 // are drained with a further bounded wait, and TMEM is freed before exit.
 #include <cuda.h>
 
+#include <algorithm>
 #include <type_traits>
 
 #include "common.cuh"
@@ -79,36 +80,47 @@ struct TcCfg {
 
 // mbarrier indices
 enum : int {
-  B_QFULL = 0,
-  B_SFULL0, B_SFULL1,      // S buffer b holds S(t) (MMA commit)
-  B_PREADY,                // P(t) written by all softmax warps (one phase per task)
-  B_PVDONE,                // PV(t) complete (one phase per task)
-  B_OFULL, B_DRAIN,
-  B_RING,                  // full[s] at B_RING + s, empty[s] at B_RING + STAGES + s
+  B_QFULL = 0, B_QEMPTY,   // Q tile loaded / its last S MMA complete
+  B_SFULL0, B_SFULL1,      // S buffer b holds S(g) (MMA commit)
+  B_PREADY,                // P(g) written by all softmax warps (one phase per task)
+  B_PVDONE,                // PV(g) complete (one phase per task)
+  B_OFULL,                 // last PV of an item complete (one phase per item with tasks)
+  B_DRAIN,
+  B_INFO_FULL0, B_INFO_FULL1,    // item slot s described by the producer warp
+  B_INFO_EMPTY0, B_INFO_EMPTY1,  // item slot s released by the MMA and softmax warps
+  B_XREADY,                // + 4 * slot + quarter: both key halves of a lane quarter merged
+  B_RING = B_XREADY + 8,   // full[s] at B_RING + s, empty[s] at B_RING + STAGES + s
 };
 
 struct TcArgs {
   const int32_t *row_ptr, *col_idx, *order, *perm;
   __nv_bfloat16* o;
   int32_t* ctrl;
-  int N, nb, n_last, residual;
+  int N, nb, n_last, residual, items;
   float sl2;  // log2(e) / sqrt(d)
+};
+
+// One work item as described by the producer warp.  Two slots: the producer
+// builds item n+1 (and starts its loads) while item n is still in the
+// softmax and epilogue.
+struct ItemInfo {
+  int item;            // bh * nb + i; -1 once the work is exhausted
+  int nkept;           // kept key blocks (CSR row length)
+  int T;               // tasks: the kept blocks, then residual centroid tiles
+  int tail_task;       // task index of the partial last key block, -1 if none
+  uint32_t res_tiles;  // bit c: centroid tile c holds a dropped block
+  uint32_t kept[64];   // kept-block bitmap (nb <= 2048)
+  uint32_t bad[64];    // tasks whose CSR block index is out of range (caller CSR)
 };
 
 struct __align__(8) TcCtrl {
   uint64_t bar[B_RING + 2 * MAX_STAGES];
   uint32_t tmem_base;
   int abort;
-  uint32_t kept[64];  // kept-block bitmap of this query block (nb <= 2048)
-  uint32_t bad[64];   // tasks whose CSR block index is out of range (caller CSR)
-  int tail_task;      // task index of the partial last key block, -1 if none
-  float xm[2][TILE_ROWS];    // epilogue: reference max of each key half
-  float xl[2][TILE_ROWS];    // epilogue: sum of each key half
+  ItemInfo info[2];
+  float xm[2][2][TILE_ROWS];  // epilogue, per item slot: reference max of each key half
+  float xl[2][2][TILE_ROWS];  // epilogue, per item slot: sum of each key half
 };
-
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 template <int D>
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -130,21 +142,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   auto full = [&](int s) { return bar(B_RING + s); };
   auto empty = [&](int s) { return bar(B_RING + STAGES + s); };
   volatile int* abort = &cs->abort;
-
-  const int item = a.order ? a.order[blockIdx.x] : blockIdx.x;
-  const int bh = item / a.nb, i = item % a.nb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r_lo = __ldg(a.row_ptr + item);
-  const int nkept = max(0, __ldg(a.row_ptr + item + 1) - r_lo);
+  // A wait made by all 32 lanes of a warp, with a warp-uniform result (one
+  // lane may see the phase complete while another sees an abort first).
+  auto wait_warp = [&](uint32_t b, uint32_t parity, int site) {
+    return __all_sync(0xffffffffu, tc::mbar_wait_fast(b, parity, abort, a.ctrl, site));
+  };
 
   if (threadIdx.x == 0) {
     tc::mbar_init(bar(B_QFULL), 1);
+    tc::mbar_init(bar(B_QEMPTY), 1);
     tc::mbar_init(bar(B_SFULL0), 1);
     tc::mbar_init(bar(B_SFULL1), 1);
     tc::mbar_init(bar(B_PREADY), NUM_SOFTMAX_WARPS);
     tc::mbar_init(bar(B_PVDONE), 1);
     tc::mbar_init(bar(B_OFULL), 1);
     tc::mbar_init(bar(B_DRAIN), 1);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(bar(B_INFO_FULL0 + s), 32);
+      tc::mbar_init(bar(B_INFO_EMPTY0 + s), 1 + NUM_SOFTMAX_WARPS);
+    }
+    for (int q = 0; q < 8; ++q) tc::mbar_init(bar(B_XREADY + q), 64);
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(full(s), 1);
       tc::mbar_init(empty(s), 1);
@@ -156,101 +174,143 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tc::tmem_alloc(smem_u32(&cs->tmem_base), TMEM_COLS);
     tc::tc_fence_before();
   }
-  if (warp < NUM_SOFTMAX_WARPS) {
-    for (int q = threadIdx.x; q < 64; q += 32 * NUM_SOFTMAX_WARPS) {
-      cs->kept[q] = 0;
-      cs->bad[q] = 0;
-    }
-    if (threadIdx.x == 0) cs->tail_task = -1;
-  }
-  __syncthreads();
-  if (warp < NUM_SOFTMAX_WARPS) {
-    for (int t = threadIdx.x; t < nkept; t += 32 * NUM_SOFTMAX_WARPS) {
-      const int j = __ldg(a.col_idx + r_lo + t);
-      if (j >= 0 && j < a.nb) {
-        atomicOr(&cs->kept[j >> 5], 1u << (j & 31));
-        if (j == a.nb - 1 && a.n_last < TILE_ROWS) cs->tail_task = t;
-      } else if (t < 2048) {
-        atomicOr(&cs->bad[t >> 5], 1u << (t & 31));
-      }
-    }
-  }
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = cs->tmem_base;
-  // Centroid tiles that hold at least one dropped block; every role derives
-  // the same task list from the shared bitmap.
-  uint32_t res_tiles = 0;
-  if (a.residual) {
-    const int ntiles = (a.nb + TILE_ROWS - 1) / TILE_ROWS;
-    for (int c = 0; c < ntiles; ++c) {
-      bool any = false;
-      for (int q = 0; q < TILE_ROWS / 32; ++q) {
-        const int j0 = c * TILE_ROWS + q * 32;
-        if (j0 >= a.nb) break;
-        const int cnt = min(32, a.nb - j0);
-        const uint32_t valid = cnt == 32 ? 0xffffffffu : ((1u << cnt) - 1u);
-        any |= (~cs->kept[j0 >> 5] & valid) != 0u;
-      }
-      if (any) res_tiles |= 1u << c;
-    }
-  }
-  const int T = nkept + __popc(res_tiles);
-  // tile of the r-th residual task
-  auto res_tile = [&](int r) { return (int)__fns(res_tiles, 0, r + 1); };
+  const int ntiles = (a.nb + TILE_ROWS - 1) / TILE_ROWS;   // centroid tiles (<= 16)
+  // centroid tile of the r-th residual task
+  auto res_tile = [](uint32_t tiles, int r) { return (int)__fns(tiles, 0, r + 1); };
 
   if (warp == WARP_PRODUCER) {
     // ---------------------------------------------------------- producer
-    // load order = consumption order: K(0), K(1), then per task t: V(t),
-    // K(t+2)
-    if (lane == 0 && T > 0) {
-      tc::mbar_expect_tx(bar(B_QFULL), TILE_BYTES);
-#pragma unroll
-      for (int c = 0; c < NCH; ++c)
-        tc::tma_load_3d(sQ + c * CHUNK_BYTES, &tmQ, bar(B_QFULL), c * 64, i * TILE_ROWS, bh);
-      int li = 0;  // loads issued
-      auto issue = [&](int t, bool is_v) -> bool {
-        const CUtensorMap* m;
-        int row;
-        if (t < nkept) {
-          int j = __ldg(a.col_idx + r_lo + t);
-          if (j < 0 || j >= a.nb) {
-            flag_error(a.ctrl, DEV_BAD_INDEX, item);
-            j = 0;  // load something valid; the softmax masks the whole task
-          }
-          m = is_v ? &tmV : &tmK;
-          row = j * TILE_ROWS;
-        } else {
-          m = is_v ? &tmVb : &tmKb;
-          row = res_tile(t - nkept) * TILE_ROWS;
-        }
-        const int s = li % STAGES;
-        if (!tc::mbar_wait_fast(empty(s), ((uint32_t)(li / STAGES) & 1u) ^ 1u, abort, a.ctrl, 1))
-          return false;
-        tc::mbar_expect_tx(full(s), TILE_BYTES);
-        const uint32_t dst = sRing + s * TILE_BYTES;
-#pragma unroll
-        for (int c = 0; c < NCH; ++c) tc::tma_load_3d(dst + c * CHUNK_BYTES, m, full(s), c * 64, row, bh);
-        ++li;
-        return true;
-      };
-      bool ok = issue(0, false);
-      if (ok && T > 1) ok = issue(1, false);
-      for (int t = 0; ok && t < T; ++t) {
-        ok = issue(t, true);
-        if (ok && t + 2 < T) ok = issue(t + 2, false);
+    // Per item: take a ticket from the device work counter, describe the
+    // item (whole warp), then TMA loads (lane 0) in consumption order:
+    // Q, K(0), K(1), then per task t: V(t), K(t+2).
+    int n = 0, qn = 0, li = 0;  // items taken, items with tasks (Q loads), K/V loads issued
+    bool ok = true;
+    for (;; ++n) {
+      const int slot = n & 1;
+      if (n >= 2 && !(ok = wait_warp(bar(B_INFO_EMPTY0 + slot), (uint32_t)((n - 2) >> 1) & 1u, 11)))
+        break;
+      int ticket = 0;
+      if (lane == 0) ticket = atomicAdd(a.ctrl + CTRL_WORK, 1);
+      ticket = __shfl_sync(0xffffffffu, ticket, 0);
+      ItemInfo& inf = cs->info[slot];
+      if (ticket >= a.items) {
+        if (lane == 0) inf.item = -1;
+        __syncwarp();
+        tc::mbar_arrive(bar(B_INFO_FULL0 + slot));
+        break;
       }
+      const int item = a.order ? __ldg(a.order + ticket) : ticket;
+      const int bh = item / a.nb, i = item % a.nb;
+      const int r_lo = __ldg(a.row_ptr + item);
+      const int nkept = max(0, __ldg(a.row_ptr + item + 1) - r_lo);
+      inf.kept[lane] = 0u;
+      inf.kept[lane + 32] = 0u;
+      inf.bad[lane] = 0u;
+      inf.bad[lane + 32] = 0u;
+      if (lane == 0) inf.tail_task = -1;
+      __syncwarp();
+      for (int t = lane; t < nkept; t += 32) {
+        const int j = __ldg(a.col_idx + r_lo + t);
+        if (j >= 0 && j < a.nb) {
+          atomicOr(&inf.kept[j >> 5], 1u << (j & 31));
+          if (j == a.nb - 1 && a.n_last < TILE_ROWS) inf.tail_task = t;
+        } else if (t < 2048) {
+          atomicOr(&inf.bad[t >> 5], 1u << (t & 31));
+        }
+      }
+      __syncwarp();
+      // centroid tiles that hold at least one dropped block
+      bool any = false;
+      if (a.residual && lane < ntiles) {
+        for (int q = 0; q < TILE_ROWS / 32; ++q) {
+          const int j0 = lane * TILE_ROWS + q * 32;
+          if (j0 >= a.nb) break;
+          const int cnt = min(32, a.nb - j0);
+          const uint32_t valid = cnt == 32 ? 0xffffffffu : ((1u << cnt) - 1u);
+          any |= (~inf.kept[j0 >> 5] & valid) != 0u;
+        }
+      }
+      const uint32_t res_tiles = __ballot_sync(0xffffffffu, any);
+      const int T = nkept + __popc(res_tiles);
+      if (lane == 0) {
+        inf.item = item;
+        inf.nkept = nkept;
+        inf.T = T;
+        inf.res_tiles = res_tiles;
+      }
+      __syncwarp();
+      tc::mbar_arrive(bar(B_INFO_FULL0 + slot));   // every lane: releases its own writes
+      if (T == 0) continue;
+      if (lane == 0) {
+        if (qn > 0)
+          ok = tc::mbar_wait_fast(bar(B_QEMPTY), (uint32_t)(qn - 1) & 1u, abort, a.ctrl, 12);
+        if (ok) {
+          tc::mbar_expect_tx(bar(B_QFULL), TILE_BYTES);
+#pragma unroll
+          for (int c = 0; c < NCH; ++c)
+            tc::tma_load_3d(sQ + c * CHUNK_BYTES, &tmQ, bar(B_QFULL), c * 64, i * TILE_ROWS, bh);
+        }
+        auto issue = [&](int t, bool is_v) -> bool {
+          const CUtensorMap* m;
+          int row;
+          if (t < nkept) {
+            int j = __ldg(a.col_idx + r_lo + t);
+            if (j < 0 || j >= a.nb) {
+              flag_error(a.ctrl, DEV_BAD_INDEX, item);
+              j = 0;  // load something valid; the softmax masks the whole task
+            }
+            m = is_v ? &tmV : &tmK;
+            row = j * TILE_ROWS;
+          } else {
+            m = is_v ? &tmVb : &tmKb;
+            row = res_tile(res_tiles, t - nkept) * TILE_ROWS;
+          }
+          const int s = li % STAGES;
+          if (!tc::mbar_wait_fast(empty(s), ((uint32_t)(li / STAGES) & 1u) ^ 1u, abort, a.ctrl, 1))
+            return false;
+          tc::mbar_expect_tx(full(s), TILE_BYTES);
+          const uint32_t dst = sRing + s * TILE_BYTES;
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) tc::tma_load_3d(dst + c * CHUNK_BYTES, m, full(s), c * 64, row, bh);
+          ++li;
+          return true;
+        };
+        if (ok) ok = issue(0, false);
+        if (ok && T > 1) ok = issue(1, false);
+        for (int t = 0; ok && t < T; ++t) {
+          ok = issue(t, true);
+          if (ok && t + 2 < T) ok = issue(t + 2, false);
+        }
+      }
+      ++qn;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+    }
+    if (lane == 0) {
       if (*abort) {
         // let the copies already issued land before the CTA can exit
-        tc::mbar_drain(bar(B_QFULL), 0);
+        if (qn > 0) tc::mbar_drain(bar(B_QFULL), (uint32_t)(qn - 1) & 1u);
         for (int k = (li > STAGES ? li - STAGES : 0); k < li; ++k)
           tc::mbar_drain(full(k % STAGES), (uint32_t)(k / STAGES) & 1u);
+        // take the remaining tickets so the retirement count below holds
+        while (atomicAdd(a.ctrl + CTRL_WORK, 1) < a.items) {
+        }
+      }
+      // The last CTA to retire resets the work counter for the next launch
+      // (every CTA has drawn its final ticket before it retires).
+      __threadfence();
+      if (atomicAdd(a.ctrl + CTRL_DONE, 1) == (int)gridDim.x - 1) {
+        atomicExch(a.ctrl + CTRL_WORK, 0);
+        atomicExch(a.ctrl + CTRL_DONE, 0);
       }
     }
     __syncwarp();
   } else if (warp == WARP_MMA) {
     // --------------------------------------------------------------- MMA
-    if (lane == 0 && T > 0) {
+    if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idO = tc::idesc_bf16_f32(128, D, true);
       // loop-invariant descriptors; k-step and slot offsets are added to the
@@ -258,53 +318,74 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint64_t dQ = tc::sdesc_sw128(sQ, 16, 1024);
       const uint64_t dK = tc::sdesc_sw128(sRing, 16, 1024);
       const uint64_t dV = tc::sdesc_sw128(sRing, CHUNK_BYTES, 1024);
-      int li = 0;  // loads consumed
-      auto issue_s = [&](int t) -> bool {
+      int n = 0, qn = 0, gt = 0, li = 0;  // items, items with tasks, tasks before this item, loads consumed
+      bool ok = true;
+      // S(g) = Q K^T into S buffer g & 1
+      auto issue_s = [&](int g) -> bool {
         const int s = li % STAGES;
         if (!tc::mbar_wait_fast(full(s), (uint32_t)(li / STAGES) & 1u, abort, a.ctrl, 4)) return false;
         tc::tc_fence_after();
         const uint64_t slot16 = (uint64_t)(s * TILE_BYTES / 16);
-        const uint32_t dS = tmem + 128u * (uint32_t)(t & 1);
+        const uint32_t dS = tmem + 128u * (uint32_t)(g & 1);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off16 = ((kk >> 2) * CHUNK_BYTES + (kk & 3) * 32) >> 4;
           tc::umma_ss(dS, dQ + off16, dK + slot16 + off16, idS, kk > 0);
         }
         tc::umma_commit(empty(s));
-        tc::umma_commit(bar(B_SFULL0 + (t & 1)));
+        tc::umma_commit(bar(B_SFULL0 + (g & 1)));
         ++li;
         return true;
       };
-      bool ok = tc::mbar_wait_fast(bar(B_QFULL), 0, abort, a.ctrl, 3);
-      if (ok) ok = issue_s(0);
-      if (ok && T > 1) ok = issue_s(1);
-      for (int t = 0; ok && t < T; ++t) {
-        if (!(ok = tc::mbar_wait_fast(bar(B_PREADY), (uint32_t)t & 1u, abort, a.ctrl, 5))) break;
-        const int s = li % STAGES;
-        if (!(ok = tc::mbar_wait_fast(full(s), (uint32_t)(li / STAGES) & 1u, abort, a.ctrl, 6))) break;
-        tc::tc_fence_after();
-        // O_h += P_h V_h for both key halves: M = 128 queries, N = d, K = 64
-        // keys in steps of 16; P is bf16 packed two per TMEM column, V is
-        // MN-major (d contiguous), rows 64h .. 64h+63 of the tile
-        const uint64_t slot16 = (uint64_t)(s * TILE_BYTES / 16);
-        const uint32_t tP = tmem + 128u * (uint32_t)(t & 1);
+      for (;; ++n) {
+        const int slot = n & 1;
+        if (!(ok = tc::mbar_wait_fast(bar(B_INFO_FULL0 + slot), (uint32_t)(n >> 1) & 1u, abort, a.ctrl, 13)))
+          break;
+        const int item = cs->info[slot].item;
+        if (item < 0) break;
+        const int T = cs->info[slot].T;
+        if (T > 0) {
+          ok = tc::mbar_wait_fast(bar(B_QFULL), (uint32_t)qn & 1u, abort, a.ctrl, 3);
+          if (ok) ok = issue_s(gt);
+          if (ok && T > 1) ok = issue_s(gt + 1);
+          if (ok && T <= 2) tc::umma_commit(bar(B_QEMPTY));
+          for (int t = 0; ok && t < T; ++t) {
+            const int g = gt + t;
+            if (!(ok = tc::mbar_wait_fast(bar(B_PREADY), (uint32_t)g & 1u, abort, a.ctrl, 5))) break;
+            const int s = li % STAGES;
+            if (!(ok = tc::mbar_wait_fast(full(s), (uint32_t)(li / STAGES) & 1u, abort, a.ctrl, 6))) break;
+            tc::tc_fence_after();
+            // O_h += P_h V_h for both key halves: M = 128 queries, N = d,
+            // K = 64 keys in steps of 16; P is bf16 packed two per TMEM
+            // column, V is MN-major (d contiguous), rows 64h .. 64h+63 of the
+            // tile
+            const uint64_t slot16 = (uint64_t)(s * TILE_BYTES / 16);
+            const uint32_t tP = tmem + 128u * (uint32_t)(g & 1);
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+            for (int h = 0; h < 2; ++h)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc::umma_ts(tmem + COL_O + 128u * h, tP + 64u * h + 8u * kk,
-                        dV + slot16 + (uint64_t)((64 * h + 16 * kk) * 128 / 16), idO,
-                        (t > 0 || kk > 0) ? 1u : 0u);
-        tc::umma_commit(empty(s));
-        tc::umma_commit(bar(B_PVDONE));
-        ++li;
-        // S buffer t & 1 (S(t), then P(t)) is free once PV(t) has run; the
-        // tensor core executes in issue order
-        if (t + 2 < T && !(ok = issue_s(t + 2))) break;
+              for (int kk = 0; kk < 4; ++kk)
+                tc::umma_ts(tmem + COL_O + 128u * h, tP + 64u * h + 8u * kk,
+                            dV + slot16 + (uint64_t)((64 * h + 16 * kk) * 128 / 16), idO,
+                            (t > 0 || kk > 0) ? 1u : 0u);
+            tc::umma_commit(empty(s));
+            tc::umma_commit(bar(B_PVDONE));
+            ++li;
+            // S buffer g & 1 (S(g), then P(g)) is free once PV(g) has run;
+            // the tensor core executes in issue order
+            if (t + 2 < T) {
+              if (!(ok = issue_s(g + 2))) break;
+              if (t + 3 == T) tc::umma_commit(bar(B_QEMPTY));   // Q's last use
+            }
+          }
+          if (ok) tc::umma_commit(bar(B_OFULL));
+          gt += T;
+          ++qn;
+        }
+        if (!ok) break;
+        tc::mbar_arrive(bar(B_INFO_EMPTY0 + slot));
       }
-      if (ok) {
-        tc::umma_commit(bar(B_OFULL));
-      } else {
+      if (!ok) {
         tc::umma_commit(bar(B_DRAIN));
         tc::mbar_drain(bar(B_DRAIN), 0);
       }
@@ -316,11 +397,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int r = quarter * 32 + lane;                 // row / TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tOh = tmem + lane_off + COL_O + 128u * (uint32_t)half;  // this half's O
-    const int rows_valid = (i == a.nb - 1) ? a.n_last : TILE_ROWS;
     const float lg_b = log2f((float)TILE_ROWS), lg_last = log2f((float)a.n_last);
-    // m: reference maximum of this row's key half (log2 units); l: sum of
-    // p at that reference; owe: factor O_h owes once PV(t-1) is done.
-    float m = -INFINITY, l = 0.f, owe = 1.f;
+    int n = 0, qn = 0, gt = 0;  // items, items with tasks, tasks before this item
     bool ok = true;
 
     auto rescale_o = [&](float f) {
@@ -335,187 +413,210 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
     };
 
-    for (int t = 0; t < T; ++t) {
-      const int b = t & 1;
-      if (!(ok = tc::mbar_wait_fast(bar(B_SFULL0 + b), (uint32_t)(t >> 1) & 1u, abort, a.ctrl, 7)))
-        break;
-      tc::tc_fence_after();
-      // this warp's 64 columns of S(t).  Key tiles: columns past n_j of the
-      // partial last block (or a whole tile with a bad index) are set to
-      // -inf.  Centroid tiles: the log2-scaled logit plus the bias log2 n_j
-      // (dropped) / -inf (kept) is formed up front.
-      uint32_t u[64];
-      const uint32_t scol = tmem + lane_off + 128u * (uint32_t)b + 64u * (uint32_t)half;
-      const float scale = t < nkept ? a.sl2 : 1.f;
-      auto load_s = [&]() {
-        tc::tmem_ld32(scol, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-        tc::tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-        tc::tmem_wait_ld();
-        if (t < nkept) {
-          const bool bad = t < 2048 && ((cs->bad[t >> 5] >> (t & 31)) & 1u);
-          const int nvalid = (bad ? 0 : (t == cs->tail_task ? a.n_last : TILE_ROWS)) - 64 * half;
-          if (nvalid < 64) {
+    for (;; ++n) {
+      const int slot = n & 1;
+      if (!(ok = wait_warp(bar(B_INFO_FULL0 + slot), (uint32_t)(n >> 1) & 1u, 14))) break;
+      const ItemInfo& inf = cs->info[slot];
+      const int item = inf.item;
+      if (item < 0) break;
+      const int T = inf.T, nkept = inf.nkept, tail_task = inf.tail_task;
+      const uint32_t res_tiles = inf.res_tiles;
+      const int bh = item / a.nb, i = item % a.nb;
+      const int rows_valid = (i == a.nb - 1) ? a.n_last : TILE_ROWS;
+      // m: reference maximum of this row's key half (log2 units); l: sum of
+      // p at that reference; owe: factor O_h owes once PV(g-1) is done.
+      float m = -INFINITY, l = 0.f, owe = 1.f;
+
+      for (int t = 0; t < T; ++t) {
+        const int g = gt + t, b = g & 1;
+        if (!(ok = wait_warp(bar(B_SFULL0 + b), (uint32_t)(g >> 1) & 1u, 7))) break;
+        tc::tc_fence_after();
+        // this warp's 64 columns of S(g).  Key tiles: columns past n_j of the
+        // partial last block (or a whole tile with a bad index) are set to
+        // -inf.  Centroid tiles: the log2-scaled logit plus the bias log2 n_j
+        // (dropped) / -inf (kept) is formed up front.
+        uint32_t u[64];
+        const uint32_t scol = tmem + lane_off + 128u * (uint32_t)b + 64u * (uint32_t)half;
+        const float scale = t < nkept ? a.sl2 : 1.f;
+        auto load_s = [&]() {
+          tc::tmem_ld32(scol, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+          tc::tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+          tc::tmem_wait_ld();
+          if (t < nkept) {
+            const bool bad = t < 2048 && ((inf.bad[t >> 5] >> (t & 31)) & 1u);
+            const int nvalid = (bad ? 0 : (t == tail_task ? a.n_last : TILE_ROWS)) - 64 * half;
+            if (nvalid < 64) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (c >= nvalid) u[c] = __float_as_uint(-INFINITY);
+              for (int c = 0; c < 64; ++c)
+                if (c >= nvalid) u[c] = __float_as_uint(-INFINITY);
+            }
+          } else {
+            const int jres = res_tile(res_tiles, t - nkept) * TILE_ROWS + 64 * half;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+              const int j = jres + c;
+              const bool dropped = j < a.nb && !((inf.kept[j >> 5] >> (j & 31)) & 1u);
+              const float bias = dropped ? (j == a.nb - 1 ? lg_last : lg_b) : -INFINITY;
+              u[c] = __float_as_uint(fmaf(__uint_as_float(u[c]), a.sl2, bias));
+            }
           }
-        } else {
-          const int jres = res_tile(t - nkept) * TILE_ROWS + 64 * half;
-#pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int j = jres + c;
-            const bool dropped = j < a.nb && !((cs->kept[j >> 5] >> (j & 31)) & 1u);
-            const float bias = dropped ? (j == a.nb - 1 ? lg_last : lg_b) : -INFINITY;
-            u[c] = __float_as_uint(fmaf(__uint_as_float(u[c]), a.sl2, bias));
-          }
-        }
-      };
-      load_s();
-      auto tile_max = [&]() {
-        float mx[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          mx[e] = tc::fmax3(__uint_as_float(u[e]), __uint_as_float(u[e + 8]), __uint_as_float(u[e + 16]));
-#pragma unroll
-        for (int c = 24; c < 64; c += 16)
+        };
+        load_s();
+        auto tile_max = [&]() {
+          float mx[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            mx[e] = c + 8 + e < 64 ? tc::fmax3(mx[e], __uint_as_float(u[c + e]), __uint_as_float(u[c + e + 8]))
-                                   : fmaxf(mx[e], __uint_as_float(u[c + e]));
-        return tc::fmax3(tc::fmax3(mx[0], mx[1], mx[2]), tc::fmax3(mx[3], mx[4], mx[5]),
-                         fmaxf(mx[6], mx[7])) * scale;
-      };
-      // a row without a reference yet (first tile, or only masked keys so
-      // far) takes this tile's maximum
-      if (__any_sync(0xffffffffu, m == -INFINITY)) {
-        if (m == -INFINITY) m = tile_max();
-      }
-      uint32_t pk[32];
-      float lt;
-      auto exps = [&]() {
-        const float nmu = (m == -INFINITY) ? 0.f : -m;
-        const uint64_t sc2 = tc::f2_pack(scale, scale), nmu2 = tc::f2_pack(nmu, nmu);
-        uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
+            mx[e] = tc::fmax3(__uint_as_float(u[e]), __uint_as_float(u[e + 8]), __uint_as_float(u[e + 16]));
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const uint64_t x2 = tc::f2_fma(
-              tc::f2_pack(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1])), sc2, nmu2);
-          float p0, p1;
-          if ((e & 7) < SPATTN_EXP_EMU) {
-            tc::f2_unpack(tc::ex2_fma2(x2), p0, p1);
-          } else {
-            float x0, x1;
-            tc::f2_unpack(x2, x0, x1);
-            p0 = tc::ex2(x0);
-            p1 = tc::ex2(x1);
-          }
-          ls2[e & 3] = tc::f2_add(ls2[e & 3], tc::f2_pack(p0, p1));
-          pk[e] = pack_bf16x2(p0, p1);
-        }
-        const uint64_t t2 = tc::f2_add(tc::f2_add(ls2[0], ls2[1]), tc::f2_add(ls2[2], ls2[3]));
-        float lo, hi;
-        tc::f2_unpack(t2, lo, hi);
-        lt = lo + hi;
-      };
-      exps();
-      // A tile far above the reference is recomputed against its own
-      // maximum, so every p stays below 2^60 (bf16 P and fp32 O cannot
-      // overflow); O_h then owes the factor before PV(t).
-      const bool over = !(lt <= 1.152921504606847e18f);   // 2^60; also catches inf / NaN
-      if (__any_sync(0xffffffffu, over)) {
-        load_s();   // S(t) is still in TMEM: reload rather than keep u live
-        if (over) {
-          const float mn = fmaxf(m, tile_max());
-          const float f = tc::ex2(m - mn);
-          l *= f;
-          owe *= f;
-          m = mn;
-        }
-        exps();
-      }
-      tc::tmem_st32(scol, pk);   // P(t) over this warp's own, already read, columns
-      l += lt;
-      // O_h owes `owe` once PV(t-1) is done (factor 1 on rows owing nothing).
-      // Every phase of the PV barrier is waited for, so its parity always
-      // names the one PV in question.
-      if (t > 0) {
-        if (!(ok = tc::mbar_wait_fast(bar(B_PVDONE), (uint32_t)(t - 1) & 1u, abort, a.ctrl, 10)))
-          break;
-        if (__any_sync(0xffffffffu, owe != 1.f)) {
-          tc::tc_fence_after();
-          rescale_o(owe);
-        }
-      }
-      owe = 1.f;
-      // keep p moderate: when this tile's sum passes 2^16 the reference moves
-      // up by the integer part of log2(sum), an exact power-of-two rescale
-      // (l now; O_h after PV(t), in the next step)
-      if (lt > 65536.f) {
-        const int e = ((int)(__float_as_uint(lt) >> 23) & 0xFF) - 127;
-        const float f = __int_as_float((127 - e) << 23);   // 2^-e
-        l *= f;
-        owe = f;
-        m += (float)e;
-      }
-      tc::tmem_wait_st();
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar(B_PREADY));
-    }
-    if (ok && T > 0) ok = tc::mbar_wait(bar(B_OFULL), 0, abort, a.ctrl, 8);
-    if (ok && __any_sync(0xffffffffu, owe != 1.f)) {
-      tc::tc_fence_after();
-      rescale_o(owe);
-      tc::tmem_wait_st();
-    }
-    // merge the two key halves of each row (named barrier per lane quarter)
-    cs->xm[half][r] = m;
-    cs->xl[half][r] = l;
-    tc::tc_fence_before();
-    named_sync(1 + quarter, 64);
-    const float m0 = cs->xm[0][r], m1 = cs->xm[1][r];
-    const float M = fmaxf(m0, m1);
-    const float a0 = m0 == -INFINITY ? 0.f : tc::ex2(m0 - M);
-    const float a1 = m1 == -INFINITY ? 0.f : tc::ex2(m1 - M);
-    const float L = a0 * cs->xl[0][r] + a1 * cs->xl[1][r];
-    if (ok) {
-      tc::tc_fence_after();
-      const int tok = i * TILE_ROWS + r;
-      const bool store = r < rows_valid;
-      const int dst = store ? (a.perm ? __ldg(a.perm + tok) : tok) : 0;
-      uint4* orow = reinterpret_cast<uint4*>(a.o + ((size_t)bh * a.N + dst) * D + half * (D / 2));
-      const float inv = L > 0.f ? 1.f / L : 0.f;
-      const float w0 = a0 * inv, w1 = a1 * inv;
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t o0[32], o1[32];
-        if (T > 0) {  // CTA-uniform: every lane of the warp takes part in the loads
-          const uint32_t col = (uint32_t)(half * (D / 2) + 32 * c);
-          tc::tmem_ld32(tmem + lane_off + COL_O + col, o0);
-          tc::tmem_ld32(tmem + lane_off + COL_O + 128u + col, o1);
-          tc::tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o0[e] = o1[e] = 0u;
-        }
-        if (store) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float v[8];
+          for (int c = 24; c < 64; c += 16)
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              v[e] = __uint_as_float(o0[8 * q + e]) * w0 + __uint_as_float(o1[8 * q + e]) * w1;
-            uint4 pv;
-            pv.x = pack_bf16x2(v[0], v[1]);
-            pv.y = pack_bf16x2(v[2], v[3]);
-            pv.z = pack_bf16x2(v[4], v[5]);
-            pv.w = pack_bf16x2(v[6], v[7]);
-            orow[c * 4 + q] = pv;
+              mx[e] = c + 8 + e < 64 ? tc::fmax3(mx[e], __uint_as_float(u[c + e]), __uint_as_float(u[c + e + 8]))
+                                     : fmaxf(mx[e], __uint_as_float(u[c + e]));
+          return tc::fmax3(tc::fmax3(mx[0], mx[1], mx[2]), tc::fmax3(mx[3], mx[4], mx[5]),
+                           fmaxf(mx[6], mx[7])) * scale;
+        };
+        // a row without a reference yet (first tile, or only masked keys so
+        // far) takes this tile's maximum
+        if (__any_sync(0xffffffffu, m == -INFINITY)) {
+          if (m == -INFINITY) m = tile_max();
+        }
+        uint32_t pk[32];
+        float lt;
+        auto exps = [&]() {
+          const float nmu = (m == -INFINITY) ? 0.f : -m;
+          const uint64_t sc2 = tc::f2_pack(scale, scale), nmu2 = tc::f2_pack(nmu, nmu);
+          uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const uint64_t x2 = tc::f2_fma(
+                tc::f2_pack(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1])), sc2, nmu2);
+            float p0, p1;
+            if ((e & 7) < SPATTN_EXP_EMU) {
+              tc::f2_unpack(tc::ex2_fma2(x2), p0, p1);
+            } else {
+              float x0, x1;
+              tc::f2_unpack(x2, x0, x1);
+              p0 = tc::ex2(x0);
+              p1 = tc::ex2(x1);
+            }
+            ls2[e & 3] = tc::f2_add(ls2[e & 3], tc::f2_pack(p0, p1));
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          const uint64_t t2 = tc::f2_add(tc::f2_add(ls2[0], ls2[1]), tc::f2_add(ls2[2], ls2[3]));
+          float lo, hi;
+          tc::f2_unpack(t2, lo, hi);
+          lt = lo + hi;
+        };
+        exps();
+        // A tile far above the reference is recomputed against its own
+        // maximum, so every p stays below 2^60 (bf16 P and fp32 O cannot
+        // overflow); O_h then owes the factor before PV(g).
+        const bool over = !(lt <= 1.152921504606847e18f);   // 2^60; also catches inf / NaN
+        if (__any_sync(0xffffffffu, over)) {
+          load_s();   // S(g) is still in TMEM: reload rather than keep u live
+          if (over) {
+            const float mn = fmaxf(m, tile_max());
+            const float f = tc::ex2(m - mn);
+            l *= f;
+            owe *= f;
+            m = mn;
+          }
+          exps();
+        }
+        tc::tmem_st32(scol, pk);   // P(g) over this warp's own, already read, columns
+        l += lt;
+        // O_h owes `owe` once PV(g-1) is done (factor 1 on rows owing
+        // nothing).  Every phase of the PV barrier inside an item is waited
+        // for, and the item's first task follows the previous item's OFULL,
+        // so the parity always names the one PV in question.
+        if (t > 0) {
+          if (!(ok = wait_warp(bar(B_PVDONE), (uint32_t)(g - 1) & 1u, 10))) break;
+          if (__any_sync(0xffffffffu, owe != 1.f)) {
+            tc::tc_fence_after();
+            rescale_o(owe);
+          }
+        }
+        owe = 1.f;
+        // keep p moderate: when this tile's sum passes 2^16 the reference
+        // moves up by the integer part of log2(sum), an exact power-of-two
+        // rescale (l now; O_h after PV(g), in the next step)
+        if (lt > 65536.f) {
+          const int e = ((int)(__float_as_uint(lt) >> 23) & 0xFF) - 127;
+          const float f = __int_as_float((127 - e) << 23);   // 2^-e
+          l *= f;
+          owe = f;
+          m += (float)e;
+        }
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar(B_PREADY));
+      }
+      if (ok && T > 0)
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_OFULL), (uint32_t)qn & 1u, abort, a.ctrl, 8));
+      if (ok && __any_sync(0xffffffffu, owe != 1.f)) {
+        tc::tc_fence_after();
+        rescale_o(owe);
+        tc::tmem_wait_st();
+      }
+      // merge the two key halves of each row (the two warps of a lane
+      // quarter meet on an mbarrier; a bounded wait, so an aborting partner
+      // cannot strand this warp)
+      cs->xm[slot][half][r] = m;
+      cs->xl[slot][half][r] = l;
+      tc::tc_fence_before();
+      tc::mbar_arrive(bar(B_XREADY + 4 * slot + quarter));
+      if (ok) ok = wait_warp(bar(B_XREADY + 4 * slot + quarter), (uint32_t)(n >> 1) & 1u, 9);
+      if (ok) {
+        tc::tc_fence_after();
+        const float m0 = cs->xm[slot][0][r], m1 = cs->xm[slot][1][r];
+        const float M = fmaxf(m0, m1);
+        const float a0 = m0 == -INFINITY ? 0.f : tc::ex2(m0 - M);
+        const float a1 = m1 == -INFINITY ? 0.f : tc::ex2(m1 - M);
+        const float L = a0 * cs->xl[slot][0][r] + a1 * cs->xl[slot][1][r];
+        const int tok = i * TILE_ROWS + r;
+        const bool store = r < rows_valid;
+        const int dst = store ? (a.perm ? __ldg(a.perm + tok) : tok) : 0;
+        uint4* orow = reinterpret_cast<uint4*>(a.o + ((size_t)bh * a.N + dst) * D + half * (D / 2));
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const float w0 = a0 * inv, w1 = a1 * inv;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t o0[32], o1[32];
+          if (T > 0) {  // warp-uniform: every lane takes part in the loads
+            const uint32_t col = (uint32_t)(half * (D / 2) + 32 * c);
+            tc::tmem_ld32(tmem + lane_off + COL_O + col, o0);
+            tc::tmem_ld32(tmem + lane_off + COL_O + 128u + col, o1);
+            tc::tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o0[e] = o1[e] = 0u;
+          }
+          if (store) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float v[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                v[e] = __uint_as_float(o0[8 * q + e]) * w0 + __uint_as_float(o1[8 * q + e]) * w1;
+              uint4 pv;
+              pv.x = pack_bf16x2(v[0], v[1]);
+              pv.y = pack_bf16x2(v[2], v[3]);
+              pv.z = pack_bf16x2(v[4], v[5]);
+              pv.w = pack_bf16x2(v[6], v[7]);
+              orow[c * 4 + q] = pv;
+            }
           }
         }
       }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (!ok) break;
+      if (lane == 0) tc::mbar_arrive(bar(B_INFO_EMPTY0 + slot));
+      gt += T;
+      if (T > 0) ++qn;
     }
-    tc::tc_fence_before();
   }
   __syncthreads();
   if (warp == WARP_MMA) {
@@ -543,7 +644,7 @@ EncodeTiledFn encode_fn() {
 }
 
 // [BH, rows, D] bf16 tensor, box = 64 channels x 128 rows x 1, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH) {
+bool encode_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)BH};
@@ -555,18 +656,56 @@ bool make_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A tensor map depends only on (pointer, D, rows, BH): the last few encoded
+// maps of each host thread are kept so repeated calls on the same buffers
+// skip the driver's encode.
+struct MapKey {
+  const void* ptr;
+  int D, rows, BH;
+};
+struct MapEntry {
+  MapKey k;
+  CUtensorMap m;
+  bool used;
+};
+
+bool make_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH) {
+  constexpr int SLOTS = 16;
+  thread_local MapEntry cache[SLOTS] = {};
+  thread_local int next = 0;
+  for (int c = 0; c < SLOTS; ++c) {
+    const MapEntry& e = cache[c];
+    if (e.used && e.k.ptr == ptr && e.k.D == D && e.k.rows == rows && e.k.BH == BH) {
+      *m = e.m;
+      return true;
+    }
+  }
+  if (!encode_map(m, ptr, D, rows, BH)) return false;
+  MapEntry& e = cache[next];
+  next = (next + 1) % SLOTS;
+  e.k = MapKey{ptr, D, rows, BH};
+  e.m = *m;
+  e.used = true;
+  return true;
+}
+
 template <int D>
 size_t tc_smem_bytes() {
   return (size_t)(1 + TcCfg<D>::STAGES) * TcCfg<D>::TILE_BYTES + sizeof(TcCtrl) + 1024;
 }
 
 template <int D>
-cudaError_t launch_tc(const CUtensorMap* maps, const TcArgs& a, int items, cudaStream_t s) {
+cudaError_t launch_tc(const CUtensorMap* maps, const TcArgs& a, cudaStream_t s) {
   const size_t smem = tc_smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_dyn_smem((const void*)attn_tc_kernel<D>, smem);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<D><<<items, TC_THREADS, smem, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], a);
+  // persistent: one CTA per SM (shared memory and TMEM admit one), at most
+  // one per work item
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int grid = std::max(1, std::min(a.items, sms));
+  attn_tc_kernel<D><<<grid, TC_THREADS, smem, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], a);
   return cudaGetLastError();
 }
 
@@ -593,8 +732,18 @@ cudaError_t launch_attend_tc(const Problem& p, const void* Q, const void* K, con
   a.ctrl = w.ctrl;
   a.N = p.N; a.nb = p.nb; a.n_last = p.n_last; a.residual = p.residual;
   a.sl2 = 1.4426950408889634f / sqrtf((float)p.d);
-  const int items = p.BH * p.nb;
-  return p.d == 128 ? launch_tc<128>(maps, a, items, s) : launch_tc<64>(maps, a, items, s);
+  a.items = p.BH * p.nb;
+  // The work counter resets itself at the end of every launch; it starts
+  // from zero after the routing call's control-block clear.  A caller CSR
+  // may come with a workspace that was never routed: clear the error word
+  // and the counters.
+  if (row_ptr != w.row_ptr) {
+    static_assert(CTRL_ERROR == 0 && CTRL_ERROR_AUX == 1 && CTRL_WORK == 2 && CTRL_DONE == 3,
+                  "control words cleared together");
+    cudaError_t e = cudaMemsetAsync(w.ctrl, 0, 4 * sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
+  }
+  return p.d == 128 ? launch_tc<128>(maps, a, s) : launch_tc<64>(maps, a, s);
 }
 
 }  // namespace spattn

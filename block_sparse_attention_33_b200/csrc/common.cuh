@@ -14,8 +14,9 @@ enum : int { DEV_OK = 0, DEV_BAD_INDEX = 1, DEV_TIMEOUT = 2 };
 enum : int {
   CTRL_ERROR = 0,      // first device error code seen (atomicCAS from 0)
   CTRL_ERROR_AUX = 1,  // where it happened (kernel specific)
-  CTRL_WORK = 2,       // persistent-kernel work counter
-  CTRL_NNZ = 3,        // total kept blocks of the last route
+  CTRL_WORK = 2,       // persistent attention: next work ticket
+  CTRL_DONE = 3,       // persistent attention: CTAs retired (the last one resets both)
+  CTRL_NNZ = 4,        // total kept blocks of the last route
   CTRL_WORDS = 64
 };
 

@@ -6,15 +6,29 @@
 // in the same pass (DFSAttn abstract: Hilbert reordering before blocking), so
 // Q/K/V are read from HBM exactly once.
 //
-// One CTA per (block j, head bh, tensor); 256 threads.  A thread owns one
-// 16-byte chunk (8 channels) of the row and walks the rows r0, r0+R, ... of
-// the block, accumulating in fp32 in a fixed order; the R partial sums are
-// then reduced in a fixed order too, so the means are bit-reproducible.
+// Persistent CTAs (two per SM), each streaming a strided share of the units
+// (tensor, head, block) through a ring of shared-memory tiles filled by TMA
+// bulk copies: one copy per block (contiguous rows), or one per row through
+// the permutation, issued by the lanes of warp 0.  The permuted copy is
+// written back from the same tile with a bulk store.  A thread owns one
+// 16-byte chunk (8 channels) and sums the rows r0, r0+R, ... of the tile in
+// fp32 in a fixed order; the R partial sums are then added in a fixed order,
+// so the means are bit-reproducible.
+//
+// CTA 0 also clears the workspace control block: this is the first kernel of
+// the routing chain.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 namespace spattn {
 namespace {
+
+constexpr int POOL_THREADS = 256;
+constexpr int POOL_STAGES = 3;
+constexpr int POOL_CTAS_PER_SM = 2;
 
 struct PoolArgs {
   const __nv_bfloat16* X[3];
@@ -22,67 +36,155 @@ struct PoolArgs {
   float* bar[3];           // fp32 means [BH, nb, d]
   __nv_bfloat16* bar16[3]; // bf16 means (K and V only; NULL for Q)
   const int32_t* perm;
-  int N, b, nb, n_last;
+  int32_t* ctrl;           // control block cleared by CTA 0 (NULL: leave it)
+  int N, b, nb, n_last, BH, units;
 };
 
 template <int D>
-__global__ void __launch_bounds__(256) pool_kernel(PoolArgs a) {
-  constexpr int CH = D / 8;          // 16-byte chunks per row
-  constexpr int R = 256 / CH;        // rows in flight per CTA pass
-  constexpr int IT = 128 / R;        // passes for the largest block (b = 128)
-  __shared__ float red[R][D + 4];
+struct PoolGeom {
+  static constexpr int CH = D / 8;              // 16-byte chunks per row
+  static constexpr int R = POOL_THREADS / CH;   // row groups
+};
 
-  const int j = blockIdx.x, bh = blockIdx.y, t = blockIdx.z;
-  const int n = (j == a.nb - 1) ? a.n_last : a.b;
-  const size_t head = (size_t)bh * a.N * D;
+template <int D>
+size_t pool_smem_bytes(int b) {
+  return (size_t)POOL_STAGES * b * D * 2 + (size_t)PoolGeom<D>::R * (D + 4) * 4 +
+         POOL_STAGES * 8 + 16;
+}
+
+template <int D>
+__global__ void __launch_bounds__(POOL_THREADS, POOL_CTAS_PER_SM) pool_kernel(const PoolArgs a) {
+  constexpr int CH = PoolGeom<D>::CH, R = PoolGeom<D>::R;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int row_bytes = D * 2, tile_bytes = a.b * row_bytes;
+  float(*red)[D + 4] = reinterpret_cast<float(*)[D + 4]>(smem + POOL_STAGES * tile_bytes);
+  uint8_t* tail = smem + POOL_STAGES * tile_bytes + R * (D + 4) * 4;
+  uint64_t* fullb = reinterpret_cast<uint64_t*>(tail);
+  volatile int* abort = reinterpret_cast<volatile int*>(tail + POOL_STAGES * 8);
+  const uint32_t ring = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (blockIdx.x == 0 && a.ctrl)
+    for (int q = tid; q < CTRL_WORDS; q += POOL_THREADS) a.ctrl[q] = 0;
+  if (tid == 0) {
+    for (int s = 0; s < POOL_STAGES; ++s) tc::mbar_init(smem_u32(&fullb[s]), 1);
+    *abort = 0;
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int per_head = a.nb, per_tensor = a.BH * a.nb;
+  auto rows_of = [&](int j) { return j == a.nb - 1 ? a.n_last : a.b; };
   // select by branch, not by indexing the parameter arrays (which would copy
   // them to local memory)
-  const __nv_bfloat16* X = (t == 0 ? a.X[0] : t == 1 ? a.X[1] : a.X[2]) + head;
-  __nv_bfloat16* Xp0 = t == 0 ? a.Xp[0] : t == 1 ? a.Xp[1] : a.Xp[2];
-  __nv_bfloat16* Xp = Xp0 ? Xp0 + head : nullptr;
-  float* bar = t == 0 ? a.bar[0] : t == 1 ? a.bar[1] : a.bar[2];
-  __nv_bfloat16* bar16 = t == 0 ? a.bar16[0] : t == 1 ? a.bar16[1] : a.bar16[2];
-  const int c = threadIdx.x % CH, r0 = threadIdx.x / CH;
+  auto src_of = [&](int t) { return t == 0 ? a.X[0] : t == 1 ? a.X[1] : a.X[2]; };
+  const int G = gridDim.x;
+  const int mine = a.units > (int)blockIdx.x ? (a.units - 1 - (int)blockIdx.x) / G + 1 : 0;
 
-  uint4 v[IT];
-#pragma unroll
-  for (int it = 0; it < IT; ++it) {
-    const int r = r0 + it * R;
-    if (r < n) {
-      const int tok = j * a.b + r;
-      const int src = a.perm ? __ldg(a.perm + tok) : tok;
-      v[it] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)src * D) + c);
+  // warp 0: fill ring slot k % STAGES with this CTA's k-th unit
+  int issued = 0;
+  auto issue = [&](int k) {
+    ++issued;
+    const int u = blockIdx.x + k * G;
+    const int t = u / per_tensor, bh = (u % per_tensor) / per_head, j = u % per_head;
+    const int n = rows_of(j);
+    const uint32_t slot = k % POOL_STAGES;
+    const uint32_t fb = smem_u32(&fullb[slot]);
+    const uint32_t dst = ring + slot * tile_bytes;
+    const __nv_bfloat16* X = src_of(t) + (size_t)bh * a.N * D;
+    if (lane == 0) tc::mbar_expect_tx(fb, (uint32_t)(n * row_bytes));
+    __syncwarp();
+    if (!a.perm) {
+      if (lane == 0) tc::bulk_load(dst, X + (size_t)j * a.b * D, (uint32_t)(n * row_bytes), fb);
+    } else {
+      for (int r = lane; r < n; r += 32) {
+        const int src = __ldg(a.perm + j * a.b + r);
+        tc::bulk_load(dst + r * row_bytes, X + (size_t)src * D, (uint32_t)row_bytes, fb);
+      }
     }
-  }
-  float acc[8];
+  };
+  if (warp == 0)
+    for (int k = 0; k < POOL_STAGES && k < mine; ++k) issue(k);
+
+  const int c = tid % CH, r0 = tid / CH;
+  for (int k = 0; k < mine; ++k) {
+    const int u = blockIdx.x + k * G;
+    const int t = u / per_tensor, bh = (u % per_tensor) / per_head, j = u % per_head;
+    const int n = rows_of(j);
+    const uint32_t slot = k % POOL_STAGES;
+    const uint8_t* tile = smem + slot * tile_bytes;
+    const bool ok = tc::mbar_wait(smem_u32(&fullb[slot]), (uint32_t)(k / POOL_STAGES) & 1u, abort,
+                                  a.ctrl, 20);
+    if (!__syncthreads_and(ok)) break;
+    __nv_bfloat16* Xp0 = t == 0 ? a.Xp[0] : t == 1 ? a.Xp[1] : a.Xp[2];
+    if (Xp0 && tid == 0) {
+      tc::bulk_store(Xp0 + ((size_t)bh * a.N + (size_t)j * a.b) * D, ring + slot * tile_bytes,
+                     (uint32_t)(n * row_bytes));
+      tc::bulk_commit();
+    }
+    float acc[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-  for (int it = 0; it < IT; ++it) {
-    const int r = r0 + it * R;
-    if (r < n) {
-      if (Xp) reinterpret_cast<uint4*>(Xp + (size_t)(j * a.b + r) * D)[c] = v[it];
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v[it]);
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int r = r0; r < n; r += R) {
+      const uint4 v = *reinterpret_cast<const uint4*>(tile + r * row_bytes + c * 16);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        float2 f = __bfloat1622float2(h[e]);
+        const float2 f = __bfloat1622float2(h[e]);
         acc[2 * e] += f.x;
         acc[2 * e + 1] += f.y;
       }
     }
-  }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[r0][c * 8 + e] = acc[e];
-  __syncthreads();
-  if (threadIdx.x < D) {
-    float s = 0.f;
+    for (int e = 0; e < 8; ++e) red[r0][c * 8 + e] = acc[e];
+    __syncthreads();
+    // the slot has been read (and, with a permutation, its bulk store has
+    // read it once thread 0 has waited): refill it
+    if (warp == 0) {
+      if (Xp0 && lane == 0) tc::bulk_wait_read_all();
+      __syncwarp();
+      if (k + POOL_STAGES < mine) issue(k + POOL_STAGES);
+    }
+    if (tid < D) {
+      float s = 0.f;
 #pragma unroll 8
-    for (int q = 0; q < R; ++q) s += red[q][threadIdx.x];
-    const float mean = s / (float)n;
-    const size_t o = ((size_t)bh * a.nb + j) * D + threadIdx.x;
-    bar[o] = mean;
-    if (bar16) bar16[o] = __float2bfloat16_rn(mean);
+      for (int q = 0; q < R; ++q) s += red[q][tid];
+      const float mean = s / (float)n;
+      const size_t o = ((size_t)bh * a.nb + j) * D + tid;
+      float* bar = t == 0 ? a.bar[0] : t == 1 ? a.bar[1] : a.bar[2];
+      __nv_bfloat16* bar16 = t == 0 ? a.bar16[0] : t == 1 ? a.bar16[1] : a.bar16[2];
+      bar[o] = mean;
+      if (bar16) bar16[o] = __float2bfloat16_rn(mean);
+    }
+    __syncthreads();
   }
+  if (*abort && warp == 0) {
+    // let the copies already issued land before the CTA can exit
+    for (int kk = issued > POOL_STAGES ? issued - POOL_STAGES : 0; kk < issued; ++kk)
+      tc::mbar_drain(smem_u32(&fullb[kk % POOL_STAGES]), (uint32_t)(kk / POOL_STAGES) & 1u);
+  }
+  if (tid == 0) tc::bulk_wait_all();   // permuted copies complete before exit
+}
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+template <int D>
+cudaError_t launch_pool_d(const PoolArgs& a, cudaStream_t s) {
+  const size_t smem = pool_smem_bytes<D>(a.b);
+  cudaError_t e = ensure_dyn_smem((const void*)pool_kernel<D>, smem);
+  if (e != cudaSuccess) return e;
+  const int grid = std::max(1, std::min(a.units, POOL_CTAS_PER_SM * sm_count()));
+  pool_kernel<D><<<grid, POOL_THREADS, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pool_any(const Problem& p, const PoolArgs& a, cudaStream_t s) {
+  return p.d == 128 ? launch_pool_d<128>(a, s) : launch_pool_d<64>(a, s);
 }
 
 }  // namespace
@@ -97,17 +199,16 @@ cudaError_t launch_pool(const Problem& p, const void* Q, const void* K, const vo
   a.bar[0] = w.qbar; a.bar[1] = w.kbar; a.bar[2] = w.vbar;
   a.bar16[0] = nullptr; a.bar16[1] = w.kbar16; a.bar16[2] = w.vbar16;
   a.perm = p.perm;
-  a.N = p.N; a.b = p.b; a.nb = p.nb; a.n_last = p.n_last;
-  dim3 grid(p.nb, p.BH, 3);
-  if (p.d == 128) pool_kernel<128><<<grid, 256, 0, s>>>(a);
-  else pool_kernel<64><<<grid, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  a.ctrl = w.ctrl;
+  a.N = p.N; a.b = p.b; a.nb = p.nb; a.n_last = p.n_last; a.BH = p.BH;
+  a.units = 3 * p.BH * p.nb;
+  return launch_pool_any(p, a, s);
 }
 
-// Means of Q and K only (grid z = 2), no bf16 copies and no permuted copies:
-// what the routing step needs, for callers that keep no other scratch.
+// Means of Q and K only, no bf16 copies and no permuted copies: what the
+// routing step needs, for callers that keep no other scratch.
 cudaError_t launch_pool_qk(const Problem& p, const void* Q, const void* K, float* qbar,
-                           float* kbar, cudaStream_t s) {
+                           float* kbar, int32_t* ctrl, cudaStream_t s) {
   PoolArgs a;
   a.X[0] = static_cast<const __nv_bfloat16*>(Q);
   a.X[1] = static_cast<const __nv_bfloat16*>(K);
@@ -116,11 +217,10 @@ cudaError_t launch_pool_qk(const Problem& p, const void* Q, const void* K, float
   a.bar[0] = qbar; a.bar[1] = kbar; a.bar[2] = nullptr;
   a.bar16[0] = a.bar16[1] = a.bar16[2] = nullptr;
   a.perm = p.perm;
-  a.N = p.N; a.b = p.b; a.nb = p.nb; a.n_last = p.n_last;
-  dim3 grid(p.nb, p.BH, 2);
-  if (p.d == 128) pool_kernel<128><<<grid, 256, 0, s>>>(a);
-  else pool_kernel<64><<<grid, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  a.ctrl = ctrl;
+  a.N = p.N; a.b = p.b; a.nb = p.nb; a.n_last = p.n_last; a.BH = p.BH;
+  a.units = 2 * p.BH * p.nb;
+  return launch_pool_any(p, a, s);
 }
 
 }  // namespace spattn

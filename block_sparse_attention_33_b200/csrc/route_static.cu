@@ -27,7 +27,7 @@
 
 namespace spattn {
 cudaError_t launch_pool_qk(const Problem& p, const void* Q, const void* K, float* qbar,
-                           float* kbar, cudaStream_t s);
+                           float* kbar, int32_t* ctrl, cudaStream_t s);
 void record_error(const char* msg);  // the message spattn_last_error() returns
 }
 
@@ -127,8 +127,8 @@ extern "C" spattn_status_t spattn_route_static(int B, int H, int N, int d, int b
   w.col_idx = col_idx;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(w.ctrl, 0, spattn::CTRL_WORDS * sizeof(int32_t), s);
-  if (e == cudaSuccess) e = spattn::launch_pool_qk(p, Q, K, w.qbar, w.kbar, s);
+  // the pooling kernel also clears the control block
+  cudaError_t e = spattn::launch_pool_qk(p, Q, K, w.qbar, w.kbar, w.ctrl, s);
   if (e == cudaSuccess) e = spattn::launch_route(p, w, nullptr, nullptr, s);
   if (e != cudaSuccess) return fail(SPATTN_ERR_CUDA, "routing kernels: %s", cudaGetErrorString(e));
   return SPATTN_OK;

@@ -41,7 +41,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait for the phase of parity `parity` to complete.  Gives up (returns
 // false) when another role has aborted, or after WAIT_LIMIT_CYCLES, in which
 // case it records DEV_TIMEOUT with `site` and raises the CTA's abort flag.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                        int32_t* ctrl, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
@@ -69,6 +69,30 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   while (!mbar_try_wait(bar, parity) && clock64() - t0 < WAIT_LIMIT_CYCLES / 8) {
   }
 }
+
+// Untiled bulk copy global -> shared (TMA engine, no multicast), completing
+// `bytes` on mbarrier `bar`.  Both addresses 16-byte aligned, bytes a
+// multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+// Untiled bulk copy shared -> global, tracked by the issuing thread's bulk
+// groups.
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(dst), "r"(src),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// Wait until the shared-memory source of every committed bulk store has been read.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+}
+// Wait until every committed bulk store has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 
 // 3D tiled TMA load (no multicast) completing on mbarrier `bar`.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,

@@ -94,7 +94,8 @@ spattn_status_t spattn_pool(spattn_plan_t plan, const void* Q, const void* K, co
                             void* workspace, void* stream);
 
 /* spattn_pool, then proxy scoring, Top-p selection and the CSR
- * of kept blocks.
+ * of kept blocks.  spattn_pool and spattn_route clear the workspace's
+ * device error word first.
  *   row_ptr  NULL or int32 [B*H*nb + 1], rows ordered (batch, head, block i);
  *   col_idx  NULL or int32 [col capacity], kept block indices j in [0, nb),
  *            ascending within a row.
@@ -109,7 +110,12 @@ spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, c
  *   row_ptr, col_idx  NULL to use the workspace CSR of the last route, or a
  *                     caller CSR in the layout above (device).  Block
  *                     indices outside [0, nb) are skipped and flagged
- *                     (SPATTN_ERR_DEVICE from spattn_check).
+ *                     (SPATTN_ERR_DEVICE from spattn_check).  With a
+ *                     caller CSR the call first clears the workspace's
+ *                     device error word (the workspace may never have
+ *                     been routed); without a permutation and with
+ *                     residual = 0 it then needs nothing else from an
+ *                     earlier call.
  *   O                 bf16 [B, H, N, d] device, written in the original
  *                     token order. */
 spattn_status_t spattn_attend(spattn_plan_t plan, const void* Q, const void* K, const void* V,

@@ -77,3 +77,80 @@ def test_tc_hilbert_stress_shape_small():
     rows = {(0, h): np.arange(0, w.N, 97) for h in range(w.H)}
     fig = oracle_check(w, Q, K, V, res, perm=perm, rows={k: perm[v] for k, v in rows.items()})
     assert fig["bad"] == 0 and fig["max_abs"] < MAX_ABS and fig["rel_l2"] < REL_L2, fig
+
+
+# ---- the persistent work loop: more items than SMs, items without tasks,
+# ---- the self-resetting work counter
+
+def _oracle_csr(w, Q, K, V):
+    from oracle import spattn_ref as R
+    from tests.harness import kept_to_csr
+    ref = R.forward(Q, K, V, w.b, w.tau, w.kmin, w.kmax, w.residual, want_output=False)
+    return {key: [np.asarray(x) for x in r["kept"]] for key, r in ref["route"].items()}
+
+
+def test_tc_caller_csr_with_empty_rows_on_unrouted_workspace():
+    """Caller CSR in which every 5th query block keeps nothing, no residual
+    (those items have no tasks and must come out as zeros), on a workspace
+    that was never routed and holds garbage: the attention call clears its
+    own work counter.  256 items, more than the SMs, so CTAs loop."""
+    import torch
+    import block_sparse_attention_33_b200 as sp
+    from oracle import spattn_ref as R
+    from tests.harness import from_dev, kept_to_csr, to_dev
+    w = get_config("medium", H=4, residual=0, tau=0.7)
+    Q, K, V = make_qkv(w)
+    kept = _oracle_csr(w, Q, K, V)
+    empty = {(0, h): [i for i in range(w.nb) if (i + h) % 5 == 0] for h in range(w.H)}
+    for key, blocks in empty.items():
+        for i in blocks:
+            kept[key][i] = np.zeros(0, np.int64)
+    rp, ci = kept_to_csr(kept, w.B, w.H, w.nb)
+    plan = sp.Plan(w.B, w.H, w.N, w.d, w.b, w.tau, w.kmin, w.kmax, w.residual)
+    try:
+        plan.workspace.fill_(0x7F)                       # never routed: garbage control words
+        q, k, v = to_dev(Q), to_dev(K), to_dev(V)
+        o = torch.full_like(q, 3.0)
+        plan.attend(q, k, v, o, torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda())
+        assert plan.check() == 0
+        O = from_dev(o)
+    finally:
+        plan.close()
+    b = w.b
+    rows = {}
+    for h in range(w.H):
+        keep_blocks = [i for i in range(w.nb) if (i + h) % 5 != 0]
+        rows[(0, h)] = np.concatenate([np.arange(i * b, i * b + b, 7) for i in keep_blocks])
+        for i in empty[(0, h)]:
+            assert np.all(O[0, h, i * b:(i + 1) * b] == 0.0), (h, i)
+    ref = R.forward(Q, K, V, w.b, w.tau, w.kmin, w.kmax, w.residual, rows=rows, kept_override=kept)
+    got = np.concatenate([O[0, h, rows[(0, h)]] for h in range(w.H)])
+    want = np.concatenate([ref["O"][(0, h)] for h in range(w.H)])
+    max_abs, rel = compare_outputs(got, want)
+    assert max_abs < MAX_ABS and rel < REL_L2, (max_abs, rel)
+
+
+def test_tc_repeated_attend_is_bitwise_stable():
+    """Three attention calls after one routing call: the work counter resets
+    itself at the end of each launch, and an item's output does not depend on
+    which CTA ran it."""
+    import torch
+    import block_sparse_attention_33_b200 as sp
+    from tests.harness import to_dev
+    w = get_config("medium", H=4)
+    Q, K, V = make_qkv(w)
+    plan = sp.Plan(w.B, w.H, w.N, w.d, w.b, w.tau, w.kmin, w.kmax, w.residual)
+    try:
+        q, k, v = to_dev(Q), to_dev(K), to_dev(V)
+        plan.route(q, k, v)
+        outs = []
+        for _ in range(3):
+            o = torch.zeros_like(q)
+            plan.attend(q, k, v, o)
+            outs.append(o)
+        assert plan.check() == 0
+        torch.cuda.synchronize()
+    finally:
+        plan.close()
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    assert torch.equal(outs[0].view(torch.int16), outs[2].view(torch.int16))
