@@ -37,7 +37,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 KERNELS_PER_STEP = 5  # pool, route, scan, compact, attend
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
@@ -54,7 +54,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="CPU time budget of the oracle baseline sample")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def load_peaks():
@@ -80,6 +80,30 @@ def workload_from_args(args, rank=0):
     if rank:
         w = w.with_(seed=w.seed + 1000 * rank)   # independent replica per rank
     return w
+
+
+def combine_over_ranks(maxes, sums, device):
+    """Every rank's timings (max over ranks: the job ends with its slowest
+    replica) and work (summed over ranks).  One all-reduce per kind, the same
+    on every rank; returns (maxes, sums) as lists of floats."""
+    import torch
+    import torch.distributed as dist
+    out_max, out_sum = list(maxes), list(sums)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if maxes:
+            t = torch.tensor(maxes, dtype=torch.float64, device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            out_max = t.tolist()
+        if sums:
+            t = torch.tensor(sums, dtype=torch.float64, device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.SUM)
+            out_sum = t.tolist()
+    return out_max, out_sum
+
+
+def job_throughput(total_flops, step_ms):
+    """Whole-job TFLOP/s: all ranks' FLOPs over the slowest rank's step time."""
+    return total_flops / (step_ms * 1e-3) / 1e12
 
 
 def attention_flops(row_ptr, col_idx, w, nb):
@@ -327,18 +351,10 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device status {status}: {sp.spattn_last_error()}")
 
-    # max over ranks of the step time (device-timed)
-    if world > 1:
-        tt = torch.tensor([step_ms, attend_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        step_ms, attend_ms = tt.tolist()
-        ff = torch.tensor([float(step_flops)], device=dev, dtype=torch.float64)
-        dist.all_reduce(ff)
-        total_flops = ff.item()
-    else:
-        total_flops = float(step_flops)
-
-    value = total_flops / (step_ms * 1e-3) / 1e12
+    # max over ranks of the step time (device-timed), work summed over ranks
+    (step_ms, attend_ms), (total_flops,) = combine_over_ranks([step_ms, attend_ms],
+                                                              [float(step_flops)], dev)
+    value = job_throughput(total_flops, step_ms)
     peaks, peak_kind = load_peaks()
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
@@ -350,10 +366,7 @@ def run_ours(args):
         dplan = sp.Plan(B, H, N, d, w.b, 1.0, 1, 1 << 30, w.residual, perm, device=dev)
         td = timed([lambda: dplan.forward(q, k, v, o)], max(3, args.steps // 3), 2)
         dense_ms = float(np.mean([x[0] for x in td]))
-        if world > 1:
-            tt = torch.tensor([dense_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            dense_ms = tt.item()
+        (dense_ms,), _ = combine_over_ranks([dense_ms], [], dev)
         dplan.close()
 
     # kernel breakdown: the pooling kernel alone (HBM-bound)
@@ -380,10 +393,7 @@ def run_ours(args):
 
         te = timed([e2e_step], max(3, args.steps // 3), 2)
         e2e_ms = float(np.mean([x[0] for x in te]))
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = tt.item()
+        (e2e_ms,), _ = combine_over_ranks([e2e_ms], [], dev)
         e2e = {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * tok_bytes,
                "d2h_bytes_per_step": tok_bytes}
