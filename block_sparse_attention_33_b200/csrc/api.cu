@@ -244,7 +244,8 @@ spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, c
   // the pooling kernel also clears the control block
   cudaError_t e = spattn::launch_pool(plan->p, Q, K, V, w, s);
   if (e != cudaSuccess) return cuda_fail(e, "pool kernel");
-  e = spattn::launch_route(plan->p, w, row_ptr, col_idx, s);
+  // the warp-MMA attention reads the compact CSR of the workspace
+  e = spattn::launch_route(plan->p, w, row_ptr, col_idx, !plan->p.use_tc, s);
   if (e != cudaSuccess) return cuda_fail(e, "route kernels");
   return SPATTN_OK;
 }

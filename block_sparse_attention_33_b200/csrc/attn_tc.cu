@@ -93,7 +93,11 @@ enum : int {
 };
 
 struct TcArgs {
-  const int32_t *row_ptr, *col_idx, *order, *perm;
+  // kept blocks of an item: the compact CSR (row_ptr, col_idx), or, with
+  // counts set, the padded per-row lists of the routing step
+  // (counts[item] entries at col_idx + item * kcap)
+  const int32_t *row_ptr, *col_idx, *counts, *order, *perm;
+  int kcap;
   __nv_bfloat16* o;
   int32_t* ctrl;
   int N, nb, n_last, residual, items;
@@ -204,8 +208,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       const int item = a.order ? __ldg(a.order + ticket) : ticket;
       const int bh = item / a.nb, i = item % a.nb;
-      const int r_lo = __ldg(a.row_ptr + item);
-      const int nkept = max(0, __ldg(a.row_ptr + item + 1) - r_lo);
+      const int r_lo = a.counts ? item * a.kcap : __ldg(a.row_ptr + item);
+      const int nkept = a.counts ? __ldg(a.counts + item) : max(0, __ldg(a.row_ptr + item + 1) - r_lo);
       inf.kept[lane] = 0u;
       inf.kept[lane + 32] = 0u;
       inf.bad[lane] = 0u;
@@ -725,8 +729,14 @@ cudaError_t launch_attend_tc(const Problem& p, const void* Q, const void* K, con
       !make_map(&maps[4], w.vbar16, p.d, p.nb, p.BH))
     return cudaErrorInvalidValue;
   TcArgs a;
-  a.row_ptr = row_ptr; a.col_idx = col_idx;
-  a.order = (row_ptr == w.row_ptr) ? w.order : nullptr;
+  if (row_ptr == w.row_ptr) {
+    // the workspace's own routing result: padded lists, longest-first order
+    a.row_ptr = nullptr; a.col_idx = w.lists; a.counts = w.counts; a.kcap = p.kcap;
+    a.order = w.order;
+  } else {
+    a.row_ptr = row_ptr; a.col_idx = col_idx; a.counts = nullptr; a.kcap = 0;
+    a.order = nullptr;
+  }
   a.perm = p.perm;
   a.o = static_cast<__nv_bfloat16*>(O);
   a.ctrl = w.ctrl;

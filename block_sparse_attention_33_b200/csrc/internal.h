@@ -34,8 +34,11 @@ struct Work {
 
 cudaError_t launch_pool(const Problem& p, const void* Q, const void* K, const void* V,
                         const Work& w, cudaStream_t s);
+// need_csr: also build the compact CSR in w.row_ptr / w.col_idx (the
+// tcgen05 attention reads the padded per-row lists directly, so the compact
+// copy is made only for callers and paths that need it).
 cudaError_t launch_route(const Problem& p, const Work& w, int32_t* row_ptr_out,
-                         int32_t* col_idx_out, cudaStream_t s);
+                         int32_t* col_idx_out, bool need_csr, cudaStream_t s);
 cudaError_t launch_attend(const Problem& p, const void* Q, const void* K, const void* V,
                           const int32_t* row_ptr, const int32_t* col_idx, void* O,
                           const Work& w, cudaStream_t s);

@@ -78,6 +78,54 @@ __device__ __forceinline__ int count_equal(const float* p, int nb, uint32_t u) {
   return warp_sum_i(c);
 }
 
+// Smallest u in [lo, hi] with pred(u) true, for pred monotone in u (false
+// ... false true ... true) and pred(hi) true; warp-uniform result.  Each
+// round the 32 lanes test 32 evenly spaced candidates and the range shrinks
+// 32-fold, so 2^30 candidates need 6 rounds.  pred is evaluated by one lane
+// alone (a full pass over the row), which suits short rows.
+template <typename Pred>
+__device__ __forceinline__ uint32_t search32(uint32_t lo, uint32_t hi, Pred pred) {
+  const int lane = threadIdx.x & 31;
+  while (lo < hi) {
+    const uint32_t span = hi - lo;                    // candidates lo .. hi - 1 undecided
+    const uint32_t step = span / 32 + 1;
+    const uint32_t u = lo + (uint32_t)lane * step;
+    const bool in = u < hi;
+    const unsigned yes = __ballot_sync(0xffffffffu, in && pred(u));
+    const unsigned cand = __ballot_sync(0xffffffffu, in);
+    if (yes == 0u) {
+      // every tested candidate is false: the answer is above the last one
+      const int last = 31 - __clz(cand);
+      lo = lo + (uint32_t)last * step + 1;
+    } else {
+      const int first = __ffs(yes) - 1;
+      const uint32_t uf = lo + (uint32_t)first * step;
+      if (first == 0) return uf;                      // pred(lo) holds
+      lo = lo + (uint32_t)(first - 1) * step + 1;
+      hi = uf;
+    }
+  }
+  return lo;
+}
+
+// Mass / count of the blocks whose probability bits exceed u, by one lane.
+__device__ __forceinline__ float mass_above_1(const float* p, int nb, uint32_t u) {
+  float s = 0.f;
+  for (int j = 0; j < nb; ++j) {
+    const float x = p[j];
+    s += (__float_as_uint(x) > u) ? x : 0.f;
+  }
+  return s;
+}
+__device__ __forceinline__ int count_above_1(const float* p, int nb, uint32_t u) {
+  int c = 0;
+  for (int j = 0; j < nb; ++j) c += (__float_as_uint(p[j]) > u) ? 1 : 0;
+  return c;
+}
+
+// rows with at most this many blocks use the 32-way search
+constexpr int SEARCH32_MAX_NB = 128;
+
 template <int D, int RT_ROWS>
 __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
   extern __shared__ __align__(16) float sm[];
@@ -93,29 +141,43 @@ __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
     Qs[e] = (e / D < rows) ? qbar[e] : 0.f;
   __syncthreads();
 
-  // ---- proxy logits: thread owns key block j, all 16 query rows ----
+  // ---- proxy logits: a group of TPJ threads owns key block j (all rows),
+  // each thread a strided share of the channels, reduced with shuffles;
+  // TPJ = 256 / nb (at most 32) keeps every thread busy when nb is small
   const float inv_sqrt_d = 1.0f / sqrtf((float)D);
-  for (int j = threadIdx.x; j < a.nb; j += RT_THREADS) {
+  const int tpj = a.nb >= RT_THREADS ? 1 : (a.nb >= 128 ? 2 : (a.nb >= 64 ? 4 : (a.nb >= 32 ? 8 : 16)));
+  const int sub = threadIdx.x % tpj, grp = threadIdx.x / tpj, ngrp = RT_THREADS / tpj;
+  for (int j0 = 0; j0 < a.nb; j0 += ngrp) {
+    const int j = j0 + grp;
+    const bool live = j < a.nb;
     float acc[RT_ROWS];
 #pragma unroll
     for (int r = 0; r < RT_ROWS; ++r) acc[r] = 0.f;
-    const float4* kr = reinterpret_cast<const float4*>(kbar + (size_t)j * D);
+    if (live) {
+      const float4* kr = reinterpret_cast<const float4*>(kbar + (size_t)j * D);
 #pragma unroll 4
-    for (int k4 = 0; k4 < D / 4; ++k4) {
-      const float4 kv = __ldg(kr + k4);
+      for (int k4 = sub; k4 < D / 4; k4 += tpj) {
+        const float4 kv = __ldg(kr + k4);
 #pragma unroll
-      for (int r = 0; r < RT_ROWS; ++r) {
-        const float4 q = reinterpret_cast<const float4*>(Qs + r * D)[k4];
-        acc[r] = fmaf(q.x, kv.x, acc[r]);
-        acc[r] = fmaf(q.y, kv.y, acc[r]);
-        acc[r] = fmaf(q.z, kv.z, acc[r]);
-        acc[r] = fmaf(q.w, kv.w, acc[r]);
+        for (int r = 0; r < RT_ROWS; ++r) {
+          const float4 q = reinterpret_cast<const float4*>(Qs + r * D)[k4];
+          acc[r] = fmaf(q.x, kv.x, acc[r]);
+          acc[r] = fmaf(q.y, kv.y, acc[r]);
+          acc[r] = fmaf(q.z, kv.z, acc[r]);
+          acc[r] = fmaf(q.w, kv.w, acc[r]);
+        }
       }
     }
-    const int nj = (j == a.nb - 1) ? a.n_last : a.b;
-    const float lnn = logf((float)nj);
+    // fixed-order tree over the group's lanes (groups are aligned within a warp)
+    for (int o = 1; o < tpj; o <<= 1)
 #pragma unroll
-    for (int r = 0; r < RT_ROWS; ++r) S[r * nbp + j] = fmaf(acc[r], inv_sqrt_d, lnn);
+      for (int r = 0; r < RT_ROWS; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], o);
+    if (live && sub == 0) {
+      const int nj = (j == a.nb - 1) ? a.n_last : a.b;
+      const float lnn = logf((float)nj);
+#pragma unroll
+      for (int r = 0; r < RT_ROWS; ++r) S[r * nbp + j] = fmaf(acc[r], inv_sqrt_d, lnn);
+    }
   }
   __syncthreads();
 
@@ -143,13 +205,18 @@ __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
     if (a.tau >= 1.0f) {
       kstar = a.nb;               // tau >= 1 keeps every block
     } else if (a.tau > 0.0f) {
-      uint32_t lo = 0, hi = 0x3F800000u;  // p <= 1, so nothing is above hi
-      while (lo < hi) {
-        const uint32_t mid = lo + ((hi - lo) >> 1);
-        if (mass_above(p, a.nb, mid) < a.tau) hi = mid; else lo = mid + 1;
+      if (a.nb <= SEARCH32_MAX_NB) {
+        thr = search32(0u, 0x3F800000u, [&](uint32_t u) { return mass_above_1(p, a.nb, u) < a.tau; });
+      } else {
+        uint32_t lo = 0, hi = 0x3F800000u;  // p <= 1, so nothing is above hi
+        while (lo < hi) {
+          const uint32_t mid = lo + ((hi - lo) >> 1);
+          if (mass_above(p, a.nb, mid) < a.tau) hi = mid; else lo = mid + 1;
+        }
+        thr = lo;
       }
-      thr = lo;
-      const float g = mass_above(p, a.nb, thr);
+      // the same summation as the search's predicate
+      const float g = a.nb <= SEARCH32_MAX_NB ? mass_above_1(p, a.nb, thr) : mass_above(p, a.nb, thr);
       const int gt = count_above(p, a.nb, thr);
       const int eq = count_equal(p, a.nb, thr);
       const float v = __uint_as_float(thr);
@@ -164,12 +231,16 @@ __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
     const bool all = (k >= a.nb);
     if (!all && !(by_mass && k == kstar)) {
       // the clamp binds (or tau <= 0): top-k in (p desc, j asc) order
-      uint32_t lo = 0, hi = 0x3F800000u;
-      while (lo < hi) {
-        const uint32_t mid = lo + ((hi - lo) >> 1);
-        if (count_above(p, a.nb, mid) < k) hi = mid; else lo = mid + 1;
+      if (a.nb <= SEARCH32_MAX_NB) {
+        thr = search32(0u, 0x3F800000u, [&](uint32_t u) { return count_above_1(p, a.nb, u) < k; });
+      } else {
+        uint32_t lo = 0, hi = 0x3F800000u;
+        while (lo < hi) {
+          const uint32_t mid = lo + ((hi - lo) >> 1);
+          if (count_above(p, a.nb, mid) < k) hi = mid; else lo = mid + 1;
+        }
+        thr = lo;
       }
-      thr = lo;
       ties = k - count_above(p, a.nb, thr);
     }
     const int row = bh * a.nb + i0 + r;
@@ -328,7 +399,7 @@ static int scan_group_rows(const Problem& p) {
 }
 
 cudaError_t launch_route(const Problem& p, const Work& w, int32_t* row_ptr_out,
-                         int32_t* col_idx_out, cudaStream_t s) {
+                         int32_t* col_idx_out, bool need_csr, cudaStream_t s) {
   RouteArgs a;
   a.qbar = w.qbar; a.kbar = w.kbar; a.counts = w.counts; a.lists = w.lists;
   a.nb = p.nb; a.b = p.b; a.n_last = p.n_last; a.kcap = p.kcap; a.kmin = p.kmin;
@@ -344,6 +415,7 @@ cudaError_t launch_route(const Problem& p, const Work& w, int32_t* row_ptr_out,
   scan_kernel<<<1, SCAN_THREADS, hist_bytes, s>>>(w.counts, rows, p.kcap, group_rows, w.row_ptr,
                                                   w.order, w.ctrl);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (!need_csr && !row_ptr_out && !col_idx_out) return cudaSuccess;
   compact_kernel<<<(rows + 7) / 8, 256, 0, s>>>(w.counts, w.lists, w.row_ptr, rows, p.kcap,
                                                 w.col_idx, row_ptr_out, col_idx_out);
   return cudaGetLastError();

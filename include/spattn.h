@@ -99,7 +99,8 @@ spattn_status_t spattn_pool(spattn_plan_t plan, const void* Q, const void* K, co
  *   row_ptr  NULL or int32 [B*H*nb + 1], rows ordered (batch, head, block i);
  *   col_idx  NULL or int32 [col capacity], kept block indices j in [0, nb),
  *            ascending within a row.
- * The CSR is always also kept in the workspace for a following attend. */
+ * The kept lists are always also left in the workspace (padded per row)
+ * for a following attend. */
 spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, const void* V,
                              void* workspace, int32_t* row_ptr, int32_t* col_idx,
                              void* stream);
