@@ -6,11 +6,12 @@
 // in the same pass (DFSAttn abstract: Hilbert reordering before blocking), so
 // Q/K/V are read from HBM exactly once.
 //
-// Persistent CTAs (two per SM), each streaming a strided share of the units
-// (tensor, head, block) through a ring of shared-memory tiles filled by TMA
-// bulk copies: one copy per block (contiguous rows), or one per row through
-// the permutation, issued by the lanes of warp 0.  The permuted copy is
-// written back from the same tile with a bulk store.  A thread owns one
+// Persistent CTAs (two per SM), each taking a strided share of the units
+// (tensor, head, block).  Without a permutation a unit's rows are contiguous
+// and stream through a ring of shared-memory tiles filled by one TMA bulk
+// copy each (pool_kernel).  With a permutation the rows are gathered with
+// 16-byte loads into registers, one unit ahead (pool_gather_kernel), and the
+// permuted copy is written from the same registers.  A thread owns one
 // 16-byte chunk (8 channels) and sums the rows r0, r0+R, ... of the tile in
 // fp32 in a fixed order; the R partial sums are then added in a fixed order,
 // so the means are bit-reproducible.
@@ -166,6 +167,83 @@ __global__ void __launch_bounds__(POOL_THREADS, POOL_CTAS_PER_SM) pool_kernel(co
   if (tid == 0) tc::bulk_wait_all();   // permuted copies complete before exit
 }
 
+// Gather form for a permutation: rows are scattered, so each thread loads its
+// share of a unit's rows with 16-byte loads straight into registers (no
+// per-row copy setup), writes the permuted copy from them and sums them.
+// The next unit's rows are loaded before the current unit is reduced, so
+// every SM keeps two units of loads in flight.
+template <int D>
+__global__ void __launch_bounds__(POOL_THREADS, POOL_CTAS_PER_SM) pool_gather_kernel(const PoolArgs a) {
+  constexpr int CH = PoolGeom<D>::CH, R = PoolGeom<D>::R;
+  constexpr int IT = 128 / R;                 // row passes for a 128-token block
+  __shared__ float red[R][D + 4];
+  const int tid = threadIdx.x;
+  if (blockIdx.x == 0 && a.ctrl)
+    for (int q = tid; q < CTRL_WORDS; q += POOL_THREADS) a.ctrl[q] = 0;
+  const int per_head = a.nb, per_tensor = a.BH * a.nb;
+  const int c = tid % CH, r0 = tid / CH;
+  const int G = gridDim.x;
+  auto rows_of = [&](int j) { return j == a.nb - 1 ? a.n_last : a.b; };
+
+  uint4 cur[IT], nxt[IT];
+  auto load = [&](int u, uint4 (&v)[IT]) {
+    const int t = u / per_tensor, bh = (u % per_tensor) / per_head, j = u % per_head;
+    const int n = rows_of(j);
+    const __nv_bfloat16* X = (t == 0 ? a.X[0] : t == 1 ? a.X[1] : a.X[2]) + (size_t)bh * a.N * D;
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int r = r0 + it * R;
+      if (r < n) {
+        const int src = __ldg(a.perm + j * a.b + r);
+        v[it] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)src * D) + c);
+      }
+    }
+  };
+  int u = blockIdx.x;
+  if (u < a.units) load(u, cur);
+  for (; u < a.units; u += G) {
+    const int un = u + G;
+    if (un < a.units) load(un, nxt);
+    const int t = u / per_tensor, bh = (u % per_tensor) / per_head, j = u % per_head;
+    const int n = rows_of(j);
+    __nv_bfloat16* Xp = t == 0 ? a.Xp[0] : t == 1 ? a.Xp[1] : a.Xp[2];
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int r = r0 + it * R;
+      if (r < n) {
+        if (Xp) reinterpret_cast<uint4*>(Xp + ((size_t)bh * a.N + (size_t)j * a.b + r) * D)[c] = cur[it];
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&cur[it]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h[e]);
+          acc[2 * e] += f.x;
+          acc[2 * e + 1] += f.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[r0][c * 8 + e] = acc[e];
+    __syncthreads();
+    if (tid < D) {
+      float s = 0.f;
+#pragma unroll 8
+      for (int q = 0; q < R; ++q) s += red[q][tid];
+      const float mean = s / (float)n;
+      const size_t o = ((size_t)bh * a.nb + j) * D + tid;
+      float* bar = t == 0 ? a.bar[0] : t == 1 ? a.bar[1] : a.bar[2];
+      __nv_bfloat16* bar16 = t == 0 ? a.bar16[0] : t == 1 ? a.bar16[1] : a.bar16[2];
+      bar[o] = mean;
+      if (bar16) bar16[o] = __float2bfloat16_rn(mean);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int it = 0; it < IT; ++it) cur[it] = nxt[it];
+  }
+}
+
 int sm_count() {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -175,6 +253,11 @@ int sm_count() {
 
 template <int D>
 cudaError_t launch_pool_d(const PoolArgs& a, cudaStream_t s) {
+  if (a.perm) {
+    const int grid = std::max(1, std::min(a.units, POOL_CTAS_PER_SM * sm_count()));
+    pool_gather_kernel<D><<<grid, POOL_THREADS, 0, s>>>(a);
+    return cudaGetLastError();
+  }
   const size_t smem = pool_smem_bytes<D>(a.b);
   cudaError_t e = ensure_dyn_smem((const void*)pool_kernel<D>, smem);
   if (e != cudaSuccess) return e;
