@@ -271,16 +271,33 @@ __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
 // group * (kcap + 1) + (kcap - count).
 constexpr int SCAN_THREADS = 1024;
 
+// Exclusive prefix sum over the CTA's threads (SCAN_THREADS = 32 warps):
+// shuffle scans inside each warp, one warp scans the warp totals.  `part`
+// holds 32 ints; the trailing barrier lets the caller reuse it at once.
 __device__ __forceinline__ int block_exclusive_scan(int v, int* part) {
-  part[threadIdx.x] = v;
-  __syncthreads();
-  for (int off = 1; off < SCAN_THREADS; off <<= 1) {
-    const int u = threadIdx.x >= off ? part[threadIdx.x - off] : 0;
-    __syncthreads();
-    part[threadIdx.x] += u;
-    __syncthreads();
+  static_assert(SCAN_THREADS == 1024, "one warp scans the 32 warp totals");
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  const int ex = threadIdx.x ? part[threadIdx.x - 1] : 0;
+  if (lane == 31) part[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = part[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    part[lane] = wi - w;
+  }
+  __syncthreads();
+  const int ex = part[warp] + x - v;
+  __syncthreads();
   return ex;
 }
 
@@ -288,7 +305,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(const int32_t* count
                                                             int kcap, int group_rows,
                                                             int32_t* row_ptr, int32_t* order,
                                                             int32_t* ctrl) {
-  __shared__ int part[SCAN_THREADS];
+  __shared__ int part[32];
   extern __shared__ int hist[];  // [ngroups * (kcap + 1)]
   const int ngroups = (rows + group_rows - 1) / group_rows;
   const int nbins = ngroups * (kcap + 1);

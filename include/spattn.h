@@ -108,6 +108,11 @@ spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, c
 /* Routed attention (+ residual pseudo-keys) and the scatter
  * of the output, using the permuted copies and block means that the last
  * spattn_pool / spattn_route left in this workspace for the same inputs.
+ * Routing reuse across calls (SVOO and PARK reuse sparse masks across
+ * diffusion steps): after one spattn_route, a spattn_pool on new inputs
+ * followed by spattn_attend with NULL row_ptr/col_idx attends the new
+ * inputs with the kept lists of that earlier route (the residual uses the
+ * new inputs' means).
  *   row_ptr, col_idx  NULL to use the workspace CSR of the last route, or a
  *                     caller CSR in the layout above (device).  Block
  *                     indices outside [0, nb) are skipped and flagged

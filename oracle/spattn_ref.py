@@ -115,6 +115,19 @@ def block_softmax(s: np.ndarray) -> np.ndarray:
     return e / e.sum(axis=-1, keepdims=True)
 
 
+def pama_importance(q: np.ndarray, Kbar: np.ndarray, n: np.ndarray) -> np.ndarray:
+    """Block importance of one query block by per-query attention-mass
+    aggregation (PARK page 5.1, PAMA): every query token q keeps its own
+    softmax over the key blocks of the centroid logit q . Kbar_j / sqrt(d) +
+    ln n_j (the same block log-mass estimate as the proxy), and the block's
+    importance row is the mean of its tokens' rows (PARK page 3.2: the
+    average attention weight the block's queries give each key block).
+    q: [n_i, d] tokens of the query block; returns p_i [nb], summing to 1."""
+    d = q.shape[-1]
+    s = q @ Kbar.T / math.sqrt(d) + np.log(n.astype(np.float64))[None, :]
+    return block_softmax(s).mean(axis=0)
+
+
 def exact_block_logmass(q: np.ndarray, Kblock: np.ndarray) -> float:
     """ln sum_{k in block} exp(q . k / sqrt(d)): the quantity s_ij bounds."""
     z = Kblock @ q / math.sqrt(q.shape[-1])
@@ -241,7 +254,8 @@ def attention_flops(kept_rows, n: np.ndarray, residual: bool, d: int) -> tuple:
 
 def forward(Q, K, V, b: int, tau: float, kmin: int, kmax: int, residual: int,
             perm: Optional[np.ndarray] = None, rows: Optional[dict] = None,
-            kept_override: Optional[dict] = None, want_output: bool = True):
+            kept_override: Optional[dict] = None, want_output: bool = True,
+            routing: str = "centroid"):
     """The whole path for bf16 inputs Q, K, V ([B, H, N, d] uint16 bits).
 
     rows:          optional {(b, h): array of token indices in the ORIGINAL
@@ -249,6 +263,8 @@ def forward(Q, K, V, b: int, tau: float, kmin: int, kmax: int, residual: int,
     kept_override: optional {(b, h): list of kept sets} to run the attention
                    with externally supplied kept sets (routing is still
                    computed and returned).
+    routing:       "centroid" (p from the block-mean proxy) or "pama" (p from
+                   pama_importance of each query block's tokens).
     Returns a dict with Qbar/Kbar/Vbar (fp64 [B,H,nb,d]), route (per (b,h)
     route_rows results), and O: either [B,H,N,d] fp64 or {(b,h): [r, d]}.
     """
@@ -272,8 +288,14 @@ def forward(Q, K, V, b: int, tau: float, kmin: int, kmax: int, residual: int,
             Qbar[bi, hi] = block_means(q, b)
             Kbar[bi, hi] = block_means(k, b)
             Vbar[bi, hi] = block_means(v, b)
-            s = proxy_logits(Qbar[bi, hi], Kbar[bi, hi], n)
-            r = route_rows(block_softmax(s), tau, kmin, kmax)
+            if routing == "pama":
+                starts = np.concatenate([[0], np.cumsum(n)[:-1]])
+                p = np.stack([pama_importance(q[s0:s0 + nj], Kbar[bi, hi], n)
+                              for s0, nj in zip(starts, n)])
+            else:
+                p = block_softmax(proxy_logits(Qbar[bi, hi], Kbar[bi, hi], n))
+            r = route_rows(p, tau, kmin, kmax)
+            r["p"] = p
             routes[(bi, hi)] = r
             if not want_output:
                 continue

@@ -154,3 +154,46 @@ def test_tc_repeated_attend_is_bitwise_stable():
         plan.close()
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
     assert torch.equal(outs[0].view(torch.int16), outs[2].view(torch.int16))
+
+
+def test_tc_routing_reuse_across_calls():
+    """Route once on inputs A, then pool + attend inputs B: the output is the
+    oracle's attention of B over A's kept sets (B's own means feed the
+    residual).  With the Hilbert permutation, so the pooling's permuted
+    copies of B are what the attention reads."""
+    import torch
+    import block_sparse_attention_33_b200 as sp
+    from oracle import spattn_ref as R
+    from tests.harness import csr_to_kept, from_dev, to_dev
+    w = get_config("medium", H=2, tau=0.8)
+    wb = w.with_(seed=w.seed + 77)
+    QA, KA, VA = make_qkv(w)
+    QB, KB, VB = make_qkv(wb)
+    perm = sp.spattn_hilbert_perm(*w.grid)
+    plan = sp.Plan(w.B, w.H, w.N, w.d, w.b, w.tau, w.kmin, w.kmax, w.residual, perm)
+    try:
+        rows = w.B * w.H * plan.nb
+        rp = torch.zeros(rows + 1, dtype=torch.int32, device="cuda")
+        ci = torch.zeros(max(plan.col_capacity, 1), dtype=torch.int32, device="cuda")
+        qa, ka, va = to_dev(QA), to_dev(KA), to_dev(VA)
+        plan.route(qa, ka, va, rp, ci)
+        qb, kb, vb = to_dev(QB), to_dev(KB), to_dev(VB)
+        o = torch.zeros_like(qb)
+        plan.pool(qb, kb, vb)
+        plan.attend(qb, kb, vb, o)
+        assert plan.check() == 0
+        O = from_dev(o)
+        kept_a = csr_to_kept(rp.cpu().numpy(), ci.cpu().numpy(), w.B, w.H, plan.nb)
+    finally:
+        plan.close()
+    pick = {(0, h): perm[np.arange(0, w.N, 53)] for h in range(w.H)}
+    ref = R.forward(QB, KB, VB, w.b, w.tau, w.kmin, w.kmax, w.residual, perm=perm, rows=pick,
+                    kept_override=kept_a)
+    got = np.concatenate([O[0, h, pick[(0, h)]] for h in range(w.H)])
+    want = np.concatenate([ref["O"][(0, h)] for h in range(w.H)])
+    max_abs, rel = compare_outputs(got, want)
+    assert max_abs < MAX_ABS and rel < REL_L2, (max_abs, rel)
+    # and it differs from B's own routing's result somewhere (A's sets are not B's)
+    own = R.forward(QB, KB, VB, w.b, w.tau, w.kmin, w.kmax, w.residual, perm=perm, rows=pick)
+    assert any(not np.array_equal(np.sort(a), np.sort(b))
+               for key in own["route"] for a, b in zip(own["route"][key]["kept"], kept_a[key]))

@@ -385,3 +385,79 @@ def test_hilbert_perm_on_stress_grid_is_a_bijection_with_local_blocks():
     # consecutive tokens in Hilbert order are near each other on the grid
     jumps = np.abs(np.diff(t)) + np.abs(np.diff(h)) + np.abs(np.diff(ww))
     assert np.median(jumps) == 1
+
+
+# --------------------------------------------------- PAMA block importance --
+# PARK page 5.1: each query keeps its own softmax over key blocks; the block's
+# importance is the mean of its queries' rows.
+
+def test_pama_hand_computed_two_tokens():
+    """d = 4 (sqrt(d) = 2), equal block sizes.  Token 1 has centroid logits
+    (ln 3, 0) -> (3/4, 1/4); token 2 has logits (0, 0) -> (1/2, 1/2); PAMA is
+    the mean (5/8, 3/8).  The block-mean query instead gives logits
+    (ln 3 / 2, 0) -> (sqrt 3, 1) / (sqrt 3 + 1), which differs."""
+    l3 = math.log(3.0)
+    q = np.array([[2 * l3, 0, 0, 0], [0, 0, 0, 0]], dtype=np.float64)
+    Kbar = np.array([[1, 0, 0, 0], [0, 0, 0, 0]], dtype=np.float64)
+    n = np.array([128, 128])
+    p = R.pama_importance(q, Kbar, n)
+    assert np.allclose(p, [5 / 8, 3 / 8], atol=1e-15)
+    pc = R.block_softmax(R.proxy_logits(q.mean(axis=0, keepdims=True), Kbar, n))[0]
+    s3 = math.sqrt(3.0)
+    assert np.allclose(pc, [s3 / (s3 + 1), 1 / (s3 + 1)], atol=1e-15)
+    assert abs(p[0] - pc[0]) > 5e-3
+
+
+def test_pama_block_size_term():
+    """Zero centroids: every token's row is n_j / sum n, so a partial block of
+    64 against a full one of 128 gets 1/3 (the ln n_j term)."""
+    q = np.random.default_rng(0).standard_normal((5, 8))
+    p = R.pama_importance(q, np.zeros((2, 8)), np.array([128, 64]))
+    assert np.allclose(p, [2 / 3, 1 / 3], atol=1e-15)
+
+
+def test_pama_equals_centroid_proxy_for_constant_query_blocks():
+    """When every token of the query block is the same vector, averaging the
+    per-token softmax rows changes nothing: PAMA equals the block-mean proxy
+    softmax."""
+    rng = np.random.default_rng(3)
+    nb, d = 7, 16
+    Kbar = rng.standard_normal((nb, d)) * 2
+    n = np.array([16] * (nb - 1) + [5])
+    q = np.repeat(rng.standard_normal((1, d)) * 3, 16, axis=0)
+    p = R.pama_importance(q, Kbar, n)
+    pc = R.block_softmax(R.proxy_logits(q[:1], Kbar, n))[0]
+    assert np.allclose(p, pc, rtol=0, atol=1e-14)
+
+
+def test_pama_rows_are_distributions_and_match_torch():
+    """Rows are probability vectors; the per-token softmax and the mean agree
+    with torch's fp64 softmax and mean on random data."""
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((33, 16)) * 4
+    Kbar = rng.standard_normal((9, 16))
+    n = np.array([64] * 8 + [17])
+    p = R.pama_importance(q, Kbar, n)
+    assert abs(p.sum() - 1) < 1e-14 and np.all(p >= 0)
+    s = torch.from_numpy(q) @ torch.from_numpy(Kbar).T / 4.0 + torch.log(torch.from_numpy(n).double())
+    want = torch.softmax(s, dim=-1).mean(dim=0).numpy()
+    assert np.allclose(p, want, atol=1e-15)
+
+
+def test_forward_pama_routes_from_token_rows():
+    """forward(routing='pama') feeds route_rows the PAMA rows of each query
+    block (checked against a direct evaluation), and at tau = 1 the output is
+    the same dense attention as with the centroid routing."""
+    w = get_config("tiny", H=1)
+    Q, K, V = make_qkv(w)
+    ref = R.forward(Q, K, V, w.b, w.tau, w.kmin, w.kmax, w.residual, routing="pama",
+                    want_output=False)
+    q = R.decode_bf16(Q[0, 0])
+    n = R.block_sizes(w.N, w.b)
+    Kbar = ref["Kbar"][0, 0]
+    for i in (0, 5, w.nb - 1):
+        p = R.pama_importance(q[i * w.b:i * w.b + n[i]], Kbar, n)
+        assert np.allclose(ref["route"][(0, 0)]["p"][i], p, atol=1e-15)
+    a = R.forward(Q, K, V, w.b, 1.0, 1, w.nb, 1, routing="pama")["O"]
+    c = R.forward(Q, K, V, w.b, 1.0, 1, w.nb, 1)["O"]
+    assert np.allclose(a, c, atol=1e-12)
