@@ -76,6 +76,9 @@ def parse_args(argv=None):
                     choices=["tiny", "medium", "wan", "hunyuan", "stress"])
     ap.add_argument("--tau", type=float, default=None)
     ap.add_argument("--residual", type=int, default=None)
+    ap.add_argument("--routing", choices=["centroid", "pama"], default="centroid",
+                    help="block-importance estimate: block-mean centroids, or per-query "
+                         "attention-mass aggregation (PAMA)")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the number of heads (smaller profiling captures)")
     ap.add_argument("--no-dense", action="store_true", help="skip the tau = 1 comparison run")
@@ -327,7 +330,9 @@ def run_ours(args):
 
     q, k, v = dev_bf16(Qh), dev_bf16(Kh), dev_bf16(Vh)
     o = torch.empty_like(q)
-    plan = sp.Plan(B, H, N, d, w.b, w.tau, w.kmin, w.kmax, w.residual, perm, device=dev)
+    routing = sp.ROUTING_PAMA if args.routing == "pama" else sp.ROUTING_CENTROID
+    plan = sp.Plan(B, H, N, d, w.b, w.tau, w.kmin, w.kmax, w.residual, perm, device=dev,
+                   routing=routing)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -403,7 +408,8 @@ def run_ours(args):
     pool_ms = float(np.mean([x[0] for x in tp]))
     # routing (proxy logits, softmax, selection, order): the proxy GEMM's FLOPs
     # on fp32 FMA lanes; its time is the step's route chain minus the pooling
-    route_flops = 2.0 * B * H * plan.nb * plan.nb * d
+    route_flops = (4.0 * B * H * N * plan.nb * d if args.routing == "pama"     # two passes over every token
+                   else 2.0 * B * H * plan.nb * plan.nb * d)
     fp32_peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
     tok_bytes = B * H * N * d * 2
     pool_bytes = 3 * tok_bytes + B * H * plan.nb * d * (3 * 4 + 2 * 2)
@@ -451,7 +457,8 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": config_of(w, "flushed (256 MiB write between timed steps)"),
+            "config": dict(config_of(w, "flushed (256 MiB write between timed steps)"),
+                           routing=args.routing),
             "dense_equiv_tflops": dense_flops * world / (step_ms * 1e-3) / 1e12,
             "attn_tflops": attn_tflops,
             "pct_of_bf16_peak": 100.0 * attn_tflops / bf16_peak,

@@ -20,7 +20,9 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA",
                 5: "TIMEOUT", 6: "DEVICE"}
 
-EXPORTS = ("spattn_plan", "spattn_plan_destroy", "spattn_plan_info", "spattn_pool",
+ROUTING_CENTROID, ROUTING_PAMA = 0, 1
+
+EXPORTS = ("spattn_plan", "spattn_plan_ex", "spattn_plan_destroy", "spattn_plan_info", "spattn_pool",
            "spattn_route", "spattn_attend", "spattn_forward", "spattn_means", "spattn_check",
            "spattn_hilbert_perm", "spattn_route_static", "spattn_last_error")
 
@@ -47,6 +49,7 @@ def lib():
                              ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_size_t))
     sig = {
         "spattn_plan": [ctypes.POINTER(P), I, I, I, I, I, F, I, I, I, P, SZP],
+        "spattn_plan_ex": [ctypes.POINTER(P), I, I, I, I, I, F, I, I, I, P, I, SZP],
         "spattn_plan_destroy": [P],
         "spattn_plan_info": [P, ctypes.POINTER(I), ctypes.POINTER(ctypes.c_int64)],
         "spattn_pool": [P, P, P, P, P, P],
@@ -100,6 +103,11 @@ def spattn_last_error() -> str:
 
 def spattn_plan(B, H, N, d, b, tau, kmin, kmax, residual, perm=None):
     """Create a plan; returns (handle, workspace_bytes).  perm: host int32 array or None."""
+    return spattn_plan_ex(B, H, N, d, b, tau, kmin, kmax, residual, perm, ROUTING_CENTROID)
+
+
+def spattn_plan_ex(B, H, N, d, b, tau, kmin, kmax, residual, perm=None, routing=ROUTING_CENTROID):
+    """spattn_plan with a routing estimate (ROUTING_CENTROID or ROUTING_PAMA)."""
     import numpy as np
     h = ctypes.c_void_p()
     ws = ctypes.c_size_t()
@@ -107,8 +115,8 @@ def spattn_plan(B, H, N, d, b, tau, kmin, kmax, residual, perm=None):
     if perm is not None:
         perm = np.ascontiguousarray(perm, dtype=np.int32)
         pp = perm.ctypes.data
-    _check(lib().spattn_plan(ctypes.byref(h), B, H, N, d, b, float(tau), kmin, kmax, residual,
-                             pp, ctypes.byref(ws)))
+    _check(lib().spattn_plan_ex(ctypes.byref(h), B, H, N, d, b, float(tau), kmin, kmax, residual,
+                                pp, int(routing), ctypes.byref(ws)))
     return h.value, ws.value
 
 
@@ -172,10 +180,12 @@ def spattn_route_static(B, H, N, d, b, tau, kmin, kmax, Q, K, row_ptr, col_idx, 
 class Plan:
     """Owning wrapper: a plan plus its device workspace (torch allocation)."""
 
-    def __init__(self, B, H, N, d, b, tau, kmin, kmax, residual, perm=None, device="cuda"):
+    def __init__(self, B, H, N, d, b, tau, kmin, kmax, residual, perm=None, device="cuda",
+                 routing=ROUTING_CENTROID):
         import torch
         self.shape = (B, H, N, d)
-        self.handle, self.ws_bytes = spattn_plan(B, H, N, d, b, tau, kmin, kmax, residual, perm)
+        self.handle, self.ws_bytes = spattn_plan_ex(B, H, N, d, b, tau, kmin, kmax, residual, perm,
+                                                    routing)
         self.nb, self.col_capacity = spattn_plan_info(self.handle)
         self.workspace = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=device)
 

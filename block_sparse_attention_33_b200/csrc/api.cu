@@ -158,8 +158,17 @@ const char* spattn_last_error(void) { return g_err; }
 spattn_status_t spattn_plan(spattn_plan_t* out, int B, int H, int N, int d, int b, float tau,
                             int kmin, int kmax, int residual, const int32_t* perm_host,
                             size_t* workspace_bytes) {
+  return spattn_plan_ex(out, B, H, N, d, b, tau, kmin, kmax, residual, perm_host,
+                        SPATTN_ROUTING_CENTROID, workspace_bytes);
+}
+
+spattn_status_t spattn_plan_ex(spattn_plan_t* out, int B, int H, int N, int d, int b, float tau,
+                               int kmin, int kmax, int residual, const int32_t* perm_host,
+                               int routing, size_t* workspace_bytes) {
   g_err[0] = 0;
   if (!out) return fail(SPATTN_ERR_INVALID_ARG, "out is NULL");
+  if (routing != SPATTN_ROUTING_CENTROID && routing != SPATTN_ROUTING_PAMA)
+    return fail(SPATTN_ERR_INVALID_ARG, "routing must be SPATTN_ROUTING_CENTROID or SPATTN_ROUTING_PAMA (got %d)", routing);
   *out = nullptr;
   if (B < 1 || H < 1 || N < 1) return fail(SPATTN_ERR_INVALID_ARG, "need B, H, N >= 1 (got %d, %d, %d)", B, H, N);
   if (d != 64 && d != 128) return fail(SPATTN_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
@@ -189,6 +198,7 @@ spattn_status_t spattn_plan(spattn_plan_t* out, int B, int H, int N, int d, int 
   p.BH = B * H;
   p.tau = tau; p.kmin = kmin; p.kmax = kmax; p.residual = residual;
   p.perm = nullptr;
+  p.routing = routing == SPATTN_ROUTING_PAMA ? spattn::ROUTING_PAMA : spattn::ROUTING_CENTROID;
   {
     // tcgen05/TMEM kernel for 128-token blocks; the warp-MMA kernel serves
     // b = 64 and, with SPATTN_ATTN=mma in the environment when the plan is
@@ -245,7 +255,7 @@ spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, c
   cudaError_t e = spattn::launch_pool(plan->p, Q, K, V, w, s);
   if (e != cudaSuccess) return cuda_fail(e, "pool kernel");
   // the warp-MMA attention reads the compact CSR of the workspace
-  e = spattn::launch_route(plan->p, w, row_ptr, col_idx, !plan->p.use_tc, s);
+  e = spattn::launch_route(plan->p, w, Q, row_ptr, col_idx, !plan->p.use_tc, s);
   if (e != cudaSuccess) return cuda_fail(e, "route kernels");
   return SPATTN_OK;
 }

@@ -8,6 +8,8 @@
 
 namespace spattn {
 
+enum { ROUTING_CENTROID = 0, ROUTING_PAMA = 1 };
+
 // Problem description derived from a plan (all sizes in elements).
 struct Problem {
   int B, H, N, d, b, nb, n_last, kcap;
@@ -16,6 +18,7 @@ struct Problem {
   int kmin, kmax;
   int residual;
   int use_tc;           // attention on the tcgen05 kernel (else warp MMA)
+  int routing;          // ROUTING_CENTROID or ROUTING_PAMA
   const int32_t* perm;  // device, NULL if none
 };
 
@@ -37,7 +40,8 @@ cudaError_t launch_pool(const Problem& p, const void* Q, const void* K, const vo
 // need_csr: also build the compact CSR in w.row_ptr / w.col_idx (the
 // tcgen05 attention reads the padded per-row lists directly, so the compact
 // copy is made only for callers and paths that need it).
-cudaError_t launch_route(const Problem& p, const Work& w, int32_t* row_ptr_out,
+// Q: the original queries (PAMA reads tokens through p.perm).
+cudaError_t launch_route(const Problem& p, const Work& w, const void* Q, int32_t* row_ptr_out,
                          int32_t* col_idx_out, bool need_csr, cudaStream_t s);
 cudaError_t launch_attend(const Problem& p, const void* Q, const void* K, const void* V,
                           const int32_t* row_ptr, const int32_t* col_idx, void* O,

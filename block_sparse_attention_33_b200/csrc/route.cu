@@ -126,6 +126,75 @@ __device__ __forceinline__ int count_above_1(const float* p, int nb, uint32_t u)
 // rows with at most this many blocks use the 32-way search
 constexpr int SEARCH32_MAX_NB = 128;
 
+// One warp: the Top-p selection and clamp on a probability row p[0..nb) in
+// shared memory, then the kept blocks of query row `row` emitted in
+// ascending j into the padded lists, and their count.
+__device__ void select_emit(const float* p, const RouteArgs& a, int row) {
+  const int lane = threadIdx.x & 31;
+  // kept set = {bits(p) > thr} + first `ties` blocks with bits(p) == thr
+  uint32_t thr = 0;
+  int ties = 0, kstar = 0;
+  bool by_mass = false;
+  if (a.tau >= 1.0f) {
+    kstar = a.nb;               // tau >= 1 keeps every block
+  } else if (a.tau > 0.0f) {
+    if (a.nb <= SEARCH32_MAX_NB) {
+      thr = search32(0u, 0x3F800000u, [&](uint32_t u) { return mass_above_1(p, a.nb, u) < a.tau; });
+    } else {
+      uint32_t lo = 0, hi = 0x3F800000u;  // p <= 1, so nothing is above hi
+      while (lo < hi) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (mass_above(p, a.nb, mid) < a.tau) hi = mid; else lo = mid + 1;
+      }
+      thr = lo;
+    }
+    // the same summation as the search's predicate
+    const float g = a.nb <= SEARCH32_MAX_NB ? mass_above_1(p, a.nb, thr) : mass_above(p, a.nb, thr);
+    const int gt = count_above(p, a.nb, thr);
+    const int eq = count_equal(p, a.nb, thr);
+    const float v = __uint_as_float(thr);
+    float e = g;
+    int keep = 0;
+    while (keep < eq && e < a.tau) { e += v; ++keep; }
+    ties = keep;
+    kstar = gt + keep;
+    by_mass = true;
+  }
+  const int k = min(max(kstar, a.kmin), a.kcap);
+  const bool all = (k >= a.nb);
+  if (!all && !(by_mass && k == kstar)) {
+    // the clamp binds (or tau <= 0): top-k in (p desc, j asc) order
+    if (a.nb <= SEARCH32_MAX_NB) {
+      thr = search32(0u, 0x3F800000u, [&](uint32_t u) { return count_above_1(p, a.nb, u) < k; });
+    } else {
+      uint32_t lo = 0, hi = 0x3F800000u;
+      while (lo < hi) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (count_above(p, a.nb, mid) < k) hi = mid; else lo = mid + 1;
+      }
+      thr = lo;
+    }
+    ties = k - count_above(p, a.nb, thr);
+  }
+  int32_t* out = a.lists + (size_t)row * a.kcap;
+  int base = 0, seen_eq = 0;
+  for (int j0 = 0; j0 < a.nb; j0 += 32) {
+    const int j = j0 + lane;
+    const bool valid = j < a.nb;
+    const uint32_t u = valid ? __float_as_uint(p[j]) : 0u;
+    const bool eq = valid && !all && u == thr;
+    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+    const int eq_rank = seen_eq + __popc(eqm & ((1u << lane) - 1u));
+    seen_eq += __popc(eqm);
+    const bool keep = valid && (all || u > thr || (eq && eq_rank < ties));
+    const unsigned km = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[base + __popc(km & ((1u << lane) - 1u))] = j;
+    base += __popc(km);
+  }
+  if (lane == 0) a.counts[row] = k;
+}
+
+
 template <int D, int RT_ROWS>
 __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
   extern __shared__ __align__(16) float sm[];
@@ -197,70 +266,170 @@ __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
     sum = warp_sum(sum);
     for (int j = lane; j < a.nb; j += 32) p[j] = p[j] / sum;
     __syncwarp();
-
-    // kept set = {bits(p) > thr} + first `ties` blocks with bits(p) == thr
-    uint32_t thr = 0;
-    int ties = 0, kstar = 0;
-    bool by_mass = false;
-    if (a.tau >= 1.0f) {
-      kstar = a.nb;               // tau >= 1 keeps every block
-    } else if (a.tau > 0.0f) {
-      if (a.nb <= SEARCH32_MAX_NB) {
-        thr = search32(0u, 0x3F800000u, [&](uint32_t u) { return mass_above_1(p, a.nb, u) < a.tau; });
-      } else {
-        uint32_t lo = 0, hi = 0x3F800000u;  // p <= 1, so nothing is above hi
-        while (lo < hi) {
-          const uint32_t mid = lo + ((hi - lo) >> 1);
-          if (mass_above(p, a.nb, mid) < a.tau) hi = mid; else lo = mid + 1;
-        }
-        thr = lo;
-      }
-      // the same summation as the search's predicate
-      const float g = a.nb <= SEARCH32_MAX_NB ? mass_above_1(p, a.nb, thr) : mass_above(p, a.nb, thr);
-      const int gt = count_above(p, a.nb, thr);
-      const int eq = count_equal(p, a.nb, thr);
-      const float v = __uint_as_float(thr);
-      float e = g;
-      int keep = 0;
-      while (keep < eq && e < a.tau) { e += v; ++keep; }
-      ties = keep;
-      kstar = gt + keep;
-      by_mass = true;
-    }
-    const int k = min(max(kstar, a.kmin), a.kcap);
-    const bool all = (k >= a.nb);
-    if (!all && !(by_mass && k == kstar)) {
-      // the clamp binds (or tau <= 0): top-k in (p desc, j asc) order
-      if (a.nb <= SEARCH32_MAX_NB) {
-        thr = search32(0u, 0x3F800000u, [&](uint32_t u) { return count_above_1(p, a.nb, u) < k; });
-      } else {
-        uint32_t lo = 0, hi = 0x3F800000u;
-        while (lo < hi) {
-          const uint32_t mid = lo + ((hi - lo) >> 1);
-          if (count_above(p, a.nb, mid) < k) hi = mid; else lo = mid + 1;
-        }
-        thr = lo;
-      }
-      ties = k - count_above(p, a.nb, thr);
-    }
-    const int row = bh * a.nb + i0 + r;
-    int32_t* out = a.lists + (size_t)row * a.kcap;
-    int base = 0, seen_eq = 0;
-    for (int j0 = 0; j0 < a.nb; j0 += 32) {
-      const int j = j0 + lane;
-      const bool valid = j < a.nb;
-      const uint32_t u = valid ? __float_as_uint(p[j]) : 0u;
-      const bool eq = valid && !all && u == thr;
-      const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-      const int eq_rank = seen_eq + __popc(eqm & ((1u << lane) - 1u));
-      seen_eq += __popc(eqm);
-      const bool keep = valid && (all || u > thr || (eq && eq_rank < ties));
-      const unsigned km = __ballot_sync(0xffffffffu, keep);
-      if (keep) out[base + __popc(km & ((1u << lane) - 1u))] = j;
-      base += __popc(km);
-    }
-    if (lane == 0) a.counts[row] = k;
+    select_emit(p, a, bh * a.nb + i0 + r);
   }
+}
+
+// PAMA block importance (PARK page 5.1): every query token of block i keeps
+// its own softmax over the key blocks of the centroid logit
+// q . Kbar_j / sqrt(d) + ln n_j, and p_i is the mean of the n_i tokens'
+// rows; then the same Top-p selection.  One CTA per (query block, head),
+// 256 threads: thread t owns token t % 128 and half t / 128 of each chunk of
+// 32 key blocks (16 dot products, fp32 FMAs over the channels).  Pass 1 runs
+// an online (max, sum) per token over all chunks; pass 2 recomputes the
+// logits, forms each token's probabilities and sums them over the tokens
+// (shuffle tree inside a warp, then the four warps of a half in a fixed
+// order).  Tokens are read through the permutation when there is one.
+constexpr int PAMA_THREADS = 256;
+constexpr int PAMA_CHUNK = 32;
+
+template <int D>
+size_t pama_smem_bytes(int nb) {
+  const int nbp = (nb + 31) & ~31;
+  return ((size_t)(128 + PAMA_CHUNK) * (D + 4) + nbp + 2 * 2 * 128 + 8 * 16) * sizeof(float);
+}
+
+template <int D>
+__global__ void __launch_bounds__(PAMA_THREADS, 2) pama_kernel(RouteArgs a,
+                                                              const __nv_bfloat16* qtok,
+                                                              const int32_t* perm, int N) {
+  constexpr int QS = D + 4;   // padded fp32 row stride (float4-aligned)
+  extern __shared__ __align__(16) float sm[];
+  const int nbp = (a.nb + 31) & ~31;
+  float* Qs = sm;                          // [128][QS]
+  float* Ks = Qs + 128 * QS;               // [PAMA_CHUNK][QS]
+  float* p = Ks + PAMA_CHUNK * QS;         // [nbp]
+  float* ml = p + nbp;                     // [2 halves][128 tokens][m, l]
+  float* part = ml + 2 * 2 * 128;          // [8 warps][16]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int i = blockIdx.x, bh = blockIdx.y;
+  const int ni = (i == a.nb - 1) ? a.n_last : a.b;
+
+  // tokens of query block i, fp32; rows past n_i are zero (masked below)
+  const __nv_bfloat16* qh = qtok + (size_t)bh * N * D;
+  for (int e = tid; e < 128 * (D / 8); e += PAMA_THREADS) {
+    const int r = e / (D / 8), c8 = e % (D / 8);
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = 0.f;
+    if (r < ni) {
+      const int tok = i * a.b + r;
+      const int src = perm ? __ldg(perm + tok) : tok;
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qh + (size_t)src * D) + c8);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(h[k]);
+        v[2 * k] = f.x;
+        v[2 * k + 1] = f.y;
+      }
+    }
+    float4* dst = reinterpret_cast<float4*>(Qs + r * QS + c8 * 8);
+    dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+    dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+
+  const float* kbar = a.kbar + (size_t)bh * a.nb * D;
+  const float inv_sqrt_d = 1.0f / sqrtf((float)D);
+  const float lg_b = logf((float)a.b), lg_last = logf((float)a.n_last);
+  const int r = tid & 127, jh = tid >> 7;
+  const int nch = (a.nb + PAMA_CHUNK - 1) / PAMA_CHUNK;
+
+  auto load_chunk = [&](int c) {
+    __syncthreads();   // the previous chunk's readers are done
+    for (int e = tid; e < PAMA_CHUNK * (D / 4); e += PAMA_THREADS) {
+      const int jj = e / (D / 4), k4 = e % (D / 4);
+      const int j = c * PAMA_CHUNK + jj;
+      const float4 v = j < a.nb ? __ldg(reinterpret_cast<const float4*>(kbar + (size_t)j * D) + k4)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+      reinterpret_cast<float4*>(Ks + jj * QS)[k4] = v;
+    }
+    __syncthreads();
+  };
+  auto logits = [&](int c, float (&sv)[16]) {
+    float acc[16];
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) acc[jj] = 0.f;
+    const float4* q4 = reinterpret_cast<const float4*>(Qs + r * QS);
+#pragma unroll 2
+    for (int k4 = 0; k4 < D / 4; ++k4) {
+      const float4 q = q4[k4];
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const float4 kv = reinterpret_cast<const float4*>(Ks + (jh * 16 + jj) * QS)[k4];
+        acc[jj] = fmaf(q.x, kv.x, acc[jj]);
+        acc[jj] = fmaf(q.y, kv.y, acc[jj]);
+        acc[jj] = fmaf(q.z, kv.z, acc[jj]);
+        acc[jj] = fmaf(q.w, kv.w, acc[jj]);
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+      const int j = c * PAMA_CHUNK + jh * 16 + jj;
+      sv[jj] = j < a.nb ? fmaf(acc[jj], inv_sqrt_d, j == a.nb - 1 ? lg_last : lg_b) : -INFINITY;
+    }
+  };
+
+  // pass 1: per token, running max and sum over this thread's half of every chunk
+  float m = -INFINITY, l = 0.f;
+  for (int c = 0; c < nch; ++c) {
+    load_chunk(c);
+    float sv[16];
+    logits(c, sv);
+    float cm = sv[0];
+#pragma unroll
+    for (int jj = 1; jj < 16; ++jj) cm = fmaxf(cm, sv[jj]);
+    const float mn = fmaxf(m, cm);
+    if (mn > -INFINITY) {
+      float add = 0.f;
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) add += expf(sv[jj] - mn);
+      l = l * expf(m - mn) + add;
+      m = mn;
+    }
+  }
+  ml[(jh * 128 + r) * 2] = m;
+  ml[(jh * 128 + r) * 2 + 1] = l;
+  __syncthreads();
+  const float m0 = ml[r * 2], l0 = ml[r * 2 + 1], m1 = ml[(128 + r) * 2], l1 = ml[(128 + r) * 2 + 1];
+  const float M = fmaxf(m0, m1);
+  const float L = (m0 > -INFINITY ? l0 * expf(m0 - M) : 0.f) + (m1 > -INFINITY ? l1 * expf(m1 - M) : 0.f);
+  const float invL = (r < ni && L > 0.f) ? 1.f / L : 0.f;   // padding rows contribute nothing
+
+  // pass 2: probabilities, summed over the block's tokens
+  for (int c = 0; c < nch; ++c) {
+    load_chunk(c);
+    float sv[16];
+    logits(c, sv);
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+      float w = sv[jj] > -INFINITY ? expf(sv[jj] - M) * invL : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) w += __shfl_xor_sync(0xffffffffu, w, o);
+      if (lane == 0) part[warp * 16 + jj] = w;
+    }
+    __syncthreads();
+    if (tid < PAMA_CHUNK) {
+      const int h = tid >> 4, jj = tid & 15;
+      const float t = ((part[(4 * h + 0) * 16 + jj] + part[(4 * h + 1) * 16 + jj]) +
+                       part[(4 * h + 2) * 16 + jj]) + part[(4 * h + 3) * 16 + jj];
+      const int j = c * PAMA_CHUNK + tid;
+      if (j < a.nb) p[j] = t / (float)ni;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) select_emit(p, a, bh * a.nb + i);
+}
+
+template <int D>
+cudaError_t launch_pama_d(const RouteArgs& a, const void* Q, const int32_t* perm, int N, int BH,
+                          cudaStream_t s) {
+  const size_t smem = pama_smem_bytes<D>(a.nb);
+  cudaError_t e = ensure_dyn_smem((const void*)pama_kernel<D>, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.nb, BH);
+  pama_kernel<D><<<grid, PAMA_THREADS, smem, s>>>(a, static_cast<const __nv_bfloat16*>(Q), perm, N);
+  return cudaGetLastError();
 }
 
 // Exclusive scan of the per-row counts into row_ptr (single CTA), total in
@@ -415,14 +584,23 @@ static int scan_group_rows(const Problem& p) {
   return heads * p.nb;
 }
 
-cudaError_t launch_route(const Problem& p, const Work& w, int32_t* row_ptr_out,
+cudaError_t launch_route(const Problem& p, const Work& w, const void* Q, int32_t* row_ptr_out,
                          int32_t* col_idx_out, bool need_csr, cudaStream_t s) {
   RouteArgs a;
   a.qbar = w.qbar; a.kbar = w.kbar; a.counts = w.counts; a.lists = w.lists;
   a.nb = p.nb; a.b = p.b; a.n_last = p.n_last; a.kcap = p.kcap; a.kmin = p.kmin;
   a.tau = p.tau;
-  cudaError_t e = p.d == 128 ? launch_route_d<128>(a, p.nb, p.BH, s)
-                             : launch_route_d<64>(a, p.nb, p.BH, s);
+  cudaError_t e;
+  if (p.routing == ROUTING_PAMA) {
+    // tokens in blocked order: the pooling's permuted copy when there is
+    // one, else the queries read through the permutation
+    const void* q = w.qp ? (const void*)w.qp : Q;
+    const int32_t* perm = w.qp ? nullptr : p.perm;
+    e = p.d == 128 ? launch_pama_d<128>(a, q, perm, p.N, p.BH, s)
+                   : launch_pama_d<64>(a, q, perm, p.N, p.BH, s);
+  } else {
+    e = p.d == 128 ? launch_route_d<128>(a, p.nb, p.BH, s) : launch_route_d<64>(a, p.nb, p.BH, s);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int rows = p.BH * p.nb;
   const int group_rows = scan_group_rows(p);

@@ -97,6 +97,7 @@ extern "C" spattn_status_t spattn_route_static(int B, int H, int N, int d, int b
   p.tau = tau; p.kmin = kmin; p.kmax = kmax;
   p.residual = 0;
   p.use_tc = 0;
+  p.routing = spattn::ROUTING_CENTROID;
   p.perm = perm;
 
   // scratch layout: Qbar, Kbar (fp32), counts, padded lists, order, control
@@ -129,7 +130,7 @@ extern "C" spattn_status_t spattn_route_static(int B, int H, int N, int d, int b
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the pooling kernel also clears the control block
   cudaError_t e = spattn::launch_pool_qk(p, Q, K, w.qbar, w.kbar, w.ctrl, s);
-  if (e == cudaSuccess) e = spattn::launch_route(p, w, nullptr, nullptr, true, s);
+  if (e == cudaSuccess) e = spattn::launch_route(p, w, Q, nullptr, nullptr, true, s);
   if (e != cudaSuccess) return fail(SPATTN_ERR_CUDA, "routing kernels: %s", cudaGetErrorString(e));
   return SPATTN_OK;
 }

@@ -80,6 +80,27 @@ spattn_status_t spattn_plan(spattn_plan_t* out, int B, int H, int N, int d, int 
                             float tau, int kmin, int kmax, int residual,
                             const int32_t* perm_host, size_t* workspace_bytes);
 
+/* Block-importance estimate that drives the Top-p selection. */
+enum {
+  SPATTN_ROUTING_CENTROID = 0, /* p_i = softmax_j(Qbar_i . Kbar_j / sqrt(d) + ln n_j):
+                                  block-mean query and key centroids (PARK page
+                                  3.2 block importance from centroids)           */
+  SPATTN_ROUTING_PAMA = 1      /* p_i = mean over the tokens q of block i of
+                                  softmax_j(q . Kbar_j / sqrt(d) + ln n_j): each
+                                  query keeps its own normalisation (PARK page
+                                  5.1, per-query attention-mass aggregation);
+                                  costs 2 * n_i * nb * d FMAs per query block
+                                  (two passes), on fp32 lanes                   */
+};
+
+/* spattn_plan with a choice of routing estimate (one of the values above;
+ * anything else is SPATTN_ERR_INVALID_ARG).  spattn_plan is
+ * spattn_plan_ex(..., SPATTN_ROUTING_CENTROID, ...).  spattn_route_static
+ * always uses the centroid estimate. */
+spattn_status_t spattn_plan_ex(spattn_plan_t* out, int B, int H, int N, int d, int b,
+                               float tau, int kmin, int kmax, int residual,
+                               const int32_t* perm_host, int routing, size_t* workspace_bytes);
+
 /* Release a plan (and its device copy of the permutation). NULL is a no-op. */
 spattn_status_t spattn_plan_destroy(spattn_plan_t plan);
 

@@ -111,3 +111,20 @@ def test_hilbert_rejects_bad_grid(L):
     buf = np.empty(4, np.int32)
     assert L.spattn_hilbert_perm(0, 2, 2, buf.ctypes.data) == sp.ERR_INVALID_ARG
     assert L.spattn_hilbert_perm(2, 2, 1, None) == sp.ERR_INVALID_ARG
+
+
+def test_plan_ex_routing_argument(L):
+    """spattn_plan_ex accepts the two routing estimates (no CUDA needed
+    without a permutation) and rejects anything else before any CUDA call."""
+    for routing, code in ((sp.ROUTING_CENTROID, sp.OK), (sp.ROUTING_PAMA, sp.OK),
+                          (2, sp.ERR_INVALID_ARG), (-1, sp.ERR_INVALID_ARG)):
+        h = ctypes.c_void_p()
+        ws = ctypes.c_size_t()
+        st = L.spattn_plan_ex(ctypes.byref(h), 1, 2, 1000, 64, 64, 0.9, 1, 8, 1, None, routing,
+                              ctypes.byref(ws))
+        assert st == code, (routing, st, L.spattn_last_error())
+        if st == sp.OK:
+            assert h.value and ws.value > 0
+            assert L.spattn_plan_destroy(h) == sp.OK
+        else:
+            assert not h.value and b"routing" in L.spattn_last_error()
