@@ -274,19 +274,20 @@ __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
 // its own softmax over the key blocks of the centroid logit
 // q . Kbar_j / sqrt(d) + ln n_j, and p_i is the mean of the n_i tokens'
 // rows; then the same Top-p selection.  One CTA per (query block, head),
-// 256 threads: thread t owns token t % 128 and half t / 128 of each chunk of
-// 32 key blocks (16 dot products, fp32 FMAs over the channels).  Pass 1 runs
-// an online (max, sum) per token over all chunks; pass 2 recomputes the
-// logits, forms each token's probabilities and sums them over the tokens
-// (shuffle tree inside a warp, then the four warps of a half in a fixed
-// order).  Tokens are read through the permutation when there is one.
+// 256 threads: thread t owns tokens t % 64 and t % 64 + 64 and quarter
+// t / 64 of each chunk of 32 key blocks (2 x 8 dot products, fp32 FMAs over
+// the channels, each centroid value read from shared memory feeding two
+// tokens).  Pass 1 runs an online (max, sum) per token over all chunks;
+// pass 2 recomputes the logits, forms each token's probabilities and sums
+// them over the tokens (shuffle tree inside a warp, then the two warps of a
+// quarter).  Tokens are read through the permutation when there is one.
 constexpr int PAMA_THREADS = 256;
 constexpr int PAMA_CHUNK = 32;
 
 template <int D>
 size_t pama_smem_bytes(int nb) {
   const int nbp = (nb + 31) & ~31;
-  return ((size_t)(128 + PAMA_CHUNK) * (D + 4) + nbp + 2 * 2 * 128 + 8 * 16) * sizeof(float);
+  return ((size_t)(128 + PAMA_CHUNK) * (D + 4) + nbp + 4 * 128 * 2 + 8 * 8) * sizeof(float);
 }
 
 template <int D>
@@ -299,8 +300,8 @@ __global__ void __launch_bounds__(PAMA_THREADS, 2) pama_kernel(RouteArgs a,
   float* Qs = sm;                          // [128][QS]
   float* Ks = Qs + 128 * QS;               // [PAMA_CHUNK][QS]
   float* p = Ks + PAMA_CHUNK * QS;         // [nbp]
-  float* ml = p + nbp;                     // [2 halves][128 tokens][m, l]
-  float* part = ml + 2 * 2 * 128;          // [8 warps][16]
+  float* ml = p + nbp;                     // [4 quarters][128 tokens][m, l]
+  float* part = ml + 4 * 128 * 2;          // [8 warps][8]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int i = blockIdx.x, bh = blockIdx.y;
   const int ni = (i == a.nb - 1) ? a.n_last : a.b;
@@ -332,7 +333,7 @@ __global__ void __launch_bounds__(PAMA_THREADS, 2) pama_kernel(RouteArgs a,
   const float* kbar = a.kbar + (size_t)bh * a.nb * D;
   const float inv_sqrt_d = 1.0f / sqrtf((float)D);
   const float lg_b = logf((float)a.b), lg_last = logf((float)a.n_last);
-  const int r = tid & 127, jh = tid >> 7;
+  const int ra = tid & 63, rb = ra + 64, qq = tid >> 6;
   const int nch = (a.nb + PAMA_CHUNK - 1) / PAMA_CHUNK;
 
   auto load_chunk = [&](int c) {
@@ -346,73 +347,98 @@ __global__ void __launch_bounds__(PAMA_THREADS, 2) pama_kernel(RouteArgs a,
     }
     __syncthreads();
   };
-  auto logits = [&](int c, float (&sv)[16]) {
-    float acc[16];
+  // logits of tokens ra, rb against blocks qq*8 .. qq*8+7 of chunk c
+  auto logits = [&](int c, float (&sa)[8], float (&sb)[8]) {
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) acc[jj] = 0.f;
-    const float4* q4 = reinterpret_cast<const float4*>(Qs + r * QS);
+    for (int jj = 0; jj < 8; ++jj) sa[jj] = sb[jj] = 0.f;
+    const float4* qa4 = reinterpret_cast<const float4*>(Qs + ra * QS);
+    const float4* qb4 = reinterpret_cast<const float4*>(Qs + rb * QS);
 #pragma unroll 2
     for (int k4 = 0; k4 < D / 4; ++k4) {
-      const float4 q = q4[k4];
+      const float4 qa = qa4[k4], qb = qb4[k4];
 #pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
-        const float4 kv = reinterpret_cast<const float4*>(Ks + (jh * 16 + jj) * QS)[k4];
-        acc[jj] = fmaf(q.x, kv.x, acc[jj]);
-        acc[jj] = fmaf(q.y, kv.y, acc[jj]);
-        acc[jj] = fmaf(q.z, kv.z, acc[jj]);
-        acc[jj] = fmaf(q.w, kv.w, acc[jj]);
+      for (int jj = 0; jj < 8; ++jj) {
+        const float4 kv = reinterpret_cast<const float4*>(Ks + (qq * 8 + jj) * QS)[k4];
+        sa[jj] = fmaf(qa.x, kv.x, sa[jj]);
+        sa[jj] = fmaf(qa.y, kv.y, sa[jj]);
+        sa[jj] = fmaf(qa.z, kv.z, sa[jj]);
+        sa[jj] = fmaf(qa.w, kv.w, sa[jj]);
+        sb[jj] = fmaf(qb.x, kv.x, sb[jj]);
+        sb[jj] = fmaf(qb.y, kv.y, sb[jj]);
+        sb[jj] = fmaf(qb.z, kv.z, sb[jj]);
+        sb[jj] = fmaf(qb.w, kv.w, sb[jj]);
       }
     }
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) {
-      const int j = c * PAMA_CHUNK + jh * 16 + jj;
-      sv[jj] = j < a.nb ? fmaf(acc[jj], inv_sqrt_d, j == a.nb - 1 ? lg_last : lg_b) : -INFINITY;
+    for (int jj = 0; jj < 8; ++jj) {
+      const int j = c * PAMA_CHUNK + qq * 8 + jj;
+      const float bias = j == a.nb - 1 ? lg_last : lg_b;
+      sa[jj] = j < a.nb ? fmaf(sa[jj], inv_sqrt_d, bias) : -INFINITY;
+      sb[jj] = j < a.nb ? fmaf(sb[jj], inv_sqrt_d, bias) : -INFINITY;
     }
   };
-
-  // pass 1: per token, running max and sum over this thread's half of every chunk
-  float m = -INFINITY, l = 0.f;
-  for (int c = 0; c < nch; ++c) {
-    load_chunk(c);
-    float sv[16];
-    logits(c, sv);
+  auto online = [&](const float (&sv)[8], float& m, float& l) {
     float cm = sv[0];
 #pragma unroll
-    for (int jj = 1; jj < 16; ++jj) cm = fmaxf(cm, sv[jj]);
+    for (int jj = 1; jj < 8; ++jj) cm = fmaxf(cm, sv[jj]);
     const float mn = fmaxf(m, cm);
     if (mn > -INFINITY) {
       float add = 0.f;
 #pragma unroll
-      for (int jj = 0; jj < 16; ++jj) add += expf(sv[jj] - mn);
+      for (int jj = 0; jj < 8; ++jj) add += expf(sv[jj] - mn);
       l = l * expf(m - mn) + add;
       m = mn;
     }
+  };
+
+  // pass 1: per token, running max and sum over this thread's quarter of every chunk
+  float ma = -INFINITY, la = 0.f, mb = -INFINITY, lb = 0.f;
+  for (int c = 0; c < nch; ++c) {
+    load_chunk(c);
+    float sa[8], sb[8];
+    logits(c, sa, sb);
+    online(sa, ma, la);
+    online(sb, mb, lb);
   }
-  ml[(jh * 128 + r) * 2] = m;
-  ml[(jh * 128 + r) * 2 + 1] = l;
+  ml[(qq * 128 + ra) * 2] = ma;
+  ml[(qq * 128 + ra) * 2 + 1] = la;
+  ml[(qq * 128 + rb) * 2] = mb;
+  ml[(qq * 128 + rb) * 2 + 1] = lb;
   __syncthreads();
-  const float m0 = ml[r * 2], l0 = ml[r * 2 + 1], m1 = ml[(128 + r) * 2], l1 = ml[(128 + r) * 2 + 1];
-  const float M = fmaxf(m0, m1);
-  const float L = (m0 > -INFINITY ? l0 * expf(m0 - M) : 0.f) + (m1 > -INFINITY ? l1 * expf(m1 - M) : 0.f);
-  const float invL = (r < ni && L > 0.f) ? 1.f / L : 0.f;   // padding rows contribute nothing
+  auto combine = [&](int r, float& M, float& invL) {
+    M = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) M = fmaxf(M, ml[(q * 128 + r) * 2]);
+    float L = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float mq = ml[(q * 128 + r) * 2];
+      if (mq > -INFINITY) L += ml[(q * 128 + r) * 2 + 1] * expf(mq - M);
+    }
+    invL = (r < ni && L > 0.f) ? 1.f / L : 0.f;   // padding rows contribute nothing
+  };
+  float Ma, iLa, Mb, iLb;
+  combine(ra, Ma, iLa);
+  combine(rb, Mb, iLb);
 
   // pass 2: probabilities, summed over the block's tokens
   for (int c = 0; c < nch; ++c) {
     load_chunk(c);
-    float sv[16];
-    logits(c, sv);
+    float sa[8], sb[8];
+    logits(c, sa, sb);
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) {
-      float w = sv[jj] > -INFINITY ? expf(sv[jj] - M) * invL : 0.f;
+    for (int jj = 0; jj < 8; ++jj) {
+      float w = (sa[jj] > -INFINITY ? expf(sa[jj] - Ma) * iLa : 0.f) +
+                (sb[jj] > -INFINITY ? expf(sb[jj] - Mb) * iLb : 0.f);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) w += __shfl_xor_sync(0xffffffffu, w, o);
-      if (lane == 0) part[warp * 16 + jj] = w;
+      if (lane == 0) part[warp * 8 + jj] = w;
     }
     __syncthreads();
     if (tid < PAMA_CHUNK) {
-      const int h = tid >> 4, jj = tid & 15;
-      const float t = ((part[(4 * h + 0) * 16 + jj] + part[(4 * h + 1) * 16 + jj]) +
-                       part[(4 * h + 2) * 16 + jj]) + part[(4 * h + 3) * 16 + jj];
+      // block tid of the chunk: quarter tid / 8, summed over its two warps
+      const int q = tid >> 3, jj = tid & 7;
+      const float t = part[(2 * q) * 8 + jj] + part[(2 * q + 1) * 8 + jj];
       const int j = c * PAMA_CHUNK + tid;
       if (j < a.nb) p[j] = t / (float)ni;
     }
