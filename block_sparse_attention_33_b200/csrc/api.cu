@@ -205,6 +205,13 @@ spattn_status_t spattn_plan_ex(spattn_plan_t* out, int B, int H, int N, int d, i
     // made, any shape (used to cross-check the two GPU paths).
     const char* env = getenv("SPATTN_ATTN");
     p.use_tc = spattn::attend_tc_supported(p) && !(env && strcmp(env, "mma") == 0);
+    // Failure-path test: with SPATTN_TEST_WAIT_TIMEOUT=1 in the environment
+    // when the plan is made, the tcgen05 attention's first CTA waits on an
+    // mbarrier phase that nothing completes; the bounded wait gives up after
+    // its limit (~2 s), the CTA winds down, and spattn_check reports
+    // SPATTN_ERR_TIMEOUT.  Nothing faults or hangs.
+    const char* st = getenv("SPATTN_TEST_WAIT_TIMEOUT");
+    p.test_stall = (st && strcmp(st, "1") == 0) ? 1 : 0;
   }
   if (perm_host) {
     cudaError_t e = cudaMalloc(&P->perm_dev, sizeof(int32_t) * (size_t)N);

@@ -101,7 +101,8 @@ struct TcArgs {
   __nv_bfloat16* o;
   int32_t* ctrl;
   int N, nb, n_last, residual, items;
-  float sl2;  // log2(e) / sqrt(d)
+  int test_stall;  // failure-path test (see Problem::test_stall)
+  float sl2;       // log2(e) / sqrt(d)
 };
 
 // One work item as described by the producer warp.  Two slots: the producer
@@ -431,6 +432,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       // p at that reference; owe: factor O_h owes once PV(g-1) is done.
       float m = -INFINITY, l = 0.f, owe = 1.f;
 
+      // failure-path test: phase 0 of the drain barrier completes only after
+      // an abort, so this bounded wait runs out and aborts the CTA
+      if (a.test_stall && blockIdx.x == 0 && n == 0 && T > 0 && !(ok = wait_warp(bar(B_DRAIN), 0u, 15)))
+        break;
       for (int t = 0; t < T; ++t) {
         const int g = gt + t, b = g & 1;
         if (!(ok = wait_warp(bar(B_SFULL0 + b), (uint32_t)(g >> 1) & 1u, 7))) break;
@@ -621,6 +626,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       gt += T;
       if (T > 0) ++qn;
     }
+    // a role that left early (abort) may still have TMEM accesses in flight
+    tc::tmem_wait_ld();
+    tc::tmem_wait_st();
+    tc::tc_fence_before();
   }
   __syncthreads();
   if (warp == WARP_MMA) {
@@ -743,6 +752,7 @@ cudaError_t launch_attend_tc(const Problem& p, const void* Q, const void* K, con
   a.N = p.N; a.nb = p.nb; a.n_last = p.n_last; a.residual = p.residual;
   a.sl2 = 1.4426950408889634f / sqrtf((float)p.d);
   a.items = p.BH * p.nb;
+  a.test_stall = p.test_stall;
   // The work counter resets itself at the end of every launch; it starts
   // from zero after the routing call's control-block clear.  A caller CSR
   // may come with a workspace that was never routed: clear the error word

@@ -19,6 +19,8 @@ struct Problem {
   int residual;
   int use_tc;           // attention on the tcgen05 kernel (else warp MMA)
   int routing;          // ROUTING_CENTROID or ROUTING_PAMA
+  int test_stall;       // failure-path test: CTA 0 of the attention waits on a phase
+                        // that never completes, so its bounded wait runs out
   const int32_t* perm;  // device, NULL if none
 };
 
