@@ -6,13 +6,13 @@
 //
 // Each CTA owns one work item = (head, query block i) of b query rows
 // (b/16 warps, 16 rows per warp).  Per query token it runs one online
-// softmax (Sol-Attn abstract: "a single online-softmax pass") over
+// softmax (Sol-Attn abstract: one online-softmax sweep over the selection) over
 //   * the exact tokens of every kept key block (CSR row i), in 64-token
 //     sub-tiles; tokens past n_j of the partial last block are masked;
 //   * in residual mode, the block centroids as pseudo-keys: tile c holds
 //     Kbar_j, Vbar_j for j in [64c, 64c+64) with logit bias ln n_j for a
-//     dropped block and -inf for a kept one (Sol-Attn: reuse the proxy
-//     scores of the unselected blocks).
+//     dropped block and -inf for a kept one (Sol-Attn abstract: skipped
+//     blocks approximated from the router's scores).
 // The epilogue divides by the softmax sum and scatters rows back through the
 // permutation (O[perm[n]] = Op[n]).
 #include "common.cuh"

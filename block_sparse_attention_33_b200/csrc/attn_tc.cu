@@ -1,11 +1,13 @@
 // Routed block-sparse attention on Blackwell tensor cores, with the residual
 // pseudo-keys folded into the same online softmax.
 //
-// One CTA per work item (head bh, query block i of 128 tokens), one CTA per
-// SM; items are launched longest budget first (the counting sort of the
-// routing step).  TMEM (512 columns) holds two S buffers and two O
-// accumulators, one per 64-key half of every key tile, so the MMA of task
-// t+1 runs while the softmax of task t is computed.  Warp roles:
+// Persistent: one CTA per SM loops over work items (head bh, query block i
+// of 128 tokens) taken from a device ticket counter in the routing step's
+// order (heads grouped so their K/V stay in L2, longest budget first); the
+// last CTA to retire resets the counter.  TMEM (512 columns) holds two S
+// buffers and two O accumulators, one per 64-key half of every key tile, so
+// the MMA of task t+1 runs while the softmax of task t is computed.  Warp
+// roles:
 //
 //   warps 0-7  softmax.  Warp w owns TMEM lane quarter w % 4 (query rows
 //              32(w%4) .. +31) and key half h = w / 4 of every S tile, and runs
@@ -19,24 +21,26 @@
 //              recomputed against its own maximum).  Optionally a fixed
 //              share of the exponentials runs on the FMA pipe (tc::ex2_fma2);
 //              measured on B200 the MUFU-only form is faster for this
-//              structure, so the share defaults to zero.  P(t) is written as packed bf16 over the warp's own,
-//              already read, columns of S(t).  The epilogue merges the two
+//              structure, so the share defaults to zero.  P(t) is written as
+//              packed bf16 over the warp's own, already read, columns of S(t).  The epilogue merges the two
 //              halves of each row, normalises and stores the row, scattered
 //              through perm.
-//   warp 8     producer: TMA loads of the Q tile and of the K and V tiles
-//              (128 tokens x d, 128-byte swizzle, no multicast) through one
-//              ring of shared-memory slots, in the order the MMA consumes them.
+//   warp 8     producer: takes the next ticket and describes the item
+//              (kept bitmap, residual tiles) in a second slot, then issues
+//              TMA loads of the Q tile and of the K and V tiles (128 tokens x
+//              d, 128-byte swizzle, no multicast) through one ring of
+//              shared-memory slots, in the order the MMA consumes them.
 //   warp 9     MMA issuer: S = Q K^T (both operands in shared memory) into
 //              S buffer t & 1, and O_h += P_h V_h for both halves (P from
 //              TMEM, V from shared memory), tcgen05.mma with fp32
 //              accumulation in TMEM.
 //
-// Tasks of an item: its kept key blocks (CSR row; Sol-Attn: "a single
-// online-softmax pass" over the selected blocks), then, in residual mode,
+// Tasks of an item: its kept key blocks (one online-softmax sweep over the
+// selected blocks, as in the Sol-Attn abstract), then, in residual mode,
 // every 128-row tile of the bf16 block centroids Kbar/Vbar that holds a
 // dropped block, as pseudo-keys with logit bias ln n_j for a dropped block and
-// -inf for a kept one (Sol-Attn: reuse the proxy scores of unselected
-// blocks).  Tokens past n_j of a partial last block are masked; TMA
+// -inf for a kept one (Sol-Attn abstract: skipped blocks approximated from the router's
+// scores).  Tokens past n_j of a partial last block are masked; TMA
 // zero-fills rows past N.
 //
 // Every mbarrier wait is bounded (tc::mbar_wait): on a timeout the CTA

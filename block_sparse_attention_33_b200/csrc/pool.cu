@@ -1,7 +1,7 @@
 // Token gather (optional permutation) fused with block-mean pooling.
 //
 // Blocks are represented by the mean of their tokens (PARK page, abstract and
-// section 4: "averaged representations of query and key blocks").  With a
+// section 4: query and key blocks are compared through their averages).  With a
 // permutation, the kernel reads X[perm[n]] and writes the permuted copy Xp[n]
 // in the same pass (DFSAttn abstract: Hilbert reordering before blocking), so
 // Q/K/V are read from HBM exactly once.

@@ -23,7 +23,7 @@
  *   4. each query token q of block i runs one softmax over the exact tokens
  *      of its kept blocks; with residual != 0 every dropped block j adds one
  *      pseudo-key with logit q . Kbar_j / sqrt(d) + ln n_j and value Vbar_j
- *      (Sol-Attn: reuse the proxy scores of unselected blocks);
+ *      (Sol-Attn abstract: skipped blocks approximated from the router's scores);
  *   5. the output is scattered back, O[perm[n]] = Op[n], bf16.
  *
  * Conventions for every call:

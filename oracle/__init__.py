@@ -12,13 +12,13 @@ plainly and slowly, in float64 from the exact bf16 inputs:
 * proxy logit Qbar_i . Kbar_j / sqrt(d) + ln n_j -- the centroid estimate
   that PARK page section D.2 shows to be a Jensen lower bound on the exact
   block log-mass -- and its softmax over key blocks;
-* Top-p routing: blocks in descending estimated importance until the
-  cumulative estimate reaches the threshold (PARK page section 3.2), with a
-  dynamic, clamped budget (Sol-Attn abstract, thelatestinai page);
+* Top-p routing: blocks taken in descending estimated importance while the
+  accumulated estimate is still below the threshold (PARK page section 3.2),
+  with a dynamic, clamped budget (Sol-Attn abstract, thelatestinai page);
 * one softmax per query token over the exact tokens of its kept blocks, plus
   (residual mode) one pseudo-key per dropped block that reuses the block's
-  proxy score (Sol-Attn abstract: "reusing the proxy scores of unselected
-  blocks");
+  proxy score (Sol-Attn abstract: the skipped blocks are approximated from
+  the scores the router already computed);
 * optional token reordering before blocking and its inverse after
   (DFSAttn abstract: Hilbert curve-based token reordering).
 

@@ -9,8 +9,9 @@ design notes):
 
 * natural logarithm in the ln n_j term; scale 1/sqrt(d) on every logit, the
   proxy and the pseudo-keys alike;
-* "until the cumulative estimate reaches the threshold" (PARK page 3.2) is
-  read as: order blocks by p descending, ties to the lower block index, and
+* the Top-p rule of PARK page 3.2 (blocks taken in descending estimated
+  importance while the accumulated estimate is below the threshold) is read
+  as: order blocks by p descending, ties to the lower block index, and
   keep rank r iff the mass of the ranks before it is < tau; so the kept count
   k* is the length of the shortest prefix whose mass is >= tau;
 * tau >= 1 keeps every block (no prefix shorter than nb is needed, and
@@ -85,7 +86,7 @@ def block_means(X: np.ndarray, b: int) -> np.ndarray:
     """Block means over the token axis: [..., N, d] -> [..., nb, d] (fp64).
 
     Blocks are represented by the average of their tokens (PARK page,
-    abstract: "averaged representations of query and key blocks").
+    abstract: query and key blocks are compared through their averages).
     """
     N = X.shape[-2]
     n = block_sizes(N, b)
