@@ -1,24 +1,29 @@
-// Proxy logits, block softmax, Top-p selection, CSR of kept blocks.
+// Proxy logits, block softmax, Top-p selection, kept lists of every query
+// block, work order, CSR.
 //
 // Block importance (PARK page 3.2): p_ij = softmax_j(Qbar_i . Kbar_j / sqrt(d)
 // + ln n_j), the centroid estimate of the block log-mass (PARK D.2).  Blocks
-// are taken in descending p until the cumulative mass reaches tau (PARK 3.2
-// "Top-p"), ties to the lower block index, budget clamped to [kmin, kmax]
+// are taken in descending p until the cumulative mass reaches tau (PARK 3.2,
+// Top-p), ties to the lower block index, budget clamped to [kmin, kmax]
 // (Sol-Attn abstract: dynamic but controllable budgets).  The proxy map never
-// leaves shared memory.
+// leaves shared memory.  pama_kernel computes p_i instead by per-query
+// attention-mass aggregation (PARK page 5.1) and shares the selection.
 //
 // Selection without a sort: with p >= 0 the float bit pattern orders p, and
 // the mass G(u) = sum of p_j whose bits exceed u is monotone in u.  The kept
 // prefix is {p_j > v} plus the first few blocks with p_j == v (ascending j),
-// where v is the smallest value whose strictly-larger mass is < tau; a binary
-// search over the bit patterns finds v with one warp reduction per step.  The
-// same search on the count #{p_j > u} yields the top-k set when the clamp
-// binds.  Kept blocks are then emitted in ascending j with warp ballots.
+// where v is the smallest value whose strictly-larger mass is < tau.  A
+// search over the bit patterns finds v: 32-way for rows of at most 128
+// blocks (each lane evaluates one candidate over the whole row), binary with
+// one warp reduction per step otherwise.  The same search on the count
+// #{p_j > u} yields the top-k set when the clamp binds.  Kept blocks are then
+// emitted in ascending j with warp ballots.
 //
 // route_kernel: one CTA per (ROWS query blocks, head), ROWS = 4, 8 or 16 by
-// the number of blocks so that small problems still fill the GPU; 8 warps;
-// the proxy tile S[ROWS][nb] is computed with fp32 FMAs (no TF32/BF16: a logit error of 1e-2
-// would move cumulative mass by more than the 1e-4 comparison margin).
+// the number of blocks so that small problems still fill the GPU; 8 warps.
+// The proxy tile S[ROWS][nb] is computed with fp32 FMAs, not TF32/BF16: a
+// logit error of 1e-2 would move the cumulative mass by more than the 1e-4
+// comparison margin.
 #include <algorithm>
 #include <atomic>
 
