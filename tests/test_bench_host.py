@@ -1,0 +1,46 @@
+"""Host-side logic of bench.py that needs no GPU: the FLOP count behind the
+headline metric, checked against the oracle's definition."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+
+@pytest.mark.parametrize("name,ov", [("tiny", {}), ("medium", {"H": 3}), ("wan", {"H": 2}),
+                                     ("tiny", {"residual": 0, "grid": (1, 5, 100), "b": 64})])
+def test_bench_flop_count_matches_oracle_definition(name, ov):
+    """The bench's vectorised FLOP count from a CSR equals the oracle's
+    per-row count (4 d per exact query-key pair and per query-pseudo-key
+    pair) on random kept sets, including the partial last block."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    from oracle import spattn_ref as R
+    from workloads import get_config
+    w = get_config(name, **ov)
+    nb = w.nb
+    n = R.block_sizes(w.N, w.b)
+    rng = np.random.default_rng(7)
+    kept, rp, ci = {}, [0], []
+    for bi in range(w.B):
+        for hi in range(w.H):
+            rows = []
+            for i in range(nb):
+                k = int(rng.integers(1, nb + 1))
+                ks = np.sort(rng.choice(nb, size=k, replace=False))
+                if i == 0:
+                    ks = np.unique(np.append(ks, nb - 1))      # the partial block at least once
+                rows.append(ks)
+                ci.extend(ks.tolist())
+                rp.append(rp[-1] + len(ks))
+            kept[(bi, hi)] = rows
+    ex, rs = bench.attention_flops(np.asarray(rp), np.asarray(ci), w, nb)
+    want_ex = want_rs = 0
+    for key, rows in kept.items():
+        e, r = R.attention_flops(rows, n, bool(w.residual), w.d)
+        want_ex += e
+        want_rs += r
+    assert (ex, rs) == (want_ex, want_rs)

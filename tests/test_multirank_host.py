@@ -67,3 +67,4 @@ def test_single_process_is_pass_through_and_throughput():
     assert maxes == [3.5, 1.25] and sums == [42.0]
     # 2e12 FLOPs in 1 ms is 2000 TFLOP/s
     assert bench.job_throughput(2e12, 1.0) == pytest.approx(2000.0)
+
