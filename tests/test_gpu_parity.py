@@ -150,3 +150,33 @@ def test_bad_csr_index_is_flagged_not_faulted():
     res = run_library(w, Q, K, V, kept_csr=(rp, ci))
     import block_sparse_attention_33_b200 as sp
     assert res["status"] == sp.ERR_DEVICE
+
+
+# The same edge cases on 128-token blocks (d = 128), i.e. through the
+# persistent tcgen05 attention kernel rather than the warp-MMA one.
+EDGE_TC = [
+    ("nb=1, N<b", dict(grid=(1, 1, 100))),
+    ("N%b=1", dict(grid=(1, 3, 43))),                      # 129 tokens: last block of 1
+    ("N%b=b-1", dict(grid=(1, 1, 255))),
+    ("kmin=kmax", dict(kmin=3, kmax=3)),
+    ("kmax>nb", dict(kmax=1000)),
+    ("tau<=0", dict(tau=-0.5, kmin=2)),
+    ("tau>1", dict(tau=1.5)),
+    ("B=2", dict(B=2, H=3)),
+    ("no residual, kmax=2", dict(residual=0, kmax=2)),
+    ("d=64", dict(d=64)),
+]
+
+
+@pytest.mark.parametrize("desc,ov", EDGE_TC, ids=[e[0] for e in EDGE_TC])
+def test_edge_cases_tcgen05(desc, ov):
+    base = dict(grid=(2, 8, 64), d=128, b=128, H=2, kmax=8)
+    base.update(ov)
+    w = get_config("tiny", **base)
+    Q, K, V = make_qkv(w)
+    res = run_library(w, Q, K, V)
+    assert res["status"] == 0
+    _assert_ok(oracle_check(w, Q, K, V, res))
+    nb = w.nb
+    k = np.diff(res["row_ptr"])
+    assert np.all(k >= min(w.kmin, nb)) and np.all(k <= min(w.kmax, nb))
