@@ -134,8 +134,9 @@ spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, c
  * followed by spattn_attend with NULL row_ptr/col_idx attends the new
  * inputs with the kept lists of that earlier route (the residual uses the
  * new inputs' means).
- *   row_ptr, col_idx  NULL to use the workspace CSR of the last route, or a
- *                     caller CSR in the layout above (device).  Block
+ *   row_ptr, col_idx  NULL to use the kept lists the last spattn_route left
+ *                     in the workspace, or a caller CSR in the layout above
+ *                     (device).  Block
  *                     indices outside [0, nb) are skipped and flagged
  *                     (SPATTN_ERR_DEVICE from spattn_check).  With a
  *                     caller CSR the call first clears the workspace's
@@ -149,7 +150,8 @@ spattn_status_t spattn_attend(spattn_plan_t plan, const void* Q, const void* K, 
                               const int32_t* row_ptr, const int32_t* col_idx, void* O,
                               void* workspace, void* stream);
 
-/* The whole path: spattn_route (CSR in the workspace only) + spattn_attend. */
+/* The whole path: spattn_route (kept lists in the workspace only) +
+ * spattn_attend. */
 spattn_status_t spattn_forward(spattn_plan_t plan, const void* Q, const void* K, const void* V,
                                void* O, void* workspace, void* stream);
 
@@ -159,7 +161,11 @@ spattn_status_t spattn_means(spattn_plan_t plan, const void* workspace, float* Q
                              float* Kbar, float* Vbar, void* stream);
 
 /* Synchronise `stream` and report the device error word of this workspace:
- * SPATTN_OK, SPATTN_ERR_DEVICE or SPATTN_ERR_TIMEOUT.  Clears the word. */
+ * SPATTN_OK, SPATTN_ERR_DEVICE or SPATTN_ERR_TIMEOUT.  Clears the word.
+ * (To exercise the timeout path without a fault: with the environment
+ * variable SPATTN_TEST_WAIT_TIMEOUT=1 set when a plan is made, the first CTA
+ * of that plan's attention waits on a phase nothing completes, gives up
+ * after about two seconds, and this call then reports SPATTN_ERR_TIMEOUT.) */
 spattn_status_t spattn_check(spattn_plan_t plan, void* workspace, void* stream);
 
 /* Host helper (no CUDA): perm[new] = old ordering the tokens of a T x Hs x W
