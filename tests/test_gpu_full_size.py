@@ -63,3 +63,18 @@ def test_full_size(name, ov):
           f"rel-L2 {fig['rel_l2']:.2e}")
     assert fig["bad"] == 0, fig
     assert fig["max_abs"] < 2e-2 and fig["rel_l2"] < 4e-3, fig
+
+
+def test_largest_supported_block_count():
+    """nb = 2048 (the supported maximum): 262144 tokens of one head in
+    128-token blocks, through the tcgen05 path, sixteen centroid tiles per
+    item in residual mode; sampled rows against the oracle."""
+    w = get_config("tiny", grid=(1, 512, 512), d=128, b=128, H=1, kmax=16, tau=0.9)
+    assert w.nb == 2048
+    Q, K, V = make_qkv(w)
+    res = run_library(w, Q, K, V)
+    assert res["status"] == 0
+    rows = sample_rows(w, res, None)
+    fig = oracle_check(w, Q, K, V, res, rows=rows)
+    assert fig["bad"] == 0, fig
+    assert fig["max_abs"] < 2e-2 and fig["rel_l2"] < 4e-3, fig
