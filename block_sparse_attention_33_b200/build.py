@@ -13,6 +13,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libspattn.so")
+STAMP = LIB + ".flags"   # extra compiler flags of the library on disk
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -35,8 +36,20 @@ def _deps():
         + glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def up_to_date() -> bool:
+def _stamp_of(extra) -> str:
+    return " ".join(extra)
+
+
+def up_to_date(extra=()) -> bool:
+    """The library exists, is newer than every source, and was built with
+    the same extra flags."""
     if not os.path.exists(LIB):
+        return False
+    try:
+        with open(STAMP) as f:
+            if f.read() != _stamp_of(extra):
+                return False
+    except OSError:
         return False
     t = os.path.getmtime(LIB)
     return all(os.path.getmtime(f) <= t for f in _deps())
@@ -44,8 +57,10 @@ def up_to_date() -> bool:
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     """Compile every .cu under csrc/ and link libspattn.so next to this file."""
-    if not force and up_to_date():
+    if not force and up_to_date(extra):
         return LIB
+    # objects built with other flags cannot be reused
+    force = force or not os.path.exists(STAMP) or open(STAMP).read() != _stamp_of(extra)
     nvcc = _nvcc()
     os.makedirs(BUILD, exist_ok=True)
     hdr_t = max(os.path.getmtime(f) for f in _deps() if not f.endswith(".cu"))
@@ -72,6 +87,8 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(_stamp_of(extra))
     return LIB
 
 
