@@ -141,6 +141,36 @@ def job_throughput(total_flops, step_ms):
     return total_flops / (step_ms * 1e-3) / 1e12
 
 
+def attention_recall(q, k, row_ptr, col_idx, b, nb, perm=None, rows_per_head=64, seed=0):
+    """Attention recall of the kept mask (PARK page 3.2: the share of the
+    full attention weight that the kept blocks cover), averaged over a
+    seeded sample of query tokens per head.  q, k: [B, H, N, d] torch
+    tensors (any device); row_ptr/col_idx: the CSR (numpy); perm: the
+    token permutation (gather) or None.  Dense softmax in fp32 on the
+    sampled rows only."""
+    import torch
+    B, H, N, d = q.shape
+    rng = np.random.default_rng(seed)
+    total, count = 0.0, 0
+    for bi in range(B):
+        for hi in range(H):
+            qp, kp = q[bi, hi], k[bi, hi]
+            if perm is not None:
+                pi = torch.as_tensor(np.asarray(perm, dtype=np.int64), device=q.device)
+                qp, kp = qp[pi], kp[pi]
+            sel = np.sort(rng.choice(N, size=min(rows_per_head, N), replace=False))
+            logits = (qp[torch.as_tensor(sel, device=q.device)].float() @ kp.float().T) / float(d) ** 0.5
+            w = torch.softmax(logits, dim=-1).cpu().numpy()          # [rows, N]
+            blk = np.arange(N) // b
+            for ri, tok in enumerate(sel):
+                row = (bi * H + hi) * nb + tok // b
+                kept = col_idx[row_ptr[row]:row_ptr[row + 1]]
+                mask = np.isin(blk, kept)
+                total += float(w[ri, mask].sum())
+                count += 1
+    return total / max(count, 1)
+
+
 def attention_flops(row_ptr, col_idx, w, nb):
     """(exact, residual) FLOPs: 4 d per query-key pair, from the CSR."""
     b, N, d = w.b, w.N, w.d
@@ -395,6 +425,11 @@ def run_ours(args):
     exact, resid = attention_flops(rp, ci, w, plan.nb)
     step_flops = exact + resid
     kept_frac = float(np.diff(rp).sum()) / (B * H * plan.nb * plan.nb)
+    try:   # a diagnostic: never let it stop the measurement
+        recall = attention_recall(q, k, rp, ci, w.b, plan.nb, perm,
+                                  rows_per_head=max(8, 512 // max(1, B * H)))
+    except Exception as e:  # pragma: no cover
+        recall = {"error": repr(e)[:200]}
     dense_flops = 4 * N * N * d * B * H
 
     clocks = ClockSampler(local)
@@ -494,6 +529,7 @@ def run_ours(args):
             "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None,
             "dense_ms_per_step": dense_ms,
             "kept_fraction": kept_frac,
+            "attention_recall": recall,
             "flops_exact": exact, "flops_residual": resid,
             "kernels_ms": {"route_total": route_ms, "attend": attend_ms, "pool": pool_ms},
             "reuse_step": {"ms_per_step": reuse_ms,

@@ -44,3 +44,22 @@ def test_bench_flop_count_matches_oracle_definition(name, ov):
         want_ex += e
         want_rs += r
     assert (ex, rs) == (want_ex, want_rs)
+
+
+def test_attention_recall_extremes_and_a_hand_case():
+    """Recall is 1 when every block is kept, and for a hand-built case it is
+    the softmax mass of the kept block: two blocks of two tokens, one query
+    whose logits are (ln 3, ln 3, 0, 0) (d = 1), kept = {0}: 6/8."""
+    sys.path.insert(0, ROOT)
+    import math
+    import numpy as np
+    import torch
+    import bench
+    B, H, N, d, b = 1, 1, 4, 1, 2
+    q = torch.full((B, H, N, d), math.log(3.0), dtype=torch.float64)
+    k = torch.tensor([1.0, 1.0, 0.0, 0.0], dtype=torch.float64).view(B, H, N, d)
+    rp_all = np.array([0, 2, 4]); ci_all = np.array([0, 1, 0, 1])
+    assert bench.attention_recall(q, k, rp_all, ci_all, b, 2, rows_per_head=4) == 1.0
+    rp = np.array([0, 1, 2]); ci = np.array([0, 0])
+    r = bench.attention_recall(q, k, rp, ci, b, 2, rows_per_head=4)
+    assert abs(r - 0.75) < 1e-6
