@@ -197,3 +197,33 @@ def test_tc_routing_reuse_across_calls():
     own = R.forward(QB, KB, VB, w.b, w.tau, w.kmin, w.kmax, w.residual, perm=perm, rows=pick)
     assert any(not np.array_equal(np.sort(a), np.sort(b))
                for key in own["route"] for a, b in zip(own["route"][key]["kept"], kept_a[key]))
+
+
+@pytest.mark.parametrize("perm_on", [False, True])
+def test_writes_stay_inside_workspace_and_output(perm_on):
+    """Canary bytes before and after the workspace and the output tensor are
+    untouched by a full forward (pool, routing, attention; with the Hilbert
+    permutation the pooling also writes the permuted copies)."""
+    import torch
+    import block_sparse_attention_33_b200 as sp
+    from tests.harness import to_dev
+    w = get_config("medium", H=2, tau=0.8)
+    Q, K, V = make_qkv(w)
+    perm = sp.spattn_hilbert_perm(*w.grid) if perm_on else None
+    plan = sp.Plan(w.B, w.H, w.N, w.d, w.b, w.tau, w.kmin, w.kmax, w.residual, perm)
+    pad = 1 << 20
+    try:
+        ws = torch.full((plan.ws_bytes + 2 * pad,), 0xA5, dtype=torch.uint8, device="cuda")
+        plan.workspace = ws[pad:pad + plan.ws_bytes]
+        q, k, v = to_dev(Q), to_dev(K), to_dev(V)
+        n = q.numel()
+        ob = torch.full((n + 2 * (pad // 2),), 7.0, dtype=torch.bfloat16, device="cuda")
+        o = ob[pad // 2:pad // 2 + n].view(q.shape)
+        plan.forward(q, k, v, o)
+        assert plan.check() == 0
+        torch.cuda.synchronize()
+        assert torch.all(ws[:pad] == 0xA5) and torch.all(ws[pad + plan.ws_bytes:] == 0xA5)
+        assert torch.all(ob[:pad // 2] == 7.0) and torch.all(ob[pad // 2 + n:] == 7.0)
+        assert torch.isfinite(o.float()).all()
+    finally:
+        plan.close()
