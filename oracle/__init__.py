@@ -20,12 +20,17 @@ plainly and slowly, in float64 from the exact bf16 inputs:
   proxy score (Sol-Attn abstract: the skipped blocks are approximated from
   the scores the router already computed);
 * optional token reordering before blocking and its inverse after
-  (DFSAttn abstract: Hilbert curve-based token reordering).
+  (DFSAttn abstract: Hilbert curve-based token reordering);
+* the probe-fitted residual correction (SparsePR page, section 2B): exact
+  dense rows for a few probes, a ridge-fitted affine map of their residuals,
+  restricted to the residuals' leading right singular subspace
+  (:mod:`oracle.probe_residual`).
 
 Readings where the pages are silent are listed in the module docstrings of
 :mod:`oracle.spattn_ref` and :mod:`oracle.hilbert`.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+and ``tests/test_oracle_probe_residual.py``
 against closed forms, library routines (torch fp64 softmax attention),
 brute-force enumeration or invariants; none is "parity unpinned".
 """
@@ -35,3 +40,4 @@ from .spattn_ref import (  # noqa: F401
     forward, exact_block_logmass, attention_flops, MASS_MARGIN, TIE_MARGIN,
 )
 from .hilbert import hilbert_index, hilbert_perm  # noqa: F401
+from . import probe_residual  # noqa: F401

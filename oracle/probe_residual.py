@@ -1,0 +1,115 @@
+"""Probe-fitted residual reconstruction, plain fp64 reference (test
+infrastructure only; the product path never imports it).
+
+SparsePR page, section 2B: a few query rows (probes) are evaluated exactly;
+their residual R = O_dense - O_sparse is modelled as an affine function of
+the sparse output, R ~ b + x B, fitted per attention call by ridge
+regression; the fitted correction is restricted to the subspace spanned by
+the leading right singular vectors of the probe residuals and added to the
+sparse output of every other row.  Probe rows keep their exact output.
+
+Readings of points the page leaves open (also listed in the design notes):
+
+* the fit is per (batch, head): one attention call per head;
+* probes: the same number of tokens from every query block, at seeded
+  offsets inside it (stratified across query groups: the page's groups are
+  the blocks here); the probe count is a parameter, since the page gives
+  none;
+* the ridge penalty lam applies to B only, not to the bias b (the usual
+  ridge-with-intercept);
+* the subspace is that of the r leading right singular vectors of R (the
+  probe residual matrix itself, without centring); r = 0 disables the
+  correction.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import numpy as np
+
+from . import spattn_ref
+
+
+def probe_rows(N: int, b: int, seed, per_block: int = 1) -> np.ndarray:
+    """per_block distinct probe tokens in each block of b tokens (all of a
+    block shorter than that), at seeded offsets: ascending token indices in
+    the blocked order.  seed is anything numpy's default_rng accepts."""
+    rng = np.random.default_rng(seed)
+    nb = (N + b - 1) // b
+    out = []
+    for i in range(nb):
+        n_i = min(b, N - i * b)
+        k = min(per_block, n_i)
+        out.extend(i * b + np.sort(rng.choice(n_i, k, replace=False)))
+    return np.asarray(out, dtype=np.int64)
+
+
+def fit_affine_residual(X: np.ndarray, R: np.ndarray, lam: float):
+    """Ridge fit of R ~ 1 b + X B with the penalty lam ||B||^2 (the bias is
+    not penalised): returns (b [d_out], B [d_in, d_out]).  Solved from the
+    normal equations of the augmented design [1, X]."""
+    m, d_in = X.shape
+    A = np.concatenate([np.ones((m, 1)), X], axis=1)
+    D = np.eye(d_in + 1) * lam
+    D[0, 0] = 0.0
+    W = np.linalg.solve(A.T @ A + D, A.T @ R)
+    return W[0], W[1:]
+
+
+def residual_subspace(R: np.ndarray, r: int) -> np.ndarray:
+    """Projector onto the span of the r leading right singular vectors of
+    the probe residuals R [m, d]: [d, d]."""
+    d = R.shape[1]
+    if r <= 0:
+        return np.zeros((d, d))
+    _, _, Vt = np.linalg.svd(R, full_matrices=False)
+    Vr = Vt[:r].T
+    return Vr @ Vr.T
+
+
+def correct(O_sparse: np.ndarray, O_dense_probe: np.ndarray, probes: np.ndarray, lam: float,
+            r: int) -> np.ndarray:
+    """The corrected output of one head: O_sparse [N, d] plus the projected
+    affine correction on every row; probe rows take their exact output."""
+    X = O_sparse[probes]
+    R = O_dense_probe - X
+    bias, B = fit_affine_residual(X, R, lam)
+    P = residual_subspace(R, r)
+    C = (bias[None, :] + O_sparse @ B) @ P
+    out = O_sparse + C
+    out[probes] = O_dense_probe
+    return out
+
+
+def dense_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, rows: np.ndarray) -> np.ndarray:
+    """Exact softmax attention of the query rows `rows` over every key
+    (scale 1/sqrt(d)), fp64: [len(rows), d]."""
+    z = q[rows] @ k.T / math.sqrt(q.shape[1])
+    w = np.exp(z - z.max(axis=1, keepdims=True))
+    return (w @ v) / w.sum(axis=1, keepdims=True)
+
+
+def forward_probe(Q, K, V, b: int, tau: float, kmin: int, kmax: int, residual: int,
+                  probes: np.ndarray, lam: float, r: int, perm: Optional[np.ndarray] = None,
+                  routing: str = "centroid"):
+    """The routed path followed by the probe-fitted correction, per head.
+
+    probes: [B, H, M] token indices in the ORIGINAL order (an input, so that
+    any implementation corrects with the same probes).
+    Returns the routed result of spattn_ref.forward with O replaced by the
+    corrected output and O_sparse holding the uncorrected one."""
+    res = spattn_ref.forward(Q, K, V, b, tau, kmin, kmax, residual, perm=perm, routing=routing)
+    O_sparse = res["O"]
+    O = np.empty_like(O_sparse)
+    B, H = Q.shape[:2]
+    for bi in range(B):
+        for hi in range(H):
+            q = spattn_ref.decode_bf16(Q[bi, hi])
+            k = spattn_ref.decode_bf16(K[bi, hi])
+            v = spattn_ref.decode_bf16(V[bi, hi])
+            rows = np.asarray(probes[bi, hi], dtype=np.int64)
+            O[bi, hi] = correct(O_sparse[bi, hi], dense_rows(q, k, v, rows), rows, lam, r)
+    res["O_sparse"] = O_sparse
+    res["O"] = O
+    return res
