@@ -2,8 +2,10 @@
 
 Argument marshalling only: every step of the path runs in the CUDA kernels of
 ``libspattn.so``.  Tensors may be passed as torch tensors (their device
-pointer is used) or as raw integer addresses.  There is no fallback: if the
-library is missing, importing a function raises.
+pointer is used, after their dtype, device, contiguity and size are checked
+against the plan, so that a wrong tensor is refused before a kernel reads
+past it) or as raw integer addresses (passed through unchecked).  There is
+no fallback: if the library is missing, importing a function raises.
 
 The functions carry the names of the C entry points in ``include/spattn.h``.
 """
@@ -34,6 +36,9 @@ class SpAttnError(RuntimeError):
 
 
 _lib = None
+# plan handle -> (B, H, N, d, nb, col_capacity, workspace_bytes), for the
+# tensor checks of the calls that take a handle
+_PLANS = {}
 
 
 def lib():
@@ -71,16 +76,57 @@ def lib():
     return L
 
 
-def _ptr(x) -> Optional[int]:
-    if x is None:
-        return None
-    if isinstance(x, int):
-        return x
-    if hasattr(x, "data_ptr"):
-        return x.data_ptr()
-    if hasattr(x, "ctypes"):
-        return x.ctypes.data
-    raise TypeError(f"cannot take a pointer of {type(x)}")
+def _devs(*specs):
+    """Pointers of device arguments, each spec (x, name, dtype, numel, exact).
+    A torch tensor must be a contiguous CUDA tensor of `dtype` ("bfloat16",
+    "float32", "int32" or "uint8") holding at least (exactly, if `exact`)
+    `numel` elements; raw addresses and None pass through.  Every argument's
+    dtype, layout and size are checked before any argument's device."""
+    for x, name, dtype, numel, exact in specs:
+        if x is None or isinstance(x, int):
+            continue
+        if not hasattr(x, "data_ptr"):
+            raise TypeError(f"{name}: expected a torch CUDA tensor or an address, got {type(x)}")
+        if str(x.dtype) != "torch." + dtype:
+            raise ValueError(f"{name}: dtype must be torch.{dtype}, got {x.dtype}")
+        if not x.is_contiguous():
+            raise ValueError(f"{name}: must be contiguous")
+        n = x.numel()
+        if (n != numel) if exact else (n < numel):
+            raise ValueError(f"{name}: needs {'exactly' if exact else 'at least'} {numel} "
+                             f"elements, has {n}")
+    out = []
+    for x, name, *_ in specs:
+        if x is None or isinstance(x, int):
+            out.append(x)
+            continue
+        if not x.is_cuda:
+            raise ValueError(f"{name}: must be a CUDA tensor")
+        out.append(x.data_ptr())
+    return out
+
+
+def _shape(plan):
+    try:
+        return _PLANS[plan]
+    except KeyError:
+        raise ValueError("unknown or destroyed plan handle") from None
+
+
+def _tokens(plan, **xs):
+    """Specs of bf16 [B, H, N, d] arguments of a plan."""
+    B, H, N, d = _shape(plan)[:4]
+    return [(x, k, "bfloat16", B * H * N * d, True) for k, x in xs.items()]
+
+
+def _workspace(plan, ws):
+    return (ws, "workspace", "uint8", _shape(plan)[6], False)
+
+
+def _csr(plan, row_ptr, col_idx, col_min):
+    B, H, _, _, nb = _shape(plan)[:5]
+    return [(row_ptr, "row_ptr", "int32", B * H * nb + 1, False),
+            (col_idx, "col_idx", "int32", col_min, False)]
 
 
 def _stream(s) -> Optional[int]:
@@ -117,11 +163,14 @@ def spattn_plan_ex(B, H, N, d, b, tau, kmin, kmax, residual, perm=None, routing=
         pp = perm.ctypes.data
     _check(lib().spattn_plan_ex(ctypes.byref(h), B, H, N, d, b, float(tau), kmin, kmax, residual,
                                 pp, int(routing), ctypes.byref(ws)))
+    nb = (N + b - 1) // b
+    _PLANS[h.value] = (B, H, N, d, nb, B * H * nb * min(kmax, nb), ws.value)
     return h.value, ws.value
 
 
 def spattn_plan_destroy(plan):
     _check(lib().spattn_plan_destroy(plan))
+    _PLANS.pop(plan, None)
 
 
 def spattn_plan_info(plan):
@@ -132,32 +181,41 @@ def spattn_plan_info(plan):
 
 
 def spattn_pool(plan, Q, K, V, workspace, stream=None):
-    _check(lib().spattn_pool(plan, _ptr(Q), _ptr(K), _ptr(V), _ptr(workspace), _stream(stream)))
+    q, k, v, w = _devs(*_tokens(plan, Q=Q, K=K, V=V), _workspace(plan, workspace))
+    _check(lib().spattn_pool(plan, q, k, v, w, _stream(stream)))
 
 
 def spattn_route(plan, Q, K, V, workspace, row_ptr=None, col_idx=None, stream=None):
-    _check(lib().spattn_route(plan, _ptr(Q), _ptr(K), _ptr(V), _ptr(workspace), _ptr(row_ptr),
-                              _ptr(col_idx), _stream(stream)))
+    q, k, v, w, rp, ci = _devs(*_tokens(plan, Q=Q, K=K, V=V), _workspace(plan, workspace),
+                               *_csr(plan, row_ptr, col_idx, _shape(plan)[5]))
+    _check(lib().spattn_route(plan, q, k, v, w, rp, ci, _stream(stream)))
 
 
 def spattn_attend(plan, Q, K, V, O, workspace, row_ptr=None, col_idx=None, stream=None):
-    _check(lib().spattn_attend(plan, _ptr(Q), _ptr(K), _ptr(V), _ptr(row_ptr), _ptr(col_idx),
-                               _ptr(O), _ptr(workspace), _stream(stream)))
+    """row_ptr/col_idx: None (the workspace's kept lists) or a caller CSR;
+    col_idx must hold every entry that row_ptr points at (not checked here)."""
+    q, k, v, o, w, rp, ci = _devs(*_tokens(plan, Q=Q, K=K, V=V, O=O), _workspace(plan, workspace),
+                                  *_csr(plan, row_ptr, col_idx, 0))
+    _check(lib().spattn_attend(plan, q, k, v, rp, ci, o, w, _stream(stream)))
 
 
 def spattn_forward(plan, Q, K, V, O, workspace, stream=None):
-    _check(lib().spattn_forward(plan, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(workspace),
-                                _stream(stream)))
+    q, k, v, o, w = _devs(*_tokens(plan, Q=Q, K=K, V=V, O=O), _workspace(plan, workspace))
+    _check(lib().spattn_forward(plan, q, k, v, o, w, _stream(stream)))
 
 
 def spattn_means(plan, workspace, Qbar=None, Kbar=None, Vbar=None, stream=None):
-    _check(lib().spattn_means(plan, _ptr(workspace), _ptr(Qbar), _ptr(Kbar), _ptr(Vbar),
-                              _stream(stream)))
+    B, H, _, d, nb = _shape(plan)[:5]
+    w, *bars = _devs(_workspace(plan, workspace),
+                     *[(x, n, "float32", B * H * nb * d, False)
+                       for n, x in (("Qbar", Qbar), ("Kbar", Kbar), ("Vbar", Vbar))])
+    _check(lib().spattn_means(plan, w, *bars, _stream(stream)))
 
 
 def spattn_check(plan, workspace, stream=None) -> int:
     """Synchronise and return the device status code (does not raise)."""
-    return lib().spattn_check(plan, _ptr(workspace), _stream(stream))
+    (w,) = _devs(_workspace(plan, workspace))
+    return lib().spattn_check(plan, w, _stream(stream))
 
 
 def spattn_hilbert_perm(T, Hs, W):
@@ -173,8 +231,14 @@ def spattn_route_static(B, H, N, d, b, tau, kmin, kmax, Q, K, row_ptr, col_idx, 
     """Routing with no device allocation (scratch in the library's static
     device array); same CSR as spattn_route.  perm: None or a device int32
     tensor of N entries."""
-    _check(lib().spattn_route_static(B, H, N, d, b, float(tau), kmin, kmax, _ptr(perm), _ptr(Q),
-                                     _ptr(K), _ptr(row_ptr), _ptr(col_idx), _stream(stream)))
+    nb = (N + b - 1) // b
+    tok = B * H * N * d
+    q, k, rp, ci, pp = _devs((Q, "Q", "bfloat16", tok, True), (K, "K", "bfloat16", tok, True),
+                             (row_ptr, "row_ptr", "int32", B * H * nb + 1, False),
+                             (col_idx, "col_idx", "int32", B * H * nb * min(max(kmax, 0), nb), False),
+                             (perm, "perm", "int32", N, True))
+    _check(lib().spattn_route_static(B, H, N, d, b, float(tau), kmin, kmax, pp, q, k, rp, ci,
+                                     _stream(stream)))
 
 
 class Plan:

@@ -363,6 +363,8 @@ spattn_status_t spattn_hilbert_perm(int T, int Hs, int W, int32_t* perm_host) {
   const long long N = (long long)T * Hs * W;
   if (N > (1LL << 31) - 1) return fail(SPATTN_ERR_UNSUPPORTED, "grid too large");
   const int side = std::max(T, std::max(Hs, W));
+  // three axes of `bits` bits each must fit the 64-bit curve index
+  if (side > (1 << 21)) return fail(SPATTN_ERR_UNSUPPORTED, "grid side %d exceeds 2^21", side);
   int bits = 1;
   while ((1 << bits) < side) ++bits;
   std::vector<uint64_t> key((size_t)N);

@@ -136,7 +136,12 @@ spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, c
  * new inputs' means).
  *   row_ptr, col_idx  NULL to use the kept lists the last spattn_route left
  *                     in the workspace, or a caller CSR in the layout above
- *                     (device).  Block
+ *                     (device).  The caller guarantees row_ptr[0] = 0, a
+ *                     non-decreasing row_ptr, at most nb entries per row,
+ *                     and a col_idx that holds every entry row_ptr
+ *                     points at: the library cannot see the size of a device
+ *                     buffer and reads col_idx[row_ptr[r] .. row_ptr[r+1]).
+ *                     A block listed twice is attended twice.  Block
  *                     indices outside [0, nb) are skipped and flagged
  *                     (SPATTN_ERR_DEVICE from spattn_check).  With a
  *                     caller CSR the call first clears the workspace's
@@ -174,7 +179,8 @@ spattn_status_t spattn_check(spattn_plan_t plan, void* workspace, void* stream);
  * The curve is J. Skilling's ("Programming the Hilbert curve", AIP Conf.
  * Proc. 707, 2004) on the smallest power-of-two cube covering the grid,
  * axes (t, h, w); tokens are stably sorted by curve index.  perm_host must
- * hold T*Hs*W int32. */
+ * hold T*Hs*W int32.  A grid side above 2^21 is SPATTN_ERR_UNSUPPORTED (the
+ * curve index of three such axes would not fit 64 bits). */
 spattn_status_t spattn_hilbert_perm(int T, int Hs, int W, int32_t* perm_host);
 
 /* Routing without any device allocation (pooling of Q and K, scoring,

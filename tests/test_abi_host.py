@@ -128,3 +128,43 @@ def test_plan_ex_routing_argument(L):
             assert L.spattn_plan_destroy(h) == sp.OK
         else:
             assert not h.value and b"routing" in L.spattn_last_error()
+
+
+def test_hilbert_rejects_a_side_beyond_the_key_width(L):
+    buf = np.empty(1, np.int32)
+    assert L.spattn_hilbert_perm((1 << 21) + 1, 1, 1, buf.ctypes.data) == sp.ERR_UNSUPPORTED
+    assert b"2^21" in L.spattn_last_error()
+
+
+def test_binding_refuses_wrong_tensors_before_any_call(L):
+    """The binding checks dtype, contiguity, size and device of torch tensors
+    against the plan before the library sees a pointer (no CUDA needed: the
+    device check comes last, so host tensors reach every other check)."""
+    import torch
+    B, H, N, d, b = 1, 2, 256, 64, 64
+    h, ws = sp.spattn_plan(B, H, N, d, b, 0.9, 1, 4, 1)
+    x = torch.zeros(B * H * N * d, dtype=torch.bfloat16)
+    w = torch.zeros(ws, dtype=torch.uint8)
+    cases = [
+        ((x.float(), x, x, x, w), "dtype"),
+        ((x, x[:-1], x, x, w), "exactly"),
+        ((x, x, x.view(2, -1).t(), x, w), "contiguous"),
+        ((x, x, x, x, w[:-1]), "at least"),
+        ((x, x, x, x, w), "CUDA tensor"),
+    ]
+    for args, msg in cases:
+        with pytest.raises(ValueError, match=msg):
+            sp.spattn_forward(h, *args)
+    rp = torch.zeros(B * H * 4 + 1, dtype=torch.int32)
+    with pytest.raises(ValueError, match="col_idx"):
+        sp.spattn_route(h, x, x, x, w, rp, torch.zeros(B * H * 4 * 4 - 1, dtype=torch.int32))
+    with pytest.raises(ValueError, match="row_ptr"):
+        sp.spattn_route(h, x, x, x, w, rp[:-1], torch.zeros(B * H * 4 * 4, dtype=torch.int32))
+    with pytest.raises(ValueError, match="Kbar"):
+        sp.spattn_means(h, w, None, torch.zeros(B * H * 4 * d - 1), None)
+    with pytest.raises(ValueError, match="col_idx"):
+        sp.spattn_route_static(B, H, N, d, b, 0.9, 1, 4, x, x, rp,
+                               torch.zeros(B * H * 4 * 4 - 1, dtype=torch.int32))
+    sp.spattn_plan_destroy(h)
+    with pytest.raises(ValueError, match="unknown or destroyed"):
+        sp.spattn_forward(h, x, x, x, x, w)
