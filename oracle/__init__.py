@@ -19,6 +19,8 @@ plainly and slowly, in float64 from the exact bf16 inputs:
   (residual mode) one pseudo-key per dropped block that reuses the block's
   proxy score (Sol-Attn abstract: the skipped blocks are approximated from
   the scores the router already computed);
+* as an alternative selection, a fixed threshold on each block's proxy
+  probability (Sol-Attn abstract: on-the-fly block thresholding);
 * optional token reordering before blocking and its inverse after
   (DFSAttn abstract: Hilbert curve-based token reordering);
 * the probe-fitted residual correction (SparsePR page, section 2B): exact
@@ -36,7 +38,7 @@ brute-force enumeration or invariants; none is "parity unpinned".
 """
 from .spattn_ref import (  # noqa: F401
     decode_bf16, block_sizes, gather_tokens, scatter_tokens, block_means,
-    proxy_logits, block_softmax, route_rows, attend_block, attention,
+    proxy_logits, block_softmax, route_rows, route_threshold, attend_block, attention,
     forward, exact_block_logmass, attention_flops, MASS_MARGIN, TIE_MARGIN,
 )
 from .hilbert import hilbert_index, hilbert_perm  # noqa: F401

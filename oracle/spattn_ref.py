@@ -17,6 +17,11 @@ design notes):
 * tau >= 1 keeps every block (no prefix shorter than nb is needed, and
   rounding must not drop a block), tau <= 0 gives k* = 0;
 * the budget is k = min(max(k*, kmin), kmax, nb);
+* the on-the-fly block thresholding of the Sol-Attn abstract (a block is
+  critical when its proxy score passes a threshold; no proxy map is stored)
+  is read as a fixed threshold on the block probability, p_ij >= theta,
+  with the same clamp and the same order (p descending, ties to the lower
+  index) when a clamp binds (route_threshold);
 * the partial last query block is routed from its own mean over n_i tokens;
 * the pseudo-key of a dropped block j uses the per-token query q (not the
   block mean): logit q . Kbar_j / sqrt(d) + ln n_j, value Vbar_j;
@@ -185,6 +190,49 @@ def route_rows(p: np.ndarray, tau: float, kmin: int, kmax: int):
     return {"kept": kept, "k": ks, "marginal": marginal, "E": E_all}
 
 
+def route_threshold(p: np.ndarray, theta: float, kmin: int, kmax: int):
+    """Per-block probability threshold (Sol-Attn abstract: on-the-fly block
+    thresholding of the proxy scores, dynamic but controllable budgets).
+
+    Reading: block j of query row i is critical iff p_ij >= theta; the
+    budget is clamped to [kmin, min(kmax, nb)] by taking blocks in the same
+    order as the Top-p rule (p descending, ties to the lower index).  The
+    critical set is a prefix of that order, so no sort is needed unless a
+    clamp binds.  Returns the same dict as route_rows (E: exclusive prefix
+    mass at each block's rank); marginal blocks are those whose p lies
+    within a relative TIE_MARGIN of theta, plus, when a clamp set the cut,
+    the near-ties across the cut."""
+    nq, nb = p.shape
+    kept, ks, marginal = [], np.empty(nq, np.int64), []
+    E_all = np.empty_like(p)
+    idx = np.arange(nb)
+    kcap = min(kmax, nb)
+    for i in range(nq):
+        row = p[i]
+        crit = np.nonzero(row >= theta)[0]
+        kstar = len(crit)
+        order = np.lexsort((idx, -row))
+        sorted_p = row[order]
+        k = min(max(kstar, kmin), kcap)
+        ks[i] = k
+        kept.append(np.sort(order[:k]) if k != kstar else crit)
+        E = np.concatenate(([0.0], np.cumsum(sorted_p)[:-1]))
+        E_rank = np.empty(nb)
+        E_rank[order] = E
+        E_all[i] = E_rank
+        marg = set()
+        if k == kstar:
+            marg.update(np.nonzero(np.abs(row - theta) <= TIE_MARGIN * abs(theta))[0].tolist())
+        elif 0 < k < nb:
+            p_in, p_out = sorted_p[k - 1], sorted_p[k]
+            r_in = np.nonzero(sorted_p[:k] - p_out <= TIE_MARGIN * sorted_p[:k])[0]
+            r_out = k + np.nonzero(p_in - sorted_p[k:] <= TIE_MARGIN * p_in)[0]
+            marg.update(order[r_in].tolist())
+            marg.update(order[r_out].tolist())
+        marginal.append(np.array(sorted(marg), dtype=np.int64))
+    return {"kept": kept, "k": ks, "marginal": marginal, "E": E_all}
+
+
 # ------------------------------------------------------------- attention ---
 
 def attend_block(q: np.ndarray, Kp: np.ndarray, Vp: np.ndarray, kept: Sequence[int],
@@ -256,7 +304,7 @@ def attention_flops(kept_rows, n: np.ndarray, residual: bool, d: int) -> tuple:
 def forward(Q, K, V, b: int, tau: float, kmin: int, kmax: int, residual: int,
             perm: Optional[np.ndarray] = None, rows: Optional[dict] = None,
             kept_override: Optional[dict] = None, want_output: bool = True,
-            routing: str = "centroid"):
+            routing: str = "centroid", selection: str = "top_p"):
     """The whole path for bf16 inputs Q, K, V ([B, H, N, d] uint16 bits).
 
     rows:          optional {(b, h): array of token indices in the ORIGINAL
@@ -266,6 +314,9 @@ def forward(Q, K, V, b: int, tau: float, kmin: int, kmax: int, residual: int,
                    computed and returned).
     routing:       "centroid" (p from the block-mean proxy) or "pama" (p from
                    pama_importance of each query block's tokens).
+    selection:     "top_p" (route_rows, tau is the mass threshold) or
+                   "threshold" (route_threshold, tau is read as the per-block
+                   probability threshold theta).
     Returns a dict with Qbar/Kbar/Vbar (fp64 [B,H,nb,d]), route (per (b,h)
     route_rows results), and O: either [B,H,N,d] fp64 or {(b,h): [r, d]}.
     """
@@ -295,7 +346,12 @@ def forward(Q, K, V, b: int, tau: float, kmin: int, kmax: int, residual: int,
                               for s0, nj in zip(starts, n)])
             else:
                 p = block_softmax(proxy_logits(Qbar[bi, hi], Kbar[bi, hi], n))
-            r = route_rows(p, tau, kmin, kmax)
+            if selection == "threshold":
+                r = route_threshold(p, tau, kmin, kmax)
+            elif selection == "top_p":
+                r = route_rows(p, tau, kmin, kmax)
+            else:
+                raise ValueError(f"selection must be 'top_p' or 'threshold', got {selection!r}")
             r["p"] = p
             routes[(bi, hi)] = r
             if not want_output:

@@ -461,3 +461,90 @@ def test_forward_pama_routes_from_token_rows():
     a = R.forward(Q, K, V, w.b, 1.0, 1, w.nb, 1, routing="pama")["O"]
     c = R.forward(Q, K, V, w.b, 1.0, 1, w.nb, 1)["O"]
     assert np.allclose(a, c, atol=1e-12)
+
+
+# ------------------------------------------------- threshold selection (f3) --
+
+def test_threshold_hand_worked_row():
+    p = np.array([[0.4, 0.1, 0.3, 0.1, 0.1]])
+    cases = [  # (theta, kmin, kmax) -> kept
+        ((0.1, 1, 5), [0, 1, 2, 3, 4]),     # >= is inclusive
+        ((0.2, 1, 5), [0, 2]),
+        ((0.35, 1, 5), [0]),
+        ((0.5, 1, 5), [0]),                 # nothing passes: kmin
+        ((0.5, 2, 5), [0, 2]),
+        ((0.5, 3, 5), [0, 1, 2]),           # three-way tie at 0.1: the lowest index
+        ((0.2, 1, 1), [0]),                 # kmax binds
+        ((0.0, 1, 9), [0, 1, 2, 3, 4]),     # kmax > nb
+    ]
+    for (theta, kmin, kmax), want in cases:
+        r = R.route_threshold(p, theta, kmin, kmax)
+        assert r["kept"][0].tolist() == want, (theta, kmin, kmax)
+        assert r["k"][0] == len(want)
+
+
+def _dyadic_rows(rng, nq, nb, bits=20):
+    """Rows of distinct positive dyadic probabilities summing to exactly 1, so
+    that every partial sum is exact in fp64."""
+    rows = []
+    while len(rows) < nq:
+        w = rng.integers(1, 1 << 12, nb)
+        w[-1] = 0
+        w[-1] = (1 << bits) - w.sum()
+        if w[-1] > 0 and len(set(w.tolist())) == nb:
+            rows.append(w / float(1 << bits))
+    return np.array(rows)
+
+
+def test_threshold_set_is_the_top_p_set_of_its_own_mass():
+    """With no clamp binding, the critical set {p >= theta} is exactly what
+    the Top-p rule keeps for tau = the mass of that set (a second,
+    independent selection routine reaching the same blocks)."""
+    rng = np.random.default_rng(21)
+    p = _dyadic_rows(rng, 40, 24)
+    for theta in (0.01, 0.03, 0.05, 0.08):
+        thr = R.route_threshold(p, theta, 1, 24)
+        for i in range(len(p)):
+            crit = np.nonzero(p[i] >= theta)[0]
+            if len(crit) == 0 or len(crit) == 24:
+                continue
+            tau = float(p[i][crit].sum())
+            top = R.route_rows(p[i:i + 1], tau, 1, 24)
+            assert np.array_equal(thr["kept"][i], crit)
+            assert np.array_equal(top["kept"][0], crit), (theta, i)
+
+
+def test_threshold_clamped_budget_is_the_heaviest_subset():
+    """When a clamp binds, the kept set is the k-subset of largest mass
+    (brute force over all subsets; distinct p make it unique)."""
+    rng = np.random.default_rng(22)
+    p = _dyadic_rows(rng, 12, 8)
+    for theta, kmin, kmax in ((0.9, 3, 8), (0.0, 1, 4), (0.2, 5, 6), (0.01, 2, 2)):
+        r = R.route_threshold(p, theta, kmin, kmax)
+        for i in range(len(p)):
+            k = min(max(int(np.count_nonzero(p[i] >= theta)), kmin), kmax, 8)
+            best = max(itertools.combinations(range(8), k), key=lambda c: p[i][list(c)].sum())
+            assert r["kept"][i].tolist() == list(best)
+
+
+def test_threshold_sets_are_nested_in_theta():
+    rng = np.random.default_rng(23)
+    p = R.block_softmax(rng.standard_normal((30, 40)) * 2.0)
+    prev = None
+    for theta in (0.0, 0.005, 0.01, 0.02, 0.05, 0.1, 0.3, 1.1):
+        r = R.route_threshold(p, theta, 2, 30)
+        if prev is not None:
+            for a, b in zip(r["kept"], prev["kept"]):
+                assert set(a.tolist()) <= set(b.tolist())
+        prev = r
+    assert all(len(k) == 2 for k in prev["kept"])          # theta > 1: kmin
+
+
+def test_forward_threshold_zero_is_dense_and_rejects_unknown_selection():
+    w = get_config("tiny", H=1, grid=(1, 4, 64))
+    Q, K, V = make_qkv(w)
+    res = R.forward(Q, K, V, w.b, 0.0, 1, w.nb, 1, selection="threshold")
+    q, k, v = (R.decode_bf16(X[0, 0]) for X in (Q, K, V))
+    np.testing.assert_allclose(res["O"][0, 0], sdpa64(q, k, v), rtol=0, atol=1e-10)
+    with pytest.raises(ValueError):
+        R.forward(Q, K, V, w.b, 0.5, 1, w.nb, 1, selection="top_k")
