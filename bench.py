@@ -54,7 +54,7 @@ MEASURED_TRAFFIC = {
 }
 
 
-def measured_traffic(kernel, w):
+def measured_traffic(kernel, w, selection="top_p"):
     import hashlib
     ent = MEASURED_TRAFFIC[kernel]
     m = hashlib.sha256()
@@ -66,6 +66,8 @@ def measured_traffic(kernel, w):
         return None
     if m.hexdigest()[:16] != ent["sha"]:
         return None
+    if kernel == "attention" and selection != "top_p":
+        return None   # captured with Top-p selection: other kept sets, other traffic
     return ent["bytes"].get((w.name, w.H, round(w.tau, 6), int(w.residual)))
 
 
@@ -82,6 +84,11 @@ def parse_args(argv=None):
     ap.add_argument("--routing", choices=["centroid", "pama"], default="centroid",
                     help="block-importance estimate: block-mean centroids, or per-query "
                          "attention-mass aggregation (PAMA)")
+    ap.add_argument("--selection", choices=["top_p", "threshold"], default="top_p",
+                    help="Top-p on the cumulative mass (tau), or a per-block threshold on p "
+                         "(Sol-Attn on-the-fly thresholding; the knob is --theta)")
+    ap.add_argument("--theta", type=float, default=0.01,
+                    help="per-block probability threshold with --selection threshold")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the number of heads (smaller profiling captures)")
     ap.add_argument("--no-dense", action="store_true", help="skip the tau = 1 comparison run")
@@ -107,6 +114,10 @@ def workload_from_args(args, rank=0):
     ov = {}
     if args.tau is not None:
         ov["tau"] = args.tau
+    if args.selection == "threshold":
+        if args.tau is not None:
+            raise SystemExit("--selection threshold takes its knob from --theta, not --tau")
+        ov["tau"] = args.theta   # the plan's tau argument carries theta
     if args.residual is not None:
         ov["residual"] = args.residual
     if args.heads is not None:
@@ -251,7 +262,8 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
-def oracle_sample(w, seconds, Q=None, K=None, V=None, perm=None):
+def oracle_sample(w, seconds, Q=None, K=None, V=None, perm=None, routing="centroid",
+                  selection="top_p"):
     """Time the fp64 oracle on a bounded sample of the workload.
 
     Sample: head (0, 0) -- decode, gather, block means, proxy, routing of all
@@ -269,7 +281,13 @@ def oracle_sample(w, seconds, Q=None, K=None, V=None, perm=None):
     v = R.gather_tokens(R.decode_bf16(V[0, 0]), perm)
     n = R.block_sizes(w.N, w.b)
     Qb, Kb, Vb = R.block_means(q, w.b), R.block_means(k, w.b), R.block_means(v, w.b)
-    route = R.route_rows(R.block_softmax(R.proxy_logits(Qb, Kb, n)), w.tau, w.kmin, w.kmax)
+    if routing == "pama":
+        starts = np.concatenate([[0], np.cumsum(n)[:-1]])
+        p = np.stack([R.pama_importance(q[s0:s0 + nj], Kb, n) for s0, nj in zip(starts, n)])
+    else:
+        p = R.block_softmax(R.proxy_logits(Qb, Kb, n))
+    select = R.route_threshold if selection == "threshold" else R.route_rows
+    route = select(p, w.tau, w.kmin, w.kmax)
     flops = 0
     blocks = 0
     order = np.random.default_rng(0).permutation(len(n))
@@ -302,10 +320,10 @@ def run_reference(args):
         perm = oracle.hilbert_perm(w.grid)
     per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_sample(w, per_step, Q, K, V, perm)
+        oracle_sample(w, per_step, Q, K, V, perm, args.routing, args.selection)
     vals, times, desc = [], [], ""
     for _ in range(args.steps):
-        v, desc, dt = oracle_sample(w, per_step, Q, K, V, perm)
+        v, desc, dt = oracle_sample(w, per_step, Q, K, V, perm, args.routing, args.selection)
         vals.append(v)
         times.append(dt)
     value = float(np.mean(vals))
@@ -314,7 +332,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * float(np.mean(times)), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w, "cpu"),
+        "config": dict(config_of(w, "cpu"), routing=args.routing, selection=args.selection),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": "each step: " + desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -364,6 +382,8 @@ def run_ours(args):
     q, k, v = dev_bf16(Qh), dev_bf16(Kh), dev_bf16(Vh)
     o = torch.empty_like(q)
     routing = sp.ROUTING_PAMA if args.routing == "pama" else sp.ROUTING_CENTROID
+    if args.selection == "threshold":
+        routing |= sp.SELECT_THRESHOLD
     plan = sp.Plan(B, H, N, d, w.b, w.tau, w.kmin, w.kmax, w.residual, perm, device=dev,
                    routing=routing)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -509,7 +529,8 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        val, desc, _ = oracle_sample(w, args.cpu_seconds, perm=perm)
+        val, desc, _ = oracle_sample(w, args.cpu_seconds, perm=perm, routing=args.routing,
+                                     selection=args.selection)
         cpu = {"value": val, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                "sample": desc}
 
@@ -522,7 +543,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": dict(config_of(w, "flushed (256 MiB write between timed steps)"),
-                           routing=args.routing),
+                           routing=args.routing, selection=args.selection),
             "dense_equiv_tflops": dense_flops * world / (step_ms * 1e-3) / 1e12,
             "attn_tflops": attn_tflops,
             "pct_of_bf16_peak": 100.0 * attn_tflops / bf16_peak,
@@ -538,7 +559,7 @@ def run_ours(args):
             "roofline": {"bound": "tensor", "kernel": "attention", "achieved": attn_tflops,
                          "peak": bf16_peak, "unit": "TFLOP/s", "frac": attn_tflops / bf16_peak,
                          "peak_kind": f"{peak_kind} bf16 dense (burst)",
-                         "traffic": measured_traffic("attention", w), "traffic_unit": "bytes/launch"},
+                         "traffic": measured_traffic("attention", w, args.selection), "traffic_unit": "bytes/launch"},
             "roofline_route": {"bound": "alu", "kernel": "route + scan",
                                "achieved": route_flops / (max(route_ms - pool_ms, 1e-6) * 1e-3) / 1e12,
                                "peak": fp32_peak, "unit": "TFLOP/s",

@@ -23,6 +23,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: 
                 5: "TIMEOUT", 6: "DEVICE"}
 
 ROUTING_CENTROID, ROUTING_PAMA = 0, 1
+SELECT_THRESHOLD = 16   # OR into routing: tau is the per-block threshold theta on p
 
 EXPORTS = ("spattn_plan", "spattn_plan_ex", "spattn_plan_destroy", "spattn_plan_info", "spattn_pool",
            "spattn_route", "spattn_attend", "spattn_forward", "spattn_means", "spattn_check",
@@ -153,7 +154,8 @@ def spattn_plan(B, H, N, d, b, tau, kmin, kmax, residual, perm=None):
 
 
 def spattn_plan_ex(B, H, N, d, b, tau, kmin, kmax, residual, perm=None, routing=ROUTING_CENTROID):
-    """spattn_plan with a routing estimate (ROUTING_CENTROID or ROUTING_PAMA)."""
+    """spattn_plan with a routing estimate (ROUTING_CENTROID or ROUTING_PAMA),
+    optionally | SELECT_THRESHOLD (tau is then the per-block threshold)."""
     import numpy as np
     h = ctypes.c_void_p()
     ws = ctypes.c_size_t()

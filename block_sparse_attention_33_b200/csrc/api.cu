@@ -167,8 +167,9 @@ spattn_status_t spattn_plan_ex(spattn_plan_t* out, int B, int H, int N, int d, i
                                int routing, size_t* workspace_bytes) {
   g_err[0] = 0;
   if (!out) return fail(SPATTN_ERR_INVALID_ARG, "out is NULL");
-  if (routing != SPATTN_ROUTING_CENTROID && routing != SPATTN_ROUTING_PAMA)
-    return fail(SPATTN_ERR_INVALID_ARG, "routing must be SPATTN_ROUTING_CENTROID or SPATTN_ROUTING_PAMA (got %d)", routing);
+  const int estimate = routing & ~SPATTN_SELECT_THRESHOLD;
+  if (estimate != SPATTN_ROUTING_CENTROID && estimate != SPATTN_ROUTING_PAMA)
+    return fail(SPATTN_ERR_INVALID_ARG, "routing must be SPATTN_ROUTING_CENTROID or SPATTN_ROUTING_PAMA, optionally | SPATTN_SELECT_THRESHOLD (got %d)", routing);
   *out = nullptr;
   if (B < 1 || H < 1 || N < 1) return fail(SPATTN_ERR_INVALID_ARG, "need B, H, N >= 1 (got %d, %d, %d)", B, H, N);
   if (d != 64 && d != 128) return fail(SPATTN_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
@@ -198,7 +199,8 @@ spattn_status_t spattn_plan_ex(spattn_plan_t* out, int B, int H, int N, int d, i
   p.BH = B * H;
   p.tau = tau; p.kmin = kmin; p.kmax = kmax; p.residual = residual;
   p.perm = nullptr;
-  p.routing = routing == SPATTN_ROUTING_PAMA ? spattn::ROUTING_PAMA : spattn::ROUTING_CENTROID;
+  p.routing = estimate == SPATTN_ROUTING_PAMA ? spattn::ROUTING_PAMA : spattn::ROUTING_CENTROID;
+  p.threshold = (routing & SPATTN_SELECT_THRESHOLD) ? 1 : 0;
   {
     // tcgen05/TMEM kernel for 128-token blocks; the warp-MMA kernel serves
     // b = 64 and, with SPATTN_ATTN=mma in the environment when the plan is

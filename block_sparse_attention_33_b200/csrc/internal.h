@@ -19,6 +19,7 @@ struct Problem {
   int residual;
   int use_tc;           // attention on the tcgen05 kernel (else warp MMA)
   int routing;          // ROUTING_CENTROID or ROUTING_PAMA
+  int threshold;        // selection: 0 Top-p (tau = mass), 1 per-block p >= tau
   int test_stall;       // failure-path test: CTA 0 of the attention waits on a phase
                         // that never completes, so its bounded wait runs out
   const int32_t* perm;  // device, NULL if none

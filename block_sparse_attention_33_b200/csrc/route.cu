@@ -9,6 +9,10 @@
 // leaves shared memory.  pama_kernel computes p_i instead by per-query
 // attention-mass aggregation (PARK page 5.1) and shares the selection.
 //
+// With a threshold instead (Sol-Attn abstract: blocks are selected by comparing
+// their proxy scores with a threshold; read as p_ij >= theta), the cut is
+// bits(theta) - 1 and only a binding clamp needs the search below.
+//
 // Selection without a sort: with p >= 0 the float bit pattern orders p, and
 // the mass G(u) = sum of p_j whose bits exceed u is monotone in u.  The kept
 // prefix is {p_j > v} plus the first few blocks with p_j == v (ascending j),
@@ -44,7 +48,8 @@ struct RouteArgs {
   int32_t* counts;
   int32_t* lists;
   int nb, b, n_last, kcap, kmin;
-  float tau;
+  float tau;      // Top-p mass, or the per-block threshold theta
+  int threshold;  // 1: keep p_ij >= tau (Sol-Attn on-the-fly thresholding)
 };
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -140,7 +145,18 @@ __device__ void select_emit(const float* p, const RouteArgs& a, int row) {
   uint32_t thr = 0;
   int ties = 0, kstar = 0;
   bool by_mass = false;
-  if (a.tau >= 1.0f) {
+  if (a.threshold) {
+    // p >= theta: for theta > 0 the bits order p, so the critical set is
+    // {bits(p) > bits(theta) - 1}, a prefix of the (p desc, j asc) order;
+    // theta <= 0 keeps every block
+    if (a.tau <= 0.0f) {
+      kstar = a.nb;
+    } else {
+      thr = __float_as_uint(a.tau) - 1u;
+      kstar = count_above(p, a.nb, thr);
+      by_mass = true;  // the cut is set: the clamp search runs only if it binds
+    }
+  } else if (a.tau >= 1.0f) {
     kstar = a.nb;               // tau >= 1 keeps every block
   } else if (a.tau > 0.0f) {
     if (a.nb <= SEARCH32_MAX_NB) {
@@ -621,6 +637,7 @@ cudaError_t launch_route(const Problem& p, const Work& w, const void* Q, int32_t
   a.qbar = w.qbar; a.kbar = w.kbar; a.counts = w.counts; a.lists = w.lists;
   a.nb = p.nb; a.b = p.b; a.n_last = p.n_last; a.kcap = p.kcap; a.kmin = p.kmin;
   a.tau = p.tau;
+  a.threshold = p.threshold;
   cudaError_t e;
   if (p.routing == ROUTING_PAMA) {
     // tokens in blocked order: the pooling's permuted copy when there is

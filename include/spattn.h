@@ -93,10 +93,22 @@ enum {
                                   (two passes), on fp32 lanes                   */
 };
 
-/* spattn_plan with a choice of routing estimate (one of the values above;
- * anything else is SPATTN_ERR_INVALID_ARG).  spattn_plan is
+/* Selection flag, OR'ed into the routing argument of spattn_plan_ex.  With
+ * it, tau is read as a per-block probability threshold theta: block j of
+ * query block i is kept iff p_ij >= theta (theta <= 0 keeps every block),
+ * and the budget is clamped to [kmin, min(kmax, nb)] in the Top-p order
+ * (p descending, ties to the lower j) when a clamp binds.  This is the
+ * on-the-fly block thresholding of the Sol-Attn abstract (thelatestinai
+ * page), which gives no rule for the threshold: a fixed threshold on p is
+ * the reading taken here.  Dropped blocks take the residual pseudo-keys as
+ * before. */
+enum { SPATTN_SELECT_THRESHOLD = 16 };
+
+/* spattn_plan with a choice of routing estimate (one of the values above,
+ * optionally | SPATTN_SELECT_THRESHOLD; anything else is
+ * SPATTN_ERR_INVALID_ARG).  spattn_plan is
  * spattn_plan_ex(..., SPATTN_ROUTING_CENTROID, ...).  spattn_route_static
- * always uses the centroid estimate. */
+ * always uses the centroid estimate and the Top-p selection. */
 spattn_status_t spattn_plan_ex(spattn_plan_t* out, int B, int H, int N, int d, int b,
                                float tau, int kmin, int kmax, int residual,
                                const int32_t* perm_host, int routing, size_t* workspace_bytes);

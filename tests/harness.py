@@ -24,7 +24,7 @@ def from_dev(t) -> np.ndarray:
 
 def run_library(w, Q, K, V, perm=None, kept_csr=None, want_means=False, tau=None, routing=0):
     """Run route + attend through the C ABI; returns dict with O (fp64), CSR, means.
-    routing: 0 centroid estimate, 1 PAMA."""
+    routing: 0 centroid estimate, 1 PAMA, optionally | SELECT_THRESHOLD."""
     import torch
     import block_sparse_attention_33_b200 as sp
     tau = w.tau if tau is None else tau
@@ -113,7 +113,8 @@ def compare_outputs(got: np.ndarray, ref: np.ndarray):
     return max_abs, rel
 
 
-def oracle_check(w, Q, K, V, res, perm=None, rows=None, tau=None, routing="centroid"):
+def oracle_check(w, Q, K, V, res, perm=None, rows=None, tau=None, routing="centroid",
+                 selection="top_p"):
     """Oracle routing vs the library CSR, then oracle attention on the library's
     kept sets vs the library output.  Returns a dict of figures."""
     tau = w.tau if tau is None else tau
@@ -121,7 +122,7 @@ def oracle_check(w, Q, K, V, res, perm=None, rows=None, tau=None, routing="centr
     nb = res["nb"]
     gpu_kept = csr_to_kept(res["row_ptr"], res["col_idx"], B, H, nb)
     ref = R.forward(Q, K, V, w.b, tau, w.kmin, w.kmax, w.residual, perm=perm, rows=rows,
-                    kept_override=gpu_kept, routing=routing)
+                    kept_override=gpu_kept, routing=routing, selection=selection)
     bad, marg, nrows = compare_routing(ref["route"], gpu_kept)
     if rows is None:
         max_abs, rel = compare_outputs(res["O"], ref["O"])

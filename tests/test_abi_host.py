@@ -114,10 +114,14 @@ def test_hilbert_rejects_bad_grid(L):
 
 
 def test_plan_ex_routing_argument(L):
-    """spattn_plan_ex accepts the two routing estimates (no CUDA needed
-    without a permutation) and rejects anything else before any CUDA call."""
+    """spattn_plan_ex accepts the two routing estimates, each with or without
+    the threshold selection flag (no CUDA needed without a permutation), and
+    rejects anything else before any CUDA call."""
+    T = sp.SELECT_THRESHOLD
     for routing, code in ((sp.ROUTING_CENTROID, sp.OK), (sp.ROUTING_PAMA, sp.OK),
-                          (2, sp.ERR_INVALID_ARG), (-1, sp.ERR_INVALID_ARG)):
+                          (sp.ROUTING_CENTROID | T, sp.OK), (sp.ROUTING_PAMA | T, sp.OK),
+                          (2, sp.ERR_INVALID_ARG), (-1, sp.ERR_INVALID_ARG), (2 | T, sp.ERR_INVALID_ARG),
+                          (32, sp.ERR_INVALID_ARG)):
         h = ctypes.c_void_p()
         ws = ctypes.c_size_t()
         st = L.spattn_plan_ex(ctypes.byref(h), 1, 2, 1000, 64, 64, 0.9, 1, 8, 1, None, routing,
