@@ -172,3 +172,14 @@ def test_binding_refuses_wrong_tensors_before_any_call(L):
     sp.spattn_plan_destroy(h)
     with pytest.raises(ValueError, match="unknown or destroyed"):
         sp.spattn_forward(h, x, x, x, x, w)
+
+
+def test_plan_rejects_a_kept_list_capacity_beyond_int32(L):
+    """B*H*nb*min(kmax, nb) must fit the int32 CSR offsets: 600 heads of 2048
+    blocks keeping up to 2048 blocks each would need 2.5e9 entries."""
+    N = 2048 * 128
+    st, h, ws = plan_status(1, 600, N, 64, 128, 0.9, 1, 2048, 1)
+    assert st == sp.ERR_UNSUPPORTED and b"2^31" in L.spattn_last_error()
+    st, h, ws = plan_status(1, 600, N, 64, 128, 0.9, 1, 1024, 1)   # 1.26e9 entries: fits
+    assert st == sp.OK
+    assert L.spattn_plan_destroy(h) == sp.OK
