@@ -93,6 +93,9 @@ def parse_args(argv=None):
                     help="override the number of heads (smaller profiling captures)")
     ap.add_argument("--no-dense", action="store_true", help="skip the tau = 1 comparison run")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunk", type=int, default=0,
+                    help="also time spattn_forward_host (host tensors, copies overlapped over "
+                         "chunks of this many heads); 0: off")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="CPU time budget of the oracle baseline sample")
@@ -527,6 +530,22 @@ def run_ours(args):
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * tok_bytes,
                "d2h_bytes_per_step": tok_bytes}
 
+    e2e_pipe = None
+    if args.e2e_chunk > 0 and e2e is not None:
+        def pipe_step():
+            plan.forward_host(qh, kh, vh, oh, chunk_heads=args.e2e_chunk)
+
+        tpp = timed([pipe_step], max(3, args.steps // 3), 2)
+        pipe_ms = float(np.mean([x[0] for x in tpp]))
+        (pipe_ms,), _ = combine_over_ranks([pipe_ms], [], dev)
+        status = plan.check()
+        if status != sp.OK:
+            raise RuntimeError(f"device status {status}: {sp.spattn_last_error()}")
+        e2e_pipe = {"value": total_flops / (pipe_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": pipe_ms, "chunk_heads": args.e2e_chunk,
+                    "h2d_bytes_per_step": 3 * tok_bytes, "d2h_bytes_per_step": tok_bytes,
+                    "what": "spattn_forward_host: host tensors, copies overlapped with the path"}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         val, desc, _ = oracle_sample(w, args.cpu_seconds, perm=perm, routing=args.routing,
@@ -574,6 +593,7 @@ def run_ours(args):
             "clocks": clk,
             "launch": launch,
             "e2e": e2e,
+            "e2e_pipelined": e2e_pipe,
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "cpu_baseline": cpu,
         }

@@ -27,7 +27,8 @@ SELECT_THRESHOLD = 16   # OR into routing: tau is the per-block threshold theta 
 
 EXPORTS = ("spattn_plan", "spattn_plan_ex", "spattn_plan_destroy", "spattn_plan_info", "spattn_pool",
            "spattn_route", "spattn_attend", "spattn_forward", "spattn_means", "spattn_check",
-           "spattn_hilbert_perm", "spattn_route_static", "spattn_last_error")
+           "spattn_hilbert_perm", "spattn_route_static", "spattn_host_staging_bytes",
+           "spattn_forward_host", "spattn_last_error")
 
 
 class SpAttnError(RuntimeError):
@@ -66,6 +67,8 @@ def lib():
         "spattn_check": [P, P, P],
         "spattn_hilbert_perm": [I, I, I, P],
         "spattn_route_static": [I, I, I, I, I, F, I, I, P, P, P, P, P, P],
+        "spattn_host_staging_bytes": [P, I, SZP],
+        "spattn_forward_host": [P, P, P, P, P, P, P, I, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -103,6 +106,30 @@ def _devs(*specs):
             continue
         if not x.is_cuda:
             raise ValueError(f"{name}: must be a CUDA tensor")
+        out.append(x.data_ptr())
+    return out
+
+
+def _hosts(*specs):
+    """Pointers of host arguments, each spec (x, name, dtype, numel): a torch
+    CPU tensor of `dtype`, contiguous, with exactly `numel` elements (pinned
+    memory lets the library's copies run asynchronously); raw addresses pass
+    through."""
+    out = []
+    for x, name, dtype, numel in specs:
+        if isinstance(x, int):
+            out.append(x)
+            continue
+        if not hasattr(x, "data_ptr"):
+            raise TypeError(f"{name}: expected a torch CPU tensor or an address, got {type(x)}")
+        if x.is_cuda:
+            raise ValueError(f"{name}: must be a host (CPU) tensor")
+        if str(x.dtype) != "torch." + dtype:
+            raise ValueError(f"{name}: dtype must be torch.{dtype}, got {x.dtype}")
+        if not x.is_contiguous():
+            raise ValueError(f"{name}: must be contiguous")
+        if x.numel() != numel:
+            raise ValueError(f"{name}: needs exactly {numel} elements, has {x.numel()}")
         out.append(x.data_ptr())
     return out
 
@@ -206,6 +233,23 @@ def spattn_forward(plan, Q, K, V, O, workspace, stream=None):
     _check(lib().spattn_forward(plan, q, k, v, o, w, _stream(stream)))
 
 
+def spattn_host_staging_bytes(plan, chunk_heads) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().spattn_host_staging_bytes(plan, int(chunk_heads), ctypes.byref(n)))
+    return n.value
+
+
+def spattn_forward_host(plan, Q, K, V, O, workspace, staging, chunk_heads, stream=None):
+    """spattn_forward on host tensors, copies overlapped over chunks of
+    chunk_heads (batch, head) pairs; synchronise the stream before reading O."""
+    B, H, N, d = _shape(plan)[:4]
+    q, k, v, o = _hosts(*[(x, n, "bfloat16", B * H * N * d)
+                          for n, x in (("Q", Q), ("K", K), ("V", V), ("O", O))])
+    w, st = _devs(_workspace(plan, workspace),
+                  (staging, "staging", "uint8", spattn_host_staging_bytes(plan, chunk_heads), False))
+    _check(lib().spattn_forward_host(plan, q, k, v, o, w, st, int(chunk_heads), _stream(stream)))
+
+
 def spattn_means(plan, workspace, Qbar=None, Kbar=None, Vbar=None, stream=None):
     B, H, _, d, nb = _shape(plan)[:5]
     w, *bars = _devs(_workspace(plan, workspace),
@@ -257,6 +301,17 @@ class Plan:
 
     def forward(self, Q, K, V, O, stream=None):
         spattn_forward(self.handle, Q, K, V, O, self.workspace, stream)
+
+    def forward_host(self, Q, K, V, O, chunk_heads=None, stream=None):
+        """Forward on host tensors (pinned for overlap); the device staging
+        is allocated on first use.  Default chunk: a quarter of the heads."""
+        import torch
+        B, H = self.shape[:2]
+        c = chunk_heads or max(1, (B * H + 3) // 4)
+        need = spattn_host_staging_bytes(self.handle, c)
+        if getattr(self, "staging", None) is None or self.staging.numel() < need:
+            self.staging = torch.empty(need, dtype=torch.uint8, device=self.workspace.device)
+        spattn_forward_host(self.handle, Q, K, V, O, self.workspace, self.staging, c, stream)
 
     def route(self, Q, K, V, row_ptr=None, col_idx=None, stream=None):
         spattn_route(self.handle, Q, K, V, self.workspace, row_ptr, col_idx, stream)

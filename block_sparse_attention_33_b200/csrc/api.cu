@@ -102,6 +102,27 @@ Work bind(const Problem& p, const Layout& L, void* ws) {
   return w;
 }
 
+// Staging bytes of one tensor of a chunk of c (batch, head) pairs.
+size_t chunk_tensor_bytes(const Problem& p, int c) { return up((size_t)c * p.N * p.d * 2); }
+
+// The problem restricted to `c` consecutive (batch, head) pairs: heads are
+// independent through the whole path, so a chunk is a problem with B = 1,
+// H = c and the same token partition, knobs and permutation.
+Problem sub_problem(const Problem& p, int c) {
+  Problem q = p;
+  q.B = 1; q.H = c; q.BH = c;
+  return q;
+}
+
+// Keep the first device error: copy a chunk's error word into the plan's
+// word unless that already holds one.
+__global__ void merge_error_kernel(int32_t* dst, const int32_t* src) {
+  if (src[spattn::CTRL_ERROR] != 0 && dst[spattn::CTRL_ERROR] == 0) {
+    dst[spattn::CTRL_ERROR] = src[spattn::CTRL_ERROR];
+    dst[spattn::CTRL_ERROR_AUX] = src[spattn::CTRL_ERROR_AUX];
+  }
+}
+
 }  // namespace
 
 namespace spattn {
@@ -293,6 +314,106 @@ spattn_status_t spattn_forward(spattn_plan_t plan, const void* Q, const void* K,
                                void* O, void* workspace, void* stream) {
   if (spattn_status_t st = spattn_route(plan, Q, K, V, workspace, nullptr, nullptr, stream)) return st;
   return spattn_attend(plan, Q, K, V, nullptr, nullptr, O, workspace, stream);
+}
+
+spattn_status_t spattn_host_staging_bytes(spattn_plan_t plan, int chunk_heads, size_t* bytes) {
+  if (spattn_status_t st = check_plan(plan)) return st;
+  if (chunk_heads < 1) return fail(SPATTN_ERR_INVALID_ARG, "chunk_heads must be >= 1");
+  if (!bytes) return fail(SPATTN_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = 8 * chunk_tensor_bytes(plan->p, std::min(chunk_heads, plan->p.BH));
+  return SPATTN_OK;
+}
+
+spattn_status_t spattn_forward_host(spattn_plan_t plan, const void* Q_host, const void* K_host,
+                                    const void* V_host, void* O_host, void* workspace,
+                                    void* staging, int chunk_heads, void* stream) {
+  if (spattn_status_t st = check_plan(plan)) return st;
+  if (!Q_host || !K_host || !V_host || !O_host)
+    return fail(SPATTN_ERR_INVALID_ARG, "Q_host, K_host, V_host and O_host must be non-NULL");
+  if (chunk_heads < 1) return fail(SPATTN_ERR_INVALID_ARG, "chunk_heads must be >= 1");
+  if (!workspace) return fail(SPATTN_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(workspace) & (ALIGN - 1))
+    return fail(SPATTN_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (!staging) return fail(SPATTN_ERR_WORKSPACE, "staging is NULL");
+  if (reinterpret_cast<uintptr_t>(staging) & (ALIGN - 1))
+    return fail(SPATTN_ERR_WORKSPACE, "staging must be 256-byte aligned");
+  const Problem& p = plan->p;
+  const int c = std::min(chunk_heads, p.BH);
+  const int G = (p.BH + c - 1) / c;
+  const size_t tb = chunk_tensor_bytes(p, c);
+  const size_t head_bytes = (size_t)p.N * p.d * 2;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* ctrl = reinterpret_cast<int32_t*>(ws + plan->L.ctrl);
+  // a chunk's workspace starts at the base; unless the chunk is the whole
+  // problem (then it is the plan's own layout) it must end before the
+  // plan's control block, which collects the chunks' errors
+  if (c < p.BH && make_layout(sub_problem(p, c)).total > plan->L.ctrl)
+    return fail(SPATTN_ERR_WORKSPACE, "internal: chunk workspace overlaps the control block");
+  auto slot_buf = [&](int slot, int t) { return static_cast<uint8_t*>(staging) + (size_t)(slot * 4 + t) * tb; };
+  const uint8_t* src[3] = {static_cast<const uint8_t*>(Q_host), static_cast<const uint8_t*>(K_host),
+                           static_cast<const uint8_t*>(V_host)};
+  uint8_t* dst = static_cast<uint8_t*>(O_host);
+
+  cudaStream_t s0 = static_cast<cudaStream_t>(stream), s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_end = nullptr, ev_in[2] = {}, ev_done[2] = {}, ev_out[2] = {};
+  cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
+  cudaEvent_t* evs[8] = {&ev_start, &ev_end, &ev_in[0], &ev_in[1], &ev_done[0], &ev_done[1],
+                         &ev_out[0], &ev_out[1]};
+  for (int i = 0; i < 8 && e == cudaSuccess; ++i)
+    e = cudaEventCreateWithFlags(evs[i], cudaEventDisableTiming);
+  const char* what = "creating streams and events";
+  // the plan's error word starts clear; the copy streams start after the
+  // caller's earlier work on `stream` (which may still use the staging)
+  if (e == cudaSuccess) { what = "clearing the error word"; e = cudaMemsetAsync(ctrl, 0, 2 * sizeof(int32_t), s0); }
+  if (e == cudaSuccess) e = cudaEventRecord(ev_start, s0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_start, 0);
+  for (int g = 0; g < G && e == cudaSuccess; ++g) {
+    const int slot = g & 1, h0 = g * c, cg = std::min(c, p.BH - h0);
+    const size_t off = (size_t)h0 * head_bytes, bytes = (size_t)cg * head_bytes;
+    // inputs of chunk g, once chunk g - 2 is done with this slot
+    what = "copying a chunk in";
+    if (g >= 2) e = cudaStreamWaitEvent(s_in, ev_done[slot], 0);
+    for (int t = 0; t < 3 && e == cudaSuccess; ++t)
+      e = cudaMemcpyAsync(slot_buf(slot, t), src[t] + off, bytes, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in[slot], s_in);
+    // the path on chunk g, once its inputs are in and chunk g - 2's output is out
+    what = "ordering a chunk";
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s0, ev_in[slot], 0);
+    if (e == cudaSuccess && g >= 2) e = cudaStreamWaitEvent(s0, ev_out[slot], 0);
+    if (e != cudaSuccess) break;
+    const Problem ps = sub_problem(p, cg);
+    const Layout Ls = make_layout(ps);
+    const Work w = bind(ps, Ls, workspace);
+    const void *q = slot_buf(slot, 0), *k = slot_buf(slot, 1), *v = slot_buf(slot, 2);
+    void* o = slot_buf(slot, 3);
+    what = "pool kernel";
+    e = spattn::launch_pool(ps, q, k, v, w, s0);
+    if (e == cudaSuccess) { what = "route kernels"; e = spattn::launch_route(ps, w, q, nullptr, nullptr, !ps.use_tc, s0); }
+    if (e == cudaSuccess) { what = "attention kernel"; e = spattn::launch_attend(ps, q, k, v, w.row_ptr, w.col_idx, o, w, s0); }
+    if (e == cudaSuccess && w.ctrl != ctrl) {
+      what = "error merge";
+      merge_error_kernel<<<1, 1, 0, s0>>>(ctrl, w.ctrl);
+      e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(ev_done[slot], s0);
+    // output of chunk g
+    what = "copying a chunk out";
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_done[slot], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dst + off, o, bytes, cudaMemcpyDeviceToHost, s_out);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_out[slot], s_out);
+  }
+  // the caller's stream sees the last output copy
+  if (e == cudaSuccess) { what = "joining the streams"; e = cudaEventRecord(ev_end, s_out); }
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s0, ev_end, 0);
+  // resources are released once the enqueued work completes
+  for (int i = 0; i < 8; ++i)
+    if (*evs[i]) cudaEventDestroy(*evs[i]);
+  if (s_in) cudaStreamDestroy(s_in);
+  if (s_out) cudaStreamDestroy(s_out);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return SPATTN_OK;
 }
 
 spattn_status_t spattn_means(spattn_plan_t plan, const void* workspace, float* Qbar, float* Kbar,

@@ -173,6 +173,36 @@ spattn_status_t spattn_attend(spattn_plan_t plan, const void* Q, const void* K, 
 spattn_status_t spattn_forward(spattn_plan_t plan, const void* Q, const void* K, const void* V,
                                void* O, void* workspace, void* stream);
 
+/* Device staging bytes spattn_forward_host needs for chunks of chunk_heads
+ * (batch, head) pairs (chunk_heads >= 1; values above B*H count as B*H):
+ * two slots of the chunk's Q, K, V and O. */
+spattn_status_t spattn_host_staging_bytes(spattn_plan_t plan, int chunk_heads, size_t* bytes);
+
+/* spattn_forward on HOST-resident tensors, with the transfers overlapped.
+ * The pages say nothing on this; it exists because heads are independent
+ * through the whole path, so the copy of one chunk of heads in, the path on
+ * the previous chunk and the copy of the chunk before it out can run at
+ * once instead of one after the other.
+ *   Q_host, K_host, V_host  bf16 [B, H, N, d] host memory (pinned memory
+ *                           lets the copies run asynchronously; pageable
+ *                           memory works but the copies then block);
+ *   O_host                  bf16 [B, H, N, d] host memory, written;
+ *   workspace               as for spattn_forward (workspace_bytes);
+ *   staging                 device, spattn_host_staging_bytes(plan,
+ *                           chunk_heads) bytes, 256-byte aligned;
+ *   chunk_heads             (batch, head) pairs per chunk, >= 1.
+ * Chunk g (heads g*c .. g*c+c-1 in (batch, head) order) is copied into one of
+ * two staging slots on a copy stream, run through pool, route and attend on
+ * `stream`, and copied out on a second copy stream; slots are reused two
+ * chunks later.  The output equals spattn_forward's bit for bit.  The call
+ * returns after enqueueing; synchronise `stream` before reading O_host or
+ * reusing the input buffers.  spattn_check reports the first device error
+ * of any chunk.  The host buffers must stay valid until then; on an error
+ * status, synchronise the device before reusing any of the buffers. */
+spattn_status_t spattn_forward_host(spattn_plan_t plan, const void* Q_host, const void* K_host,
+                                    const void* V_host, void* O_host, void* workspace,
+                                    void* staging, int chunk_heads, void* stream);
+
 /* Copy the fp32 block means [B, H, nb, d] left in the workspace by the last
  * pool/route into caller device buffers (any may be NULL). */
 spattn_status_t spattn_means(spattn_plan_t plan, const void* workspace, float* Qbar,

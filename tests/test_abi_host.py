@@ -183,3 +183,43 @@ def test_plan_rejects_a_kept_list_capacity_beyond_int32(L):
     st, h, ws = plan_status(1, 600, N, 64, 128, 0.9, 1, 1024, 1)   # 1.26e9 entries: fits
     assert st == sp.OK
     assert L.spattn_plan_destroy(h) == sp.OK
+
+
+def test_host_forward_staging_size_and_argument_checks(L):
+    """spattn_host_staging_bytes: two slots of four tensors of the chunk,
+    each rounded up to 256 bytes; spattn_forward_host refuses NULL and
+    misaligned arguments before any CUDA call."""
+    B, H, N, d = 1, 5, 1000, 64
+    st, h, ws = plan_status(B, H, N, d, 64, 0.9, 1, 4, 1)
+    assert st == sp.OK
+    up = lambda x: (x + 255) // 256 * 256
+    n = ctypes.c_size_t()
+    for c, eff in ((1, 1), (2, 2), (5, 5), (9, 5)):
+        assert L.spattn_host_staging_bytes(h, c, ctypes.byref(n)) == sp.OK
+        assert n.value == 8 * up(eff * N * d * 2)
+    assert L.spattn_host_staging_bytes(h, 0, ctypes.byref(n)) == sp.ERR_INVALID_ARG
+    f = L.spattn_forward_host
+    assert f(h, None, 16, 16, 16, 256, 256, 2, None) == sp.ERR_INVALID_ARG
+    assert f(h, 16, 16, 16, 16, 256, 256, 0, None) == sp.ERR_INVALID_ARG
+    assert f(h, 16, 16, 16, 16, None, 256, 2, None) == sp.ERR_WORKSPACE
+    assert f(h, 16, 16, 16, 16, 256, None, 2, None) == sp.ERR_WORKSPACE
+    assert f(h, 16, 16, 16, 16, 256, 272, 2, None) == sp.ERR_WORKSPACE   # misaligned staging
+    assert L.spattn_plan_destroy(h) == sp.OK
+
+
+def test_binding_checks_host_tensors_of_the_host_forward(L):
+    import torch
+    B, H, N, d = 1, 2, 256, 64
+    h, ws = sp.spattn_plan(B, H, N, d, 64, 0.9, 1, 4, 1)
+    x = torch.zeros(B * H * N * d, dtype=torch.bfloat16)
+    w = torch.zeros(ws, dtype=torch.uint8)
+    stg = torch.zeros(sp.spattn_host_staging_bytes(h, 1), dtype=torch.uint8)
+    for args, msg in (((x.float(), x, x, x), "dtype"), ((x, x, x, x[:-1]), "exactly"),
+                      ((x, x.view(2, -1).t(), x, x), "contiguous")):
+        with pytest.raises(ValueError, match=msg):
+            sp.spattn_forward_host(h, *args, w, stg, 1)
+    with pytest.raises(ValueError, match="staging"):
+        sp.spattn_forward_host(h, x, x, x, x, torch.zeros(ws, dtype=torch.uint8), stg[:-1], 1)
+    with pytest.raises(ValueError, match="CUDA tensor"):       # host tensors pass; the workspace must be on the device
+        sp.spattn_forward_host(h, x, x, x, x, w, stg, 1)
+    sp.spattn_plan_destroy(h)
