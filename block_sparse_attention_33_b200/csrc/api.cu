@@ -114,6 +114,16 @@ Problem sub_problem(const Problem& p, int c) {
   return q;
 }
 
+// Heads per chunk of spattn_forward_host.  A chunk's workspace starts at the
+// base and must end before the plan's control block, which collects the
+// chunks' errors; when rounding makes a smaller chunk reach it (tiny
+// problems), the whole problem is one chunk and uses the plan's own layout.
+int effective_chunk(const Problem& p, const Layout& L, int chunk_heads) {
+  const int c = std::min(chunk_heads, p.BH);
+  if (c < p.BH && make_layout(sub_problem(p, c)).total > L.ctrl) return p.BH;
+  return c;
+}
+
 // Keep the first device error: copy a chunk's error word into the plan's
 // word unless that already holds one.
 __global__ void merge_error_kernel(int32_t* dst, const int32_t* src) {
@@ -320,7 +330,7 @@ spattn_status_t spattn_host_staging_bytes(spattn_plan_t plan, int chunk_heads, s
   if (spattn_status_t st = check_plan(plan)) return st;
   if (chunk_heads < 1) return fail(SPATTN_ERR_INVALID_ARG, "chunk_heads must be >= 1");
   if (!bytes) return fail(SPATTN_ERR_INVALID_ARG, "bytes is NULL");
-  *bytes = 8 * chunk_tensor_bytes(plan->p, std::min(chunk_heads, plan->p.BH));
+  *bytes = 8 * chunk_tensor_bytes(plan->p, effective_chunk(plan->p, plan->L, chunk_heads));
   return SPATTN_OK;
 }
 
@@ -338,17 +348,12 @@ spattn_status_t spattn_forward_host(spattn_plan_t plan, const void* Q_host, cons
   if (reinterpret_cast<uintptr_t>(staging) & (ALIGN - 1))
     return fail(SPATTN_ERR_WORKSPACE, "staging must be 256-byte aligned");
   const Problem& p = plan->p;
-  const int c = std::min(chunk_heads, p.BH);
+  const int c = effective_chunk(p, plan->L, chunk_heads);
   const int G = (p.BH + c - 1) / c;
   const size_t tb = chunk_tensor_bytes(p, c);
   const size_t head_bytes = (size_t)p.N * p.d * 2;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* ctrl = reinterpret_cast<int32_t*>(ws + plan->L.ctrl);
-  // a chunk's workspace starts at the base; unless the chunk is the whole
-  // problem (then it is the plan's own layout) it must end before the
-  // plan's control block, which collects the chunks' errors
-  if (c < p.BH && make_layout(sub_problem(p, c)).total > plan->L.ctrl)
-    return fail(SPATTN_ERR_WORKSPACE, "internal: chunk workspace overlaps the control block");
   auto slot_buf = [&](int slot, int t) { return static_cast<uint8_t*>(staging) + (size_t)(slot * 4 + t) * tb; };
   const uint8_t* src[3] = {static_cast<const uint8_t*>(Q_host), static_cast<const uint8_t*>(K_host),
                            static_cast<const uint8_t*>(V_host)};

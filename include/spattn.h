@@ -174,8 +174,10 @@ spattn_status_t spattn_forward(spattn_plan_t plan, const void* Q, const void* K,
                                void* O, void* workspace, void* stream);
 
 /* Device staging bytes spattn_forward_host needs for chunks of chunk_heads
- * (batch, head) pairs (chunk_heads >= 1; values above B*H count as B*H):
- * two slots of the chunk's Q, K, V and O. */
+ * (batch, head) pairs (chunk_heads >= 1; values above B*H count as B*H, and
+ * so does any chunk too large for the workspace to hold a chunk's scratch
+ * beside the plan's error word, which only happens on tiny problems): two
+ * slots of the chunk's Q, K, V and O. */
 spattn_status_t spattn_host_staging_bytes(spattn_plan_t plan, int chunk_heads, size_t* bytes);
 
 /* spattn_forward on HOST-resident tensors, with the transfers overlapped.
