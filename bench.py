@@ -89,6 +89,8 @@ def parse_args(argv=None):
                          "(Sol-Attn on-the-fly thresholding; the knob is --theta)")
     ap.add_argument("--theta", type=float, default=0.01,
                     help="per-block probability threshold with --selection threshold")
+    ap.add_argument("--no-threshold", action="store_true",
+                    help="skip the extra timing of threshold selection at --theta")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the number of heads (smaller profiling captures)")
     ap.add_argument("--no-dense", action="store_true", help="skip the tau = 1 comparison run")
@@ -530,6 +532,39 @@ def run_ours(args):
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * tok_bytes,
                "d2h_bytes_per_step": tok_bytes}
 
+    # threshold selection (p >= theta, Sol-Attn on-the-fly thresholding) on the
+    # same inputs: a second plan, timed like the main step; one rank only
+    thresh = None
+    if world == 1 and args.selection == "top_p" and not args.no_threshold:
+        try:
+            tplan = sp.Plan(B, H, N, d, w.b, args.theta, w.kmin, w.kmax, w.residual, perm,
+                            device=dev, routing=routing | sp.SELECT_THRESHOLD)
+            trp = torch.zeros(B * H * tplan.nb + 1, dtype=torch.int32, device=dev)
+            tci = torch.zeros(max(tplan.col_capacity, 1), dtype=torch.int32, device=dev)
+            tplan.route(q, k, v, trp, tci)
+            torch.cuda.synchronize(dev)
+            t_rp, t_ci = trp.cpu().numpy(), tci.cpu().numpy()
+            t_exact, t_resid = attention_flops(t_rp, t_ci, w, tplan.nb)
+            n_graphs = len(graphs)
+            tt = timed([as_graph(lambda: tplan.route(q, k, v)),
+                        as_graph(lambda: tplan.attend(q, k, v, o))], max(3, args.steps // 3), 2)
+            t_route = float(np.mean([x[0] for x in tt]))
+            t_attend = float(np.mean([x[1] for x in tt]))
+            status = tplan.check()
+            del graphs[n_graphs:]      # release its graphs before its plan
+            tplan.close()
+            if status != sp.OK:
+                raise RuntimeError(f"device status {status}: {sp.spattn_last_error()}")
+            thresh = {"theta": args.theta,
+                      "kept_fraction": float(np.diff(t_rp).sum()) / (B * H * tplan.nb * tplan.nb),
+                      "ms_per_step": t_route + t_attend, "route_ms": t_route, "attend_ms": t_attend,
+                      "value": (t_exact + t_resid) / ((t_route + t_attend) * 1e-3) / 1e12,
+                      "attn_tflops": (t_exact + t_resid) / (t_attend * 1e-3) / 1e12,
+                      "unit": "TFLOP/s",
+                      "what": "per-block threshold p >= theta in the route kernel, same attention"}
+        except Exception as ex:   # reported in the line; the measurements above stand
+            thresh = {"error": f"{type(ex).__name__}: {ex}"[:300], "theta": args.theta}
+
     e2e_pipe = None
     chunk = args.e2e_chunk if args.e2e_chunk >= 0 else max(1, (B * H + 3) // 4)
     # one rank only: an error on one rank must not leave the others in a collective
@@ -562,8 +597,8 @@ def run_ours(args):
         graphs.clear()
         plan.close()
     except Exception:
-        if not (e2e_pipe and "error" in e2e_pipe):
-            raise   # the failure already recorded in the line may also fail the clean-up
+        if not any(x and "error" in x for x in (e2e_pipe, thresh)):
+            raise   # a failure already recorded in the line may also fail the clean-up
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -603,6 +638,7 @@ def run_ours(args):
             "launch": launch,
             "e2e": e2e,
             "e2e_pipelined": e2e_pipe,
+            "threshold_selection": thresh,
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "cpu_baseline": cpu,
         }
