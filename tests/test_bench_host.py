@@ -63,3 +63,40 @@ def test_attention_recall_extremes_and_a_hand_case():
     rp = np.array([0, 1, 2]); ci = np.array([0, 0])
     r = bench.attention_recall(q, k, rp, ci, b, 2, rows_per_head=4)
     assert abs(r - 0.75) < 1e-6
+
+
+@pytest.mark.parametrize("extra", [[], ["--selection", "threshold", "--theta", "0.05"], ["--routing", "pama"]])
+def test_reference_arm_prints_one_contract_line(extra):
+    """`bench.py --impl reference` (the oracle on the host cores) prints one
+    JSON line with the keys the benchmark contract names, on the tiny
+    workload with a short sample."""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "3", *extra],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e", "impl"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["steps"] == 1 and line["warmup"] == 3
+    assert line["value"] > 0 and line["higher_is_better"] is True
+    assert line["config"]["workload"] == "tiny"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    if extra:
+        assert line["config"][extra[0].lstrip("-")] == extra[1]
+
+
+def test_warmup_below_three_is_refused():
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "2"],
+                       capture_output=True, text=True, timeout=120, cwd=ROOT)
+    assert r.returncode != 0 and "warmup" in (r.stderr + r.stdout)
