@@ -89,6 +89,8 @@ def parse_args(argv=None):
                          "(Sol-Attn on-the-fly thresholding; the knob is --theta)")
     ap.add_argument("--theta", type=float, default=0.01,
                     help="per-block probability threshold with --selection threshold")
+    ap.add_argument("--no-probe", action="store_true",
+                    help="skip the extra timing of the probe-fitted residual correction")
     ap.add_argument("--no-threshold", action="store_true",
                     help="skip the extra timing of threshold selection at --theta")
     ap.add_argument("--heads", type=int, default=None,
@@ -565,6 +567,35 @@ def run_ours(args):
         except Exception as ex:   # reported in the line; the measurements above stand
             thresh = {"error": f"{type(ex).__name__}: {ex}"[:300], "theta": args.theta}
 
+    # probe-fitted residual correction (SparsePR) of the routed output: enough
+    # probe rows per block for at least 2 (d + 1) rows per head; one rank only
+    probe = None
+    if world == 1 and not args.no_probe:
+        try:
+            from workloads import probe_rows
+            per_block = max(1, -(-2 * (d + 1) // plan.nb))
+            pr = np.stack([np.stack([probe_rows(N, w.b, (w.seed, 7, bi, hi), per_block)
+                                     for hi in range(H)]) for bi in range(B)]).astype(np.int32)
+            M = int(pr.shape[-1])
+            pr_dev = torch.from_numpy(pr).to(dev)
+            p_lam, p_r = 100.0, 16
+            plan.forward(q, k, v, o)
+            n_graphs = len(graphs)
+            tpc = timed([as_graph(lambda: plan.probe_correct(q, k, v, o, pr_dev, p_lam, p_r))],
+                        max(3, args.steps // 3), 2)
+            p_ms = float(np.mean([x[0] for x in tpc]))
+            del graphs[n_graphs:]
+            status = plan.check()
+            if status != sp.OK:
+                raise RuntimeError(f"device status {status}: {sp.spattn_last_error()}")
+            probe = {"ms": p_ms, "share_of_step": p_ms / step_ms, "M": M, "per_block": per_block,
+                     "lam": p_lam, "r": p_r,
+                     "dense_row_flops": 4.0 * B * H * M * N * d,
+                     "what": "probe-fitted residual correction: exact probe rows, ridge fit, "
+                             "Jacobi subspace, O += O (B P) + b P"}
+        except Exception as ex:   # reported in the line; the measurements above stand
+            probe = {"error": f"{type(ex).__name__}: {ex}"[:300]}
+
     e2e_pipe = None
     chunk = args.e2e_chunk if args.e2e_chunk >= 0 else max(1, (B * H + 3) // 4)
     # one rank only: an error on one rank must not leave the others in a collective
@@ -597,7 +628,7 @@ def run_ours(args):
         graphs.clear()
         plan.close()
     except Exception:
-        if not any(x and "error" in x for x in (e2e_pipe, thresh)):
+        if not any(x and "error" in x for x in (e2e_pipe, thresh, probe)):
             raise   # a failure already recorded in the line may also fail the clean-up
     if rank == 0:
         line = {
@@ -639,6 +670,7 @@ def run_ours(args):
             "e2e": e2e,
             "e2e_pipelined": e2e_pipe,
             "threshold_selection": thresh,
+            "probe_correction": probe,
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "cpu_baseline": cpu,
         }

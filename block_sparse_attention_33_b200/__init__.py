@@ -28,7 +28,8 @@ SELECT_THRESHOLD = 16   # OR into routing: tau is the per-block threshold theta 
 EXPORTS = ("spattn_plan", "spattn_plan_ex", "spattn_plan_destroy", "spattn_plan_info", "spattn_pool",
            "spattn_route", "spattn_attend", "spattn_forward", "spattn_means", "spattn_check",
            "spattn_hilbert_perm", "spattn_route_static", "spattn_host_staging_bytes",
-           "spattn_forward_host", "spattn_last_error")
+           "spattn_forward_host", "spattn_probe_scratch_bytes", "spattn_probe_correct",
+           "spattn_last_error")
 
 
 class SpAttnError(RuntimeError):
@@ -69,6 +70,8 @@ def lib():
         "spattn_route_static": [I, I, I, I, I, F, I, I, P, P, P, P, P, P],
         "spattn_host_staging_bytes": [P, I, SZP],
         "spattn_forward_host": [P, P, P, P, P, P, P, I, P],
+        "spattn_probe_scratch_bytes": [P, I, SZP],
+        "spattn_probe_correct": [P, P, P, P, P, P, I, F, I, P, P, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -250,6 +253,25 @@ def spattn_forward_host(plan, Q, K, V, O, workspace, staging, chunk_heads, strea
     _check(lib().spattn_forward_host(plan, q, k, v, o, w, st, int(chunk_heads), _stream(stream)))
 
 
+def spattn_probe_scratch_bytes(plan, M) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().spattn_probe_scratch_bytes(plan, int(M), ctypes.byref(n)))
+    return n.value
+
+
+def spattn_probe_correct(plan, Q, K, V, O, probes, M, lam, r, workspace, scratch, stream=None):
+    """Probe-fitted residual correction of the routed output O, in place.
+    probes: int32 device tensor [B, H, M] of token indices."""
+    B, H = _shape(plan)[:2]
+    q, k, v, o, pr, w, st = _devs(*_tokens(plan, Q=Q, K=K, V=V, O=O),
+                                  (probes, "probes", "int32", B * H * int(M), True),
+                                  _workspace(plan, workspace),
+                                  (scratch, "scratch", "uint8", spattn_probe_scratch_bytes(plan, M),
+                                   False))
+    _check(lib().spattn_probe_correct(plan, q, k, v, o, pr, int(M), float(lam), int(r), w, st,
+                                      _stream(stream)))
+
+
 def spattn_means(plan, workspace, Qbar=None, Kbar=None, Vbar=None, stream=None):
     B, H, _, d, nb = _shape(plan)[:5]
     w, *bars = _devs(_workspace(plan, workspace),
@@ -301,6 +323,17 @@ class Plan:
 
     def forward(self, Q, K, V, O, stream=None):
         spattn_forward(self.handle, Q, K, V, O, self.workspace, stream)
+
+    def probe_correct(self, Q, K, V, O, probes, lam, r, stream=None):
+        """Probe-fitted residual correction of O (the output of forward on the
+        same inputs), in place.  probes: int32 device tensor [B, H, M]."""
+        import torch
+        M = probes.shape[-1]
+        need = spattn_probe_scratch_bytes(self.handle, M)
+        if getattr(self, "probe_scratch", None) is None or self.probe_scratch.numel() < need:
+            self.probe_scratch = torch.empty(need, dtype=torch.uint8, device=self.workspace.device)
+        spattn_probe_correct(self.handle, Q, K, V, O, probes, M, lam, r, self.workspace,
+                             self.probe_scratch, stream)
 
     def forward_host(self, Q, K, V, O, chunk_heads=None, stream=None):
         """Forward on host tensors (pinned for overlap); the device staging

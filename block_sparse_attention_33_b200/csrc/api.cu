@@ -421,6 +421,37 @@ spattn_status_t spattn_forward_host(spattn_plan_t plan, const void* Q_host, cons
   return SPATTN_OK;
 }
 
+spattn_status_t spattn_probe_scratch_bytes(spattn_plan_t plan, int M, size_t* bytes) {
+  if (spattn_status_t st = check_plan(plan)) return st;
+  if (M < 1) return fail(SPATTN_ERR_INVALID_ARG, "need M >= 1 probe rows (got %d)", M);
+  if (!bytes) return fail(SPATTN_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = spattn::probe_scratch_bytes(plan->p, M);
+  return SPATTN_OK;
+}
+
+spattn_status_t spattn_probe_correct(spattn_plan_t plan, const void* Q, const void* K,
+                                     const void* V, void* O, const int32_t* probes, int M,
+                                     float lam, int r, void* workspace, void* scratch,
+                                     void* stream) {
+  if (spattn_status_t st = check_inputs(plan, Q, K, V, workspace)) return st;
+  const Problem& p = plan->p;
+  if (!O || (reinterpret_cast<uintptr_t>(O) & 15))
+    return fail(SPATTN_ERR_INVALID_ARG, "O must be non-NULL and 16-byte aligned");
+  if (!probes) return fail(SPATTN_ERR_INVALID_ARG, "probes is NULL");
+  if (M < 1 || (long long)M * p.BH > (1LL << 30))
+    return fail(SPATTN_ERR_INVALID_ARG, "need 1 <= M and B*H*M <= 2^30 (got M = %d)", M);
+  if (!isfinite(lam) || lam < 0.f) return fail(SPATTN_ERR_INVALID_ARG, "lam must be finite and >= 0");
+  if (r < 0 || r > p.d) return fail(SPATTN_ERR_INVALID_ARG, "need 0 <= r <= d (got %d)", r);
+  if (p.BH > 65535) return fail(SPATTN_ERR_UNSUPPORTED, "the probe correction takes B*H <= 65535");
+  if (!scratch || (reinterpret_cast<uintptr_t>(scratch) & (ALIGN - 1)))
+    return fail(SPATTN_ERR_WORKSPACE, "scratch must be non-NULL and 256-byte aligned");
+  const Work w = bind(p, plan->L, workspace);
+  cudaError_t e = spattn::launch_probe_correct(p, Q, K, V, O, probes, M, lam, r, scratch, w.ctrl,
+                                               static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "probe correction kernels");
+  return SPATTN_OK;
+}
+
 spattn_status_t spattn_means(spattn_plan_t plan, const void* workspace, float* Qbar, float* Kbar,
                              float* Vbar, void* stream) {
   if (spattn_status_t st = check_plan(plan)) return st;
@@ -451,9 +482,13 @@ spattn_status_t spattn_check(spattn_plan_t plan, void* workspace, void* stream) 
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
   if (h[0] == spattn::DEV_BAD_INDEX)
-    return fail(SPATTN_ERR_DEVICE, "a CSR block index outside [0, nb) was skipped (work item %d)", h[1]);
+    return fail(SPATTN_ERR_DEVICE, "an index outside its range was skipped: a CSR block index "
+                "(work item %d) or a probe token (entry %d of probes)", h[1], h[1]);
   if (h[0] == spattn::DEV_TIMEOUT)
     return fail(SPATTN_ERR_TIMEOUT, "a device-side wait gave up (site %d)", h[1]);
+  if (h[0] == spattn::DEV_NUMERIC)
+    return fail(SPATTN_ERR_DEVICE, "the probe fit's normal equations were not positive definite "
+                "(head %d left uncorrected)", h[1]);
   if (h[0] != 0) return fail(SPATTN_ERR_DEVICE, "device error code %d (aux %d)", h[0], h[1]);
   return SPATTN_OK;
 }

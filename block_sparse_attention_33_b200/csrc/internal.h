@@ -50,6 +50,13 @@ cudaError_t launch_attend(const Problem& p, const void* Q, const void* K, const 
                           const int32_t* row_ptr, const int32_t* col_idx, void* O,
                           const Work& w, cudaStream_t s);
 
+// Probe-fitted residual correction (SparsePR page, section 2B) of the routed
+// output O in place; scratch of probe_scratch_bytes(p, M) bytes.
+size_t probe_scratch_bytes(const Problem& p, int M);
+cudaError_t launch_probe_correct(const Problem& p, const void* Q, const void* K, const void* V,
+                                 void* O, const int32_t* probes, int M, float lam, int r,
+                                 void* scratch, int32_t* ctrl, cudaStream_t s);
+
 // Raise kernel `fn`'s dynamic shared-memory limit on the current device to at
 // least `bytes`; the attribute call is made only when a launch needs more
 // than was granted before (thread-safe).

@@ -205,6 +205,42 @@ spattn_status_t spattn_forward_host(spattn_plan_t plan, const void* Q_host, cons
                                     const void* V_host, void* O_host, void* workspace,
                                     void* staging, int chunk_heads, void* stream);
 
+/* Device scratch bytes spattn_probe_correct needs for M probe rows per
+ * (batch, head) pair. */
+spattn_status_t spattn_probe_scratch_bytes(spattn_plan_t plan, int M, size_t* bytes);
+
+/* Probe-fitted residual correction of a routed output, in place (SparsePR
+ * page, section 2B: a few query rows are evaluated exactly, the residual
+ * R = O_dense - O_sparse of those rows is fitted as an affine function
+ * b + x B of the sparse output by ridge regression, the fitted correction is
+ * restricted to the span of the r leading right singular vectors of R, and
+ * it is added to every row; probe rows take their exact output).  Per
+ * (batch, head) pair:
+ *   Q, K, V   bf16 [B, H, N, d] device, original token order (the inputs of
+ *             the spattn_forward that produced O);
+ *   O         bf16 [B, H, N, d] device: in, the routed output; out, the
+ *             corrected output;
+ *   probes    int32 [B, H, M] device token indices in [0, N) (the page
+ *             stratifies them across query groups; the caller chooses them).
+ *             An index outside [0, N) is skipped and flagged (spattn_check:
+ *             SPATTN_ERR_DEVICE);
+ *   lam       ridge penalty on B (>= 0; the bias b is not penalised);
+ *   r         0 <= r <= d: rank of the residual subspace (0: no correction
+ *             off the probes; d: the whole output space);
+ *   workspace the plan's workspace (its device error word only);
+ *   scratch   device, spattn_probe_scratch_bytes(plan, M) bytes, 256-byte
+ *             aligned.
+ * Everything is fp32 on the device: the exact probe rows, the (d+1) x (d+1)
+ * normal equations solved by Cholesky factorisation, the eigenvectors of
+ * R^T R by cyclic Jacobi rotations, and one pass O += O (B P) + b P.  Normal
+ * equations that are not positive definite (lam = 0 with fewer than d + 1
+ * independent probe rows, for instance) leave that head uncorrected and are
+ * flagged (spattn_check: SPATTN_ERR_DEVICE).  B*H <= 65535. */
+spattn_status_t spattn_probe_correct(spattn_plan_t plan, const void* Q, const void* K,
+                                     const void* V, void* O, const int32_t* probes, int M,
+                                     float lam, int r, void* workspace, void* scratch,
+                                     void* stream);
+
 /* Copy the fp32 block means [B, H, nb, d] left in the workspace by the last
  * pool/route into caller device buffers (any may be NULL). */
 spattn_status_t spattn_means(spattn_plan_t plan, const void* workspace, float* Qbar,

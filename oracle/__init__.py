@@ -24,9 +24,9 @@ plainly and slowly, in float64 from the exact bf16 inputs:
 * optional token reordering before blocking and its inverse after
   (DFSAttn abstract: Hilbert curve-based token reordering);
 * the probe-fitted residual correction (SparsePR page, section 2B): exact
-  dense rows for a few probes, a ridge-fitted affine map of their residuals,
-  restricted to the residuals' leading right singular subspace
-  (:mod:`oracle.probe_residual`).
+  dense rows for a few probes (chosen by the seeded generator and passed in),
+  a ridge-fitted affine map of their residuals, restricted to the residuals'
+  leading right singular subspace (:mod:`oracle.probe_residual`).
 
 Readings where the pages are silent are listed in the module docstrings of
 :mod:`oracle.spattn_ref` and :mod:`oracle.hilbert`.

@@ -11,10 +11,11 @@ sparse output of every other row.  Probe rows keep their exact output.
 Readings of points the page leaves open (also listed in the design notes):
 
 * the fit is per (batch, head): one attention call per head;
-* probes: the same number of tokens from every query block, at seeded
-  offsets inside it (stratified across query groups: the page's groups are
-  the blocks here); the probe count is a parameter, since the page gives
-  none;
+* probes are an input (random draws of the method, made by the seeded
+  generator workloads.probe_rows: the same number of tokens from every
+  query block at seeded offsets, i.e. stratified across query groups, the
+  page's groups being the blocks here); the probe count is a parameter,
+  since the page gives none;
 * the ridge penalty lam applies to B only, not to the bias b (the usual
   ridge-with-intercept);
 * the subspace is that of the r leading right singular vectors of R (the
@@ -29,20 +30,6 @@ from typing import Optional
 import numpy as np
 
 from . import spattn_ref
-
-
-def probe_rows(N: int, b: int, seed, per_block: int = 1) -> np.ndarray:
-    """per_block distinct probe tokens in each block of b tokens (all of a
-    block shorter than that), at seeded offsets: ascending token indices in
-    the blocked order.  seed is anything numpy's default_rng accepts."""
-    rng = np.random.default_rng(seed)
-    nb = (N + b - 1) // b
-    out = []
-    for i in range(nb):
-        n_i = min(b, N - i * b)
-        k = min(per_block, n_i)
-        out.extend(i * b + np.sort(rng.choice(n_i, k, replace=False)))
-    return np.asarray(out, dtype=np.int64)
 
 
 def fit_affine_residual(X: np.ndarray, R: np.ndarray, lam: float):

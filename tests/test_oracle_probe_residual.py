@@ -15,17 +15,7 @@ from sklearn.linear_model import Ridge
 
 from oracle import probe_residual as P
 from oracle import spattn_ref as R
-from workloads import get_config, make_qkv
-
-
-@pytest.mark.parametrize("per_block", [1, 3, 64])
-def test_probe_rows_are_stratified_over_blocks(per_block):
-    for N, b in ((10, 4), (64, 64), (65, 64), (1000, 64), (7, 8)):
-        rows = P.probe_rows(N, b, 3, per_block)
-        n = R.block_sizes(N, b)
-        assert np.array_equal(np.bincount(rows // b, minlength=len(n)), np.minimum(n, per_block))
-        assert np.all(np.diff(rows) > 0) and rows[-1] < N
-        assert np.array_equal(rows, P.probe_rows(N, b, 3, per_block))
+from workloads import get_config, make_qkv, probe_rows
 
 
 def test_one_dimensional_fit_by_hand():
@@ -84,7 +74,7 @@ def test_affine_low_rank_residual_is_recovered_exactly():
     B0 = rng.standard_normal((d, r0)) @ U.T
     O = rng.standard_normal((N, d))
     truth = O + b0[None, :] + O @ B0
-    probes = P.probe_rows(N, 5, 0)[:m]
+    probes = probe_rows(N, 5, 0)[:m]
     out = P.correct(O, truth[probes], probes, 1e-12, r0)
     np.testing.assert_allclose(out, truth, rtol=0, atol=1e-8)
 
@@ -144,7 +134,7 @@ def test_forward_probe_keeps_probes_exact_and_shrinks_the_error():
     w = get_config("tiny")
     Q, K, V = make_qkv(w)
     B, H, N, d = Q.shape
-    probes = np.stack([np.stack([P.probe_rows(N, w.b, (5, bi, hi), 16) for hi in range(H)])
+    probes = np.stack([np.stack([probe_rows(N, w.b, (5, bi, hi), 16) for hi in range(H)])
                        for bi in range(B)])
     res = P.forward_probe(Q, K, V, w.b, w.tau, 1, 2, 1, probes, 100.0, d)
     for hi in range(H):

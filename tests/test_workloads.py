@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from workloads import (bf16_bits_to_f32, f32_to_bf16_bits, get_config, grid_positions,
-                       make_qkv)
+                       make_qkv, probe_rows)
 
 
 def test_bf16_rounding_matches_torch():
@@ -64,3 +64,13 @@ def test_logits_follow_the_recipe(name, scale):
             assert abs(s[m].mean() - want) < 0.08 * scale, (h, lo, s[m].mean(), want)
         assert abs(v.mean()) < 0.01 and abs(v.var() - 1.0) < 0.01
         assert abs((q - k).var() - 2 * 0.3 ** 2) < 0.01                  # independent N(0, 0.3^2) noise
+
+
+@pytest.mark.parametrize("per_block", [1, 3, 64])
+def test_probe_rows_are_stratified_over_blocks(per_block):
+    for N, b in ((10, 4), (64, 64), (65, 64), (1000, 64), (7, 8)):
+        rows = probe_rows(N, b, 3, per_block)
+        n = np.array([min(b, N - i * b) for i in range(-(-N // b))])
+        assert np.array_equal(np.bincount(rows // b, minlength=len(n)), np.minimum(n, per_block))
+        assert np.all(np.diff(rows) > 0) and rows[-1] < N
+        assert np.array_equal(rows, probe_rows(N, b, 3, per_block))

@@ -1,0 +1,76 @@
+"""Probe-fitted residual correction (SparsePR page, section 2B) through the C
+ABI against the oracle: the library's routed output is corrected on the GPU
+and, from the same routed output, by oracle.probe_residual.correct with the
+oracle's own exact probe rows; the two must agree within the output bounds,
+and the probe rows must hold their exact output."""
+import numpy as np
+import pytest
+
+from oracle import probe_residual as P
+from oracle import spattn_ref as R
+from tests.harness import MAX_ABS, REL_L2, compare_outputs, from_dev, to_dev
+from workloads import get_config, make_qkv, probe_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu(gpu_required):
+    import block_sparse_attention_33_b200 as sp
+    sp.lib()
+
+
+def _run(w, per_block, lam, r, bad_probe=False):
+    import torch
+    import block_sparse_attention_33_b200 as sp
+    Q, K, V = make_qkv(w)
+    probes = np.stack([np.stack([probe_rows(w.N, w.b, (5, bi, hi), per_block)
+                                 for hi in range(w.H)]) for bi in range(w.B)]).astype(np.int32)
+    if bad_probe:
+        probes[0, 0, 0] = w.N + 3
+    plan = sp.Plan(w.B, w.H, w.N, w.d, w.b, w.tau, w.kmin, w.kmax, w.residual)
+    try:
+        q, k, v = to_dev(Q), to_dev(K), to_dev(V)
+        o = torch.zeros_like(q)
+        plan.forward(q, k, v, o)
+        assert plan.check() == sp.OK
+        o_sparse = from_dev(o)
+        plan.probe_correct(q, k, v, o, torch.from_numpy(probes).cuda(), lam, r)
+        status = plan.check()
+        return Q, K, V, probes, o_sparse, from_dev(o), status
+    finally:
+        plan.close()
+
+
+CASES = [
+    ("tiny d=64, r=16", "tiny", dict(kmax=2), 16, 100.0, 16),
+    ("medium 2 heads, r=8", "medium", dict(H=2, tau=0.8), 4, 100.0, 8),
+    ("medium 2 heads, r=d", "medium", dict(H=2, tau=0.8), 4, 10.0, 128),
+    ("medium 2 heads, r=0", "medium", dict(H=2, tau=0.8), 2, 100.0, 0),
+]
+
+
+@pytest.mark.parametrize("desc,name,ov,per_block,lam,r", CASES, ids=[c[0] for c in CASES])
+def test_probe_correction_against_oracle(desc, name, ov, per_block, lam, r):
+    import block_sparse_attention_33_b200 as sp
+    w = get_config(name, **ov)
+    Q, K, V, probes, o_sparse, o_corr, status = _run(w, per_block, lam, r)
+    assert status == sp.OK
+    for bi in range(w.B):
+        for hi in range(w.H):
+            q, k, v = (R.decode_bf16(X[bi, hi]) for X in (Q, K, V))
+            rows = probes[bi, hi].astype(np.int64)
+            dense = P.dense_rows(q, k, v, rows)
+            want = P.correct(o_sparse[bi, hi], dense, rows, lam, r)
+            max_abs, rel = compare_outputs(o_corr[bi, hi], want)
+            assert max_abs < MAX_ABS and rel < REL_L2, (bi, hi, max_abs, rel)
+            # probe rows: the exact output, one bf16 rounding
+            assert np.abs(o_corr[bi, hi][rows] - dense).max() <= 2.0 ** -8 * np.abs(dense).max()
+
+
+def test_probe_index_out_of_range_is_flagged():
+    import block_sparse_attention_33_b200 as sp
+    w = get_config("tiny", kmax=2)
+    *_, o_sparse, o_corr, status = _run(w, 4, 100.0, 8, bad_probe=True)
+    assert status == sp.ERR_DEVICE
+    assert np.isfinite(o_corr).all()

@@ -34,7 +34,7 @@ import numpy as np
 
 __all__ = [
     "Workload", "CONFIGS", "get_config", "grid_positions", "make_qkv",
-    "f32_to_bf16_bits", "bf16_bits_to_f32",
+    "f32_to_bf16_bits", "bf16_bits_to_f32", "probe_rows",
 ]
 
 
@@ -157,3 +157,18 @@ def make_qkv(w: Workload, threads: Optional[int] = None):
         with ThreadPoolExecutor(n_threads) as ex:
             list(ex.map(run, jobs))
     return Q, K, V
+
+
+def probe_rows(N: int, b: int, seed, per_block: int = 1) -> np.ndarray:
+    """Probe tokens of one head for the probe-fitted residual correction:
+    per_block distinct tokens drawn from each block of b tokens (all of a
+    block shorter than that), ascending.  seed is anything numpy's
+    default_rng accepts."""
+    rng = np.random.default_rng(seed)
+    nb = (N + b - 1) // b
+    out = []
+    for i in range(nb):
+        n_i = min(b, N - i * b)
+        k = min(per_block, n_i)
+        out.extend(i * b + np.sort(rng.choice(n_i, k, replace=False)))
+    return np.asarray(out, dtype=np.int64)
