@@ -8,7 +8,7 @@
 namespace spattn {
 
 // Device error word codes (workspace control block, word 0).
-enum : int { DEV_OK = 0, DEV_BAD_INDEX = 1, DEV_TIMEOUT = 2, DEV_NUMERIC = 3 };
+enum : int { DEV_OK = 0, DEV_BAD_INDEX = 1, DEV_TIMEOUT = 2 };
 
 // Control block layout inside the workspace (int32 words).
 enum : int {

@@ -10,6 +10,10 @@ namespace spattn {
 
 enum { ROUTING_CENTROID = 0, ROUTING_PAMA = 1 };
 
+// Device error code of the probe correction (after DEV_OK, DEV_BAD_INDEX and
+// DEV_TIMEOUT): normal equations that are not positive definite.
+enum : int { DEV_NUMERIC = 3 };
+
 // Problem description derived from a plan (all sizes in elements).
 struct Problem {
   int B, H, N, d, b, nb, n_last, kcap;
