@@ -223,3 +223,51 @@ def test_binding_checks_host_tensors_of_the_host_forward(L):
     with pytest.raises(ValueError, match="CUDA tensor"):       # host tensors pass; the workspace must be on the device
         sp.spattn_forward_host(h, x, x, x, x, w, stg, 1)
     sp.spattn_plan_destroy(h)
+
+
+def test_probe_correct_argument_checks(L):
+    """spattn_probe_scratch_bytes sizes the exact rows, the fit, B P and b P;
+    spattn_probe_correct refuses bad arguments before any CUDA call."""
+    B, H, N, d = 1, 3, 1000, 64
+    st, h, ws = plan_status(B, H, N, d, 64, 0.9, 1, 4, 1)
+    assert st == sp.OK
+    up = lambda x: (x + 255) // 256 * 256
+    n = ctypes.c_size_t()
+    M = 48
+    assert L.spattn_probe_scratch_bytes(h, M, ctypes.byref(n)) == sp.OK
+    assert n.value == (up(B * H * M * d * 4) + up(B * H * (d + 1) * d * 4) + up(B * H * d * d * 4)
+                       + up(B * H * d * 4))
+    assert L.spattn_probe_scratch_bytes(h, 0, ctypes.byref(n)) == sp.ERR_INVALID_ARG
+    f = L.spattn_probe_correct
+    ok = dict(Q=16, K=16, V=16, O=16, probes=16, M=M, lam=100.0, r=8, ws=256, scratch=256)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(h, a["Q"], a["K"], a["V"], a["O"], a["probes"], a["M"], a["lam"], a["r"],
+                 a["ws"], a["scratch"], None)
+    assert call(O=None) == sp.ERR_INVALID_ARG
+    assert call(O=8) == sp.ERR_INVALID_ARG                      # misaligned O
+    assert call(probes=None) == sp.ERR_INVALID_ARG
+    assert call(M=0) == sp.ERR_INVALID_ARG
+    assert call(lam=-1.0) == sp.ERR_INVALID_ARG
+    assert call(lam=float("nan")) == sp.ERR_INVALID_ARG
+    assert call(r=-1) == sp.ERR_INVALID_ARG and call(r=d + 1) == sp.ERR_INVALID_ARG
+    assert call(scratch=None) == sp.ERR_WORKSPACE and call(scratch=272) == sp.ERR_WORKSPACE
+    assert call(ws=None) == sp.ERR_WORKSPACE
+    assert L.spattn_plan_destroy(h) == sp.OK
+
+
+def test_binding_checks_the_probe_tensor(L):
+    import torch
+    B, H, N, d = 1, 2, 256, 64
+    h, ws = sp.spattn_plan(B, H, N, d, 64, 0.9, 1, 4, 1)
+    x = torch.zeros(B * H * N * d, dtype=torch.bfloat16)
+    w = torch.zeros(ws, dtype=torch.uint8)
+    stg = torch.zeros(sp.spattn_probe_scratch_bytes(h, 8), dtype=torch.uint8)
+    with pytest.raises(ValueError, match="probes: dtype"):
+        sp.spattn_probe_correct(h, x, x, x, x, torch.zeros(B * H * 8, dtype=torch.int64), 8, 1.0, 4, w, stg)
+    with pytest.raises(ValueError, match="probes: needs exactly"):
+        sp.spattn_probe_correct(h, x, x, x, x, torch.zeros(B * H * 8 - 1, dtype=torch.int32), 8, 1.0, 4, w, stg)
+    with pytest.raises(ValueError, match="scratch"):
+        sp.spattn_probe_correct(h, x, x, x, x, torch.zeros(B * H * 8, dtype=torch.int32), 8, 1.0, 4, w, stg[:-1])
+    sp.spattn_plan_destroy(h)
