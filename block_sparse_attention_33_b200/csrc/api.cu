@@ -13,6 +13,8 @@
 #include <utility>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "spattn.h"
 #include "common.cuh"
 #include "internal.h"
@@ -45,6 +47,15 @@ spattn_status_t fail(spattn_status_t st, const char* fmt, ...) {
 spattn_status_t cuda_fail(cudaError_t e, const char* what) {
   return fail(SPATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
+
+// NVTX range over one library call (host side), so that profilers can group
+// the kernels a call enqueues; free when no tool is attached.
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
 
 constexpr size_t ALIGN = 256;
 inline size_t up(size_t x) { return (x + ALIGN - 1) / ALIGN * ALIGN; }
@@ -251,7 +262,13 @@ spattn_status_t spattn_plan_ex(spattn_plan_t* out, int B, int H, int N, int d, i
     p.test_stall = (st && strcmp(st, "1") == 0) ? 1 : 0;
   }
   if (perm_host) {
-    cudaError_t e = cudaMalloc(&P->perm_dev, sizeof(int32_t) * (size_t)N);
+    // Failure-path test: with SPATTN_TEST_FAIL_ALLOC=1 in the environment the
+    // permutation's device allocation reports out-of-memory without being
+    // attempted, so the error path runs without exhausting any memory.
+    const char* fa = getenv("SPATTN_TEST_FAIL_ALLOC");
+    cudaError_t e = (fa && strcmp(fa, "1") == 0)
+                        ? cudaErrorMemoryAllocation
+                        : cudaMalloc(&P->perm_dev, sizeof(int32_t) * (size_t)N);
     if (e != cudaSuccess) { delete P; return cuda_fail(e, "cudaMalloc(perm)"); }
     e = cudaMemcpy(P->perm_dev, perm_host, sizeof(int32_t) * (size_t)N, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) { cudaFree(P->perm_dev); delete P; return cuda_fail(e, "cudaMemcpy(perm)"); }
@@ -281,6 +298,7 @@ spattn_status_t spattn_plan_info(spattn_plan_t plan, int* nb, int64_t* col_capac
 
 spattn_status_t spattn_pool(spattn_plan_t plan, const void* Q, const void* K, const void* V,
                             void* workspace, void* stream) {
+  Range range("spattn_pool");
   if (spattn_status_t st = check_inputs(plan, Q, K, V, workspace)) return st;
   const Work w = bind(plan->p, plan->L, workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -292,6 +310,7 @@ spattn_status_t spattn_pool(spattn_plan_t plan, const void* Q, const void* K, co
 
 spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, const void* V,
                              void* workspace, int32_t* row_ptr, int32_t* col_idx, void* stream) {
+  Range range("spattn_route");
   if (spattn_status_t st = check_inputs(plan, Q, K, V, workspace)) return st;
   const Work w = bind(plan->p, plan->L, workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -307,6 +326,7 @@ spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, c
 spattn_status_t spattn_attend(spattn_plan_t plan, const void* Q, const void* K, const void* V,
                               const int32_t* row_ptr, const int32_t* col_idx, void* O,
                               void* workspace, void* stream) {
+  Range range("spattn_attend");
   if (spattn_status_t st = check_inputs(plan, Q, K, V, workspace)) return st;
   if (!O) return fail(SPATTN_ERR_INVALID_ARG, "O must be non-NULL");
   if (reinterpret_cast<uintptr_t>(O) & 15) return fail(SPATTN_ERR_INVALID_ARG, "O must be 16-byte aligned");
@@ -322,6 +342,7 @@ spattn_status_t spattn_attend(spattn_plan_t plan, const void* Q, const void* K, 
 
 spattn_status_t spattn_forward(spattn_plan_t plan, const void* Q, const void* K, const void* V,
                                void* O, void* workspace, void* stream) {
+  Range range("spattn_forward");
   if (spattn_status_t st = spattn_route(plan, Q, K, V, workspace, nullptr, nullptr, stream)) return st;
   return spattn_attend(plan, Q, K, V, nullptr, nullptr, O, workspace, stream);
 }
@@ -337,6 +358,7 @@ spattn_status_t spattn_host_staging_bytes(spattn_plan_t plan, int chunk_heads, s
 spattn_status_t spattn_forward_host(spattn_plan_t plan, const void* Q_host, const void* K_host,
                                     const void* V_host, void* O_host, void* workspace,
                                     void* staging, int chunk_heads, void* stream) {
+  Range range("spattn_forward_host");
   if (spattn_status_t st = check_plan(plan)) return st;
   if (!Q_host || !K_host || !V_host || !O_host)
     return fail(SPATTN_ERR_INVALID_ARG, "Q_host, K_host, V_host and O_host must be non-NULL");
@@ -433,6 +455,7 @@ spattn_status_t spattn_probe_correct(spattn_plan_t plan, const void* Q, const vo
                                      const void* V, void* O, const int32_t* probes, int M,
                                      float lam, int r, void* workspace, void* scratch,
                                      void* stream) {
+  Range range("spattn_probe_correct");
   if (spattn_status_t st = check_inputs(plan, Q, K, V, workspace)) return st;
   const Problem& p = plan->p;
   if (!O || (reinterpret_cast<uintptr_t>(O) & 15))

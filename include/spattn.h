@@ -74,6 +74,9 @@ typedef struct spattn_plan_s* spattn_plan_t;
  *                       memory it owns (this needs a current CUDA device);
  *   workspace_bytes     out: bytes of device workspace the route/attend/
  *                       forward calls need (256-byte aligned base).
+ * (Failure-path test: with SPATTN_TEST_FAIL_ALLOC=1 in the environment, the
+ * device allocation of the permutation reports out-of-memory without being
+ * attempted, and the call returns SPATTN_ERR_CUDA with no plan.)
  * Validation happens before any CUDA call.  The plan is immutable and may
  * be shared by threads; one workspace must not be used by two calls that
  * overlap on the device. */

@@ -271,3 +271,18 @@ def test_binding_checks_the_probe_tensor(L):
     with pytest.raises(ValueError, match="scratch"):
         sp.spattn_probe_correct(h, x, x, x, x, torch.zeros(B * H * 8, dtype=torch.int32), 8, 1.0, 4, w, stg[:-1])
     sp.spattn_plan_destroy(h)
+
+
+def test_injected_allocation_failure_returns_an_error_and_no_plan(L, monkeypatch):
+    """Host-side fault injection: the permutation's device allocation reports
+    out-of-memory (SPATTN_TEST_FAIL_ALLOC=1); the plan call returns
+    SPATTN_ERR_CUDA, leaves no plan and names the failing call."""
+    monkeypatch.setenv("SPATTN_TEST_FAIL_ALLOC", "1")
+    perm = np.arange(256, dtype=np.int32)[::-1].copy()
+    st, h, ws = plan_status(1, 2, 256, 64, 64, 0.9, 1, 4, 1, perm=perm)
+    assert st == sp.ERR_CUDA and not h
+    msg = L.spattn_last_error()
+    assert b"cudaMalloc(perm)" in msg and b"out of memory" in msg
+    with pytest.raises(sp.SpAttnError) as ei:
+        sp.Plan(1, 2, 256, 64, 64, 0.9, 1, 4, 1, perm=perm, device="cpu")
+    assert ei.value.status == sp.ERR_CUDA
