@@ -286,3 +286,43 @@ def test_injected_allocation_failure_returns_an_error_and_no_plan(L, monkeypatch
     with pytest.raises(sp.SpAttnError) as ei:
         sp.Plan(1, 2, 256, 64, 64, 0.9, 1, 4, 1, perm=perm, device="cpu")
     assert ei.value.status == sp.ERR_CUDA
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <stdlib.h>
+#include "spattn.h"
+
+int main(void) {
+  spattn_plan_t plan = NULL;
+  size_t ws = 0;
+  int nb = 0;
+  int64_t cap = 0;
+  int32_t perm[2 * 3 * 4];
+  if (spattn_plan(&plan, 1, 2, 1000, 64, 64, 0.9f, 1, 4, 1, NULL, &ws) != SPATTN_OK) return 1;
+  if (spattn_plan_info(plan, &nb, &cap) != SPATTN_OK || nb != 16 || cap != 2 * 16 * 4) return 2;
+  if (spattn_plan_destroy(plan) != SPATTN_OK) return 3;
+  if (spattn_plan(&plan, 1, 2, 1000, 96, 64, 0.9f, 1, 4, 1, NULL, &ws) != SPATTN_ERR_UNSUPPORTED) return 4;
+  if (spattn_last_error()[0] == 0) return 5;
+  if (spattn_hilbert_perm(2, 3, 4, perm) != SPATTN_OK) return 6;
+  printf("ok %zu %d\n", ws, perm[0]);
+  return 0;
+}
+"""
+
+
+def test_header_is_c_and_the_library_links_from_c(L, tmp_path):
+    """The boundary is a C ABI: a C99 program built with gcc against
+    include/spattn.h and libspattn.so runs the host-side calls."""
+    import subprocess
+    from block_sparse_attention_33_b200 import build
+    src = tmp_path / "use.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "use"
+    libdir = os.path.dirname(build.LIB)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        str(src), "-o", str(exe), "-L", libdir, "-lspattn",
+                        f"-Wl,-rpath,{libdir}"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.startswith("ok "), (r.returncode, r.stdout, r.stderr)
