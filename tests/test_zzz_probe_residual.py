@@ -64,8 +64,10 @@ def test_probe_correction_against_oracle(desc, name, ov, per_block, lam, r):
             want = P.correct(o_sparse[bi, hi], dense, rows, lam, r)
             max_abs, rel = compare_outputs(o_corr[bi, hi], want)
             assert max_abs < MAX_ABS and rel < REL_L2, (bi, hi, max_abs, rel)
-            # probe rows: the exact output, one bf16 rounding
-            assert np.abs(o_corr[bi, hi][rows] - dense).max() <= 2.0 ** -8 * np.abs(dense).max()
+            # probe rows: the exact output (fp32 on the device), one bf16 rounding (at most
+            # 2^-8 relative)
+            assert (np.abs(o_corr[bi, hi][rows] - dense).max()
+                    <= 2.0 ** -8 * np.abs(dense).max() + 1e-5)
 
 
 def test_probe_index_out_of_range_is_flagged():
