@@ -39,7 +39,8 @@ def _route_both(w, perm=None):
         ci = torch.full((plan.col_capacity,), -5, dtype=torch.int32, device="cuda")
         perm_dev = None if perm is None else torch.from_numpy(np.asarray(perm, np.int32)).cuda()
         st = sp.lib().spattn_route_static(w.B, w.H, w.N, w.d, w.b, float(w.tau), w.kmin, w.kmax,
-                                          sp._ptr(perm_dev), q.data_ptr(), k.data_ptr(),
+                                          None if perm_dev is None else perm_dev.data_ptr(),
+                                          q.data_ptr(), k.data_ptr(),
                                           rp.data_ptr(), ci.data_ptr(),
                                           torch.cuda.current_stream().cuda_stream)
         assert st == sp.OK, sp.spattn_last_error()
