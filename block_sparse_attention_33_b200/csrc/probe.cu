@@ -29,8 +29,6 @@
 // leave that head uncorrected and are flagged (DEV_NUMERIC).
 #include <math.h>
 
-#include <algorithm>
-
 #include "common.cuh"
 #include "internal.h"
 
