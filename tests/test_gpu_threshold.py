@@ -65,3 +65,19 @@ def test_threshold_zero_keeps_everything_like_tau_one():
     assert np.array_equal(a["row_ptr"], c["row_ptr"]) and np.array_equal(a["col_idx"], c["col_idx"])
     assert a["row_ptr"][-1] == w.H * w.nb * w.nb
     assert np.array_equal(a["O"], c["O"])
+
+
+@pytest.mark.parametrize("theta,kmax", [(0.005, 256), (0.002, 64)],
+                         ids=["wan theta 0.005 (no clamp)", "wan theta 0.002, kmax 64 (every row clamped)"])
+def test_threshold_at_wan_size(theta, kmax):
+    """nb = 256: above 128 blocks a binding clamp takes the binary-search
+    top-k; routing is compared on every query block, outputs on the sampled
+    rows of the full-size tests."""
+    import block_sparse_attention_33_b200 as sp
+    from tests.test_gpu_full_size import sample_rows
+    w = get_config("wan", H=2, tau=theta, kmax=kmax)
+    Q, K, V = make_qkv(w)
+    res = run_library(w, Q, K, V, routing=sp.ROUTING_CENTROID | sp.SELECT_THRESHOLD)
+    assert res["status"] == 0
+    rows = sample_rows(w, res, None)
+    _ok(oracle_check(w, Q, K, V, res, rows=rows, selection="threshold"))
