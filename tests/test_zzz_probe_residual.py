@@ -47,6 +47,7 @@ CASES = [
     ("medium 2 heads, r=8", "medium", dict(H=2, tau=0.8), 4, 100.0, 8),
     ("medium 2 heads, r=d", "medium", dict(H=2, tau=0.8), 4, 10.0, 128),
     ("medium 2 heads, r=0", "medium", dict(H=2, tau=0.8), 2, 100.0, 0),
+    ("wan 2 heads (512 key tiles), r=8", "wan", dict(H=2), 1, 100.0, 8),
 ]
 
 
