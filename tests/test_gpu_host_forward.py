@@ -28,6 +28,7 @@ CASES = [
     ("medium, pageable host memory", "medium", dict(H=4, tau=0.8), 2, False),
     ("tiny b=64 (warp-MMA attention), chunks of 1", "tiny", dict(H=3), 1, True),
     ("stress with Hilbert permutation, chunks of 1", "stress", dict(H=3), 1, True),
+    ("wan 8 heads, chunks of 3 (3+3+2)", "wan", dict(H=8), 3, True),
 ]
 
 
