@@ -8,7 +8,7 @@ regression; the fitted correction is restricted to the subspace spanned by
 the leading right singular vectors of the probe residuals and added to the
 sparse output of every other row.  Probe rows keep their exact output.
 
-Readings of points the page leaves open (also listed in the design notes):
+Readings of points the page leaves open:
 
 * the fit is per (batch, head): one attention call per head;
 * probes are an input (random draws of the method, made by the seeded

@@ -4,8 +4,7 @@ Notation: Q, K, V are [B, H, N, d]; tokens are cut into nb = ceil(N/b) blocks
 of b tokens, block j holding n_j tokens (only the last block may be partial).
 Query blocks use the same partition as key blocks.
 
-Readings of points the pages leave open (each one is also listed in the
-design notes):
+Readings of points the pages leave open:
 
 * natural logarithm in the ln n_j term; scale 1/sqrt(d) on every logit, the
   proxy and the pseudo-keys alike;
