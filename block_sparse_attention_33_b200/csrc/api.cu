@@ -223,6 +223,9 @@ spattn_status_t spattn_plan_ex(spattn_plan_t* out, int B, int H, int N, int d, i
   if (nb > 2048) return fail(SPATTN_ERR_UNSUPPORTED, "nb = %lld blocks exceeds 2048", nb);
   if ((long long)B * H * nb > (1LL << 30) || (long long)B * H * (long long)N * d > (1LL << 40))
     return fail(SPATTN_ERR_UNSUPPORTED, "problem too large");
+  // the routing kernels index (batch, head) pairs by the grid's y dimension
+  if ((long long)B * H > 65535)
+    return fail(SPATTN_ERR_UNSUPPORTED, "B*H = %lld exceeds 65535", (long long)B * H);
   // kept-list offsets (CSR row_ptr, per-row list bases) are int32
   if ((long long)B * H * nb * std::min<long long>(kmax, nb) > 0x7FFFFFFFLL)
     return fail(SPATTN_ERR_UNSUPPORTED, "kept-list capacity B*H*nb*min(kmax, nb) = %lld exceeds 2^31 - 1",

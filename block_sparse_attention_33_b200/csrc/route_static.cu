@@ -87,6 +87,7 @@ extern "C" spattn_status_t spattn_route_static(int B, int H, int N, int d, int b
     return fail(SPATTN_ERR_INVALID_ARG, "Q and K must be 16-byte aligned");
   const long long nb = (N + (long long)b - 1) / b;
   if (nb > 2048) return fail(SPATTN_ERR_UNSUPPORTED, "nb = %lld blocks exceeds 2048", nb);
+  if ((long long)B * H > 65535) return fail(SPATTN_ERR_UNSUPPORTED, "B*H exceeds 65535");
 
   spattn::Problem p;
   p.B = B; p.H = H; p.N = N; p.d = d; p.b = b;

@@ -39,7 +39,7 @@
  *     C++ exception crosses this boundary.
  *   - Supported: d in {64, 128}; b in {64, 128}; 1 <= N; nb <= 2048;
  *     1 <= kmin <= kmax (kmax > nb is clamped to nb); tau finite;
- *     B*H*nb*min(kmax, nb) <= 2^31 - 1 (int32 CSR offsets).
+ *     B*H <= 65535; B*H*nb*min(kmax, nb) <= 2^31 - 1 (int32 CSR offsets).
  */
 #ifndef SPATTN_H_
 #define SPATTN_H_

@@ -326,3 +326,13 @@ def test_header_is_c_and_the_library_links_from_c(L, tmp_path):
     assert r.returncode == 0, r.stderr
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0 and r.stdout.startswith("ok "), (r.returncode, r.stdout, r.stderr)
+
+
+def test_plan_rejects_more_than_65535_heads(L):
+    st, h, ws = plan_status(1, 65536, 64, 64, 64, 0.9, 1, 4, 1)
+    assert st == sp.ERR_UNSUPPORTED and b"65535" in L.spattn_last_error()
+    st, h, ws = plan_status(3, 21845, 64, 64, 64, 0.9, 1, 4, 1)      # 65535 pairs: accepted
+    assert st == sp.OK
+    assert L.spattn_plan_destroy(h) == sp.OK
+    assert L.spattn_route_static(2, 40000, 64, 64, 64, 0.9, 1, 4, None, 16, 16, 16, 16, None) \
+        == sp.ERR_UNSUPPORTED
