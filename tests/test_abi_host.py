@@ -336,3 +336,15 @@ def test_plan_rejects_more_than_65535_heads(L):
     assert L.spattn_plan_destroy(h) == sp.OK
     assert L.spattn_route_static(2, 40000, 64, 64, 64, 0.9, 1, 4, None, 16, 16, 16, 16, None) \
         == sp.ERR_UNSUPPORTED
+
+
+def test_build_stamp_tells_variant_builds_apart(L):
+    """The library on disk records its extra compiler flags: the default build
+    is up to date for no extra flags and not for others, so a variant build
+    is never mistaken for the default one (and vice versa)."""
+    from block_sparse_attention_33_b200 import build
+    build.build()
+    assert build.up_to_date(())
+    assert not build.up_to_date(("-DSPATTN_EXP_EMU=2",))
+    with open(build.STAMP) as f:
+        assert f.read() == ""
