@@ -37,6 +37,14 @@
  *   - Every call returns a spattn_status_t; spattn_last_error() gives a
  *     human-readable message for the calling thread's last failure.  No
  *     C++ exception crosses this boundary.
+ *   - CUDA graphs: spattn_pool, spattn_route, spattn_attend, spattn_forward,
+ *     spattn_means and spattn_probe_correct enqueue kernels and async copies
+ *     only, so they can be captured once each has run eagerly with the same
+ *     plan (the first call may raise a kernel's shared-memory limit and, for
+ *     spattn_probe_correct, does so for its kernels).  spattn_plan (device
+ *     allocation with a permutation), spattn_check (synchronises),
+ *     spattn_forward_host (creates streams and events) and the first
+ *     spattn_route_static call on a device are not capturable.
  *   - Supported: d in {64, 128}; b in {64, 128}; 1 <= N; nb <= 2048;
  *     1 <= kmin <= kmax (kmax > nb is clamped to nb); tau finite;
  *     B*H <= 65535; B*H*nb*min(kmax, nb) <= 2^31 - 1 (int32 CSR offsets).
