@@ -100,3 +100,23 @@ def test_warmup_below_three_is_refused():
                         "--workload", "tiny", "--steps", "1", "--warmup", "2"],
                        capture_output=True, text=True, timeout=120, cwd=ROOT)
     assert r.returncode != 0 and "warmup" in (r.stderr + r.stdout)
+
+
+def test_reference_arm_on_a_nonzero_rank_prints_nothing():
+    """Under torchrun the reference arm runs on rank 0 alone: another rank
+    exits 0 without work or output."""
+    import subprocess
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--workload", "tiny", "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=120, cwd=ROOT, env=env)
+    assert r.returncode == 0 and not [l for l in r.stdout.splitlines() if l.startswith("{")]
+
+
+def test_default_arguments_are_one_gpu_and_a_short_run():
+    sys.path.insert(0, ROOT)
+    import bench
+    a = bench.parse_args([])
+    assert a.gpus == 1 and a.impl == "ours" and a.workload == "medium"
+    assert a.warmup >= 3 and 1 <= a.steps <= 100
+    assert a.selection == "top_p" and a.routing == "centroid"
