@@ -13,7 +13,7 @@ The line also carries the dense-equivalent rate, the fraction of the
 measured bf16 tensor peak, and the speedup over the same library's dense
 (tau = 1) path on the same inputs.
 
-  python bench.py [--gpus N --steps K --warmup W] [--workload medium]
+  python bench.py [--gpus N --steps K --warmup W] [--workload hunyuan]
   python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
 """
 from __future__ import annotations
@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 METRIC = "block-sparse attn fwd: effective TFLOP/s, % of B200 BF16 peak, speedup vs dense"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS_PER_STEP = 4  # pool, route, scan, attend (the compact CSR is not asked for)
+L2_NOTE = "flushed (256 MiB write between timed steps)"
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
 # ncu capture of the bench command for that workload, keyed by kernel and
@@ -77,7 +78,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="medium",
+    ap.add_argument("--workload", default="hunyuan",
                     choices=["tiny", "medium", "wan", "hunyuan", "stress"])
     ap.add_argument("--tau", type=float, default=None)
     ap.add_argument("--residual", type=int, default=None)
@@ -97,9 +98,11 @@ def parse_args(argv=None):
                     help="override the number of heads (smaller profiling captures)")
     ap.add_argument("--no-dense", action="store_true", help="skip the tau = 1 comparison run")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-chunk", type=int, default=-1,
-                    help="also time spattn_forward_host (host tensors, copies overlapped over "
-                         "chunks of this many heads); -1: a quarter of the heads, 0: off")
+    ap.add_argument("--e2e-chunk", type=int, default=0,
+                    help="heads per chunk of spattn_forward_host in the e2e figure (host "
+                         "tensors, copies overlapped over chunks); 0: a quarter of the heads")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the compact timing of every seeded configuration")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="CPU time budget of the oracle baseline sample")
@@ -339,7 +342,8 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * float(np.mean(times)), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": dict(config_of(w, "cpu"), routing=args.routing, selection=args.selection),
+        # the GPU arm's config, so that the two lines describe the same workload
+        "config": dict(config_of(w, L2_NOTE), routing=args.routing, selection=args.selection),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": "each step: " + desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -353,6 +357,79 @@ def config_of(w, l2):
             "nb": w.nb, "tau": w.tau, "kmin": w.kmin, "kmax": w.kmax, "residual": w.residual,
             "hilbert": w.hilbert, "grid": list(w.grid), "global_batch": w.B, "seq_len": w.N,
             "parallelism": "replicas", "l2": l2}
+
+
+# The seeded configurations and the knob values they are quoted at.
+PER_CONFIG = (("tiny", {}), ("medium", {}), ("medium", {"residual": 0}),
+              ("wan", {"tau": 0.8}), ("wan", {}), ("wan", {"tau": 0.95}),
+              ("hunyuan", {"tau": 0.8}), ("hunyuan", {}),
+              ("stress", {}), ("stress", {"residual": 0}))
+
+
+def measure_configs(sp, main_w, main_qkv, main_perm, main_dense_ms, timed, as_graph, graphs,
+                    dev, steps):
+    """Step time (route + attend, CUDA-graph replays, L2 flushed between
+    steps), attention TFLOP/s, kept fraction and speedup over the dense path
+    of every entry of PER_CONFIG.  Inputs of the main workload are reused."""
+    import torch
+    from workloads import get_config, make_qkv
+    out = []
+    by_name = {}
+    for name, ov in PER_CONFIG:
+        by_name.setdefault(name, []).append(ov)
+    for name, variants in by_name.items():
+        base = get_config(name)
+        if name == main_w.name and main_w.H == base.H:
+            (q, k, v), perm = main_qkv, main_perm
+        else:
+            Qh, Kh, Vh = make_qkv(base)
+            q, k, v = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+                       for x in (Qh, Kh, Vh))
+            del Qh, Kh, Vh
+            perm = sp.spattn_hilbert_perm(*base.grid) if base.hilbert else None
+        o = torch.empty_like(q)
+        B, H, N, d = q.shape
+        dense_flops = 4 * N * N * d * B * H
+        dense_ms = main_dense_ms if (q is main_qkv[0] and main_dense_ms) else None
+        if dense_ms is None:
+            dplan = sp.Plan(B, H, N, d, base.b, 1.0, 1, 1 << 30, base.residual, perm, device=dev)
+            n0 = len(graphs)
+            td = timed([as_graph(lambda: dplan.forward(q, k, v, o))], steps, 3)
+            dense_ms = float(np.mean([x[0] for x in td]))
+            del graphs[n0:]
+            dplan.close()
+        for ov in variants:
+            w = base.with_(**ov)
+            plan = sp.Plan(B, H, N, d, w.b, w.tau, w.kmin, w.kmax, w.residual, perm, device=dev)
+            try:
+                rp = torch.zeros(B * H * plan.nb + 1, dtype=torch.int32, device=dev)
+                ci = torch.zeros(max(plan.col_capacity, 1), dtype=torch.int32, device=dev)
+                plan.route(q, k, v, rp, ci)
+                torch.cuda.synchronize(dev)
+                rpn, cin = rp.cpu().numpy(), ci.cpu().numpy()
+                exact, resid = attention_flops(rpn, cin, w, plan.nb)
+                n0 = len(graphs)
+                t = timed([as_graph(lambda: plan.route(q, k, v)),
+                           as_graph(lambda: plan.attend(q, k, v, o))], steps, 3)
+                del graphs[n0:]
+                status = plan.check()
+            finally:
+                plan.close()
+            r_ms = float(np.mean([x[0] for x in t]))
+            a_ms = float(np.mean([x[1] for x in t]))
+            kept = float(np.diff(rpn).sum()) / (B * H * plan.nb * plan.nb)
+            out.append({"workload": name, "tau": w.tau, "residual": w.residual, "H": H, "N": N,
+                        "ms_per_step": r_ms + a_ms, "route_ms": r_ms, "attend_ms": a_ms,
+                        "step_tflops": (exact + resid) / ((r_ms + a_ms) * 1e-3) / 1e12,
+                        "attn_tflops": (exact + resid) / (a_ms * 1e-3) / 1e12,
+                        "dense_equiv_tflops": dense_flops / ((r_ms + a_ms) * 1e-3) / 1e12,
+                        "kept_fraction": kept, "dense_ms": dense_ms,
+                        "speedup_vs_dense": dense_ms / (r_ms + a_ms),
+                        "dense_over_computed_flops": dense_flops / max(exact + resid, 1),
+                        "status": int(status)})
+        del q, k, v, o
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args):
@@ -477,7 +554,12 @@ def run_ours(args):
                                                               [float(step_flops)], dev)
     value = job_throughput(total_flops, step_ms)
     peaks, peak_kind = load_peaks()
-    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    # The attention kernel's peak: the burst figure when the timed region is
+    # short, the sustained (power-capped) one when the timed launches keep
+    # the GPU busy for a second or more, as the long layers do.
+    sustained = attend_ms * args.steps >= 1000.0
+    bf16_key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    bf16_peak = float(peaks.get(bf16_key, FALLBACK_PEAKS[bf16_key]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     attn_tflops = step_flops / (attend_ms * 1e-3) / 1e12
 
@@ -514,25 +596,46 @@ def run_ours(args):
     reuse_ms = float(np.mean([x[0] + x[1] for x in tr]))
     (reuse_ms,), _ = combine_over_ranks([reuse_ms], [], dev)
 
-    e2e = None
+    # end to end through the public host-buffer call: spattn_forward_host on
+    # pinned host tensors (copies in, the path, the copy out, overlapped over
+    # chunks of heads); the plain sequence of torch copies around
+    # spattn_forward is kept beside it for comparison
+    e2e = e2e_copies = None
     if not args.no_e2e:
         qh, kh, vh = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
                       for x in (Qh, Kh, Vh))
         oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        chunk = args.e2e_chunk if args.e2e_chunk > 0 else max(1, (B * H + 3) // 4)
 
-        def e2e_step():
+        def pipe_step():
+            plan.forward_host(qh, kh, vh, oh, chunk_heads=chunk)
+
+        def copies_step():
             q.copy_(qh, non_blocking=True)
             k.copy_(kh, non_blocking=True)
             v.copy_(vh, non_blocking=True)
             plan.forward(q, k, v, o)
             oh.copy_(o, non_blocking=True)
 
-        te = timed([e2e_step], max(3, args.steps // 3), 2)
-        e2e_ms = float(np.mean([x[0] for x in te]))
-        (e2e_ms,), _ = combine_over_ranks([e2e_ms], [], dev)
-        e2e = {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * tok_bytes,
-               "d2h_bytes_per_step": tok_bytes}
+        tpp = timed([pipe_step], max(3, args.steps // 3), 3)
+        pipe_ms = float(np.mean([x[0] for x in tpp]))
+        (pipe_ms,), _ = combine_over_ranks([pipe_ms], [], dev)
+        pipe_status = plan.check()
+        e2e = {"value": total_flops / (pipe_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": pipe_ms, "h2d_bytes_per_step": 3 * tok_bytes,
+               "d2h_bytes_per_step": tok_bytes, "chunk_heads": chunk,
+               "what": "spattn_forward_host through the C ABI: pinned host Q, K, V in, host O "
+                       "out, copies overlapped with the path over chunks of heads"}
+        if pipe_status != sp.OK:   # reported in the line: every rank still takes the same steps
+            e2e["error"] = f"device status {pipe_status}: {sp.spattn_last_error()}"
+        te = timed([copies_step], max(3, args.steps // 3), 3)
+        copies_ms = float(np.mean([x[0] for x in te]))
+        (copies_ms,), _ = combine_over_ranks([copies_ms], [], dev)
+        e2e_copies = {"value": total_flops / (copies_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "ms_per_step": copies_ms, "h2d_bytes_per_step": 3 * tok_bytes,
+                      "d2h_bytes_per_step": tok_bytes,
+                      "what": "torch copies in, spattn_forward, torch copy out, one after the "
+                              "other"}
 
     # threshold selection (p >= theta, Sol-Attn on-the-fly thresholding) on the
     # same inputs: a second plan, timed like the main step; one rank only
@@ -596,26 +699,16 @@ def run_ours(args):
         except Exception as ex:   # reported in the line; the measurements above stand
             probe = {"error": f"{type(ex).__name__}: {ex}"[:300]}
 
-    e2e_pipe = None
-    chunk = args.e2e_chunk if args.e2e_chunk >= 0 else max(1, (B * H + 3) // 4)
-    # one rank only: an error on one rank must not leave the others in a collective
-    if chunk > 0 and e2e is not None and world == 1:
+    # every seeded configuration (and its knob variants) timed the same way,
+    # each beside the same library's dense (tau = 1) path on its inputs; one
+    # rank only
+    per_config = None
+    if world == 1 and not args.no_per_config:
         try:
-            def pipe_step():
-                plan.forward_host(qh, kh, vh, oh, chunk_heads=chunk)
-
-            tpp = timed([pipe_step], max(3, args.steps // 3), 2)
-            pipe_ms = float(np.mean([x[0] for x in tpp]))
-            (pipe_ms,), _ = combine_over_ranks([pipe_ms], [], dev)
-            status = plan.check()
-            if status != sp.OK:
-                raise RuntimeError(f"device status {status}: {sp.spattn_last_error()}")
-            e2e_pipe = {"value": total_flops / (pipe_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                        "ms_per_step": pipe_ms, "chunk_heads": chunk,
-                        "h2d_bytes_per_step": 3 * tok_bytes, "d2h_bytes_per_step": tok_bytes,
-                        "what": "spattn_forward_host: host tensors, copies overlapped with the path"}
+            per_config = measure_configs(sp, w, (q, k, v), perm, dense_ms, timed, as_graph, graphs,
+                                         dev, max(3, min(args.steps, 10)))
         except Exception as ex:   # reported in the line; the measurements above stand
-            e2e_pipe = {"error": f"{type(ex).__name__}: {ex}"[:300], "chunk_heads": chunk}
+            per_config = {"error": f"{type(ex).__name__}: {ex}"[:300]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -628,7 +721,7 @@ def run_ours(args):
         graphs.clear()
         plan.close()
     except Exception:
-        if not any(x and "error" in x for x in (e2e_pipe, thresh, probe)):
+        if not any(x and "error" in x for x in (thresh, probe)):
             raise   # a failure already recorded in the line may also fail the clean-up
     if rank == 0:
         line = {
@@ -636,7 +729,7 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": dict(config_of(w, "flushed (256 MiB write between timed steps)"),
+            "config": dict(config_of(w, L2_NOTE),
                            routing=args.routing, selection=args.selection),
             "dense_equiv_tflops": dense_flops * world / (step_ms * 1e-3) / 1e12,
             "attn_tflops": attn_tflops,
@@ -652,7 +745,8 @@ def run_ours(args):
                            "what": "pool + attend with the kept lists of the last route"},
             "roofline": {"bound": "tensor", "kernel": "attention", "achieved": attn_tflops,
                          "peak": bf16_peak, "unit": "TFLOP/s", "frac": attn_tflops / bf16_peak,
-                         "peak_kind": f"{peak_kind} bf16 dense (burst)",
+                         "peak_kind": f"{peak_kind} bf16 dense "
+                                      f"({'sustained' if sustained else 'burst'})",
                          "traffic": measured_traffic("attention", w, args.selection), "traffic_unit": "bytes/launch"},
             "roofline_route": {"bound": "alu", "kernel": "route + scan",
                                "achieved": route_flops / (max(route_ms - pool_ms, 1e-6) * 1e-3) / 1e12,
@@ -668,7 +762,8 @@ def run_ours(args):
             "clocks": clk,
             "launch": launch,
             "e2e": e2e,
-            "e2e_pipelined": e2e_pipe,
+            "e2e_torch_copies": e2e_copies,
+            "per_config": per_config,
             "threshold_selection": thresh,
             "probe_correction": probe,
             "gpu_launches": KERNELS_PER_STEP * args.steps,

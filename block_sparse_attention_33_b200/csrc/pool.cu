@@ -93,15 +93,9 @@ __global__ void __launch_bounds__(POOL_THREADS, POOL_CTAS_PER_SM) pool_kernel(co
     const uint32_t fb = smem_u32(&fullb[slot]);
     const uint32_t dst = ring + slot * tile_bytes;
     const __nv_bfloat16* X = src_of(t) + (size_t)bh * a.N * D;
-    if (lane == 0) tc::mbar_expect_tx(fb, (uint32_t)(n * row_bytes));
-    __syncwarp();
-    if (!a.perm) {
-      if (lane == 0) tc::bulk_load(dst, X + (size_t)j * a.b * D, (uint32_t)(n * row_bytes), fb);
-    } else {
-      for (int r = lane; r < n; r += 32) {
-        const int src = __ldg(a.perm + j * a.b + r);
-        tc::bulk_load(dst + r * row_bytes, X + (size_t)src * D, (uint32_t)row_bytes, fb);
-      }
+    if (lane == 0) {
+      tc::mbar_expect_tx(fb, (uint32_t)(n * row_bytes));
+      tc::bulk_load(dst, X + (size_t)j * a.b * D, (uint32_t)(n * row_bytes), fb);
     }
   };
   if (warp == 0)
@@ -117,12 +111,6 @@ __global__ void __launch_bounds__(POOL_THREADS, POOL_CTAS_PER_SM) pool_kernel(co
     const bool ok = tc::mbar_wait(smem_u32(&fullb[slot]), (uint32_t)(k / POOL_STAGES) & 1u, abort,
                                   a.ctrl, 20);
     if (!__syncthreads_and(ok)) break;
-    __nv_bfloat16* Xp0 = t == 0 ? a.Xp[0] : t == 1 ? a.Xp[1] : a.Xp[2];
-    if (Xp0 && tid == 0) {
-      tc::bulk_store(Xp0 + ((size_t)bh * a.N + (size_t)j * a.b) * D, ring + slot * tile_bytes,
-                     (uint32_t)(n * row_bytes));
-      tc::bulk_commit();
-    }
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -139,13 +127,8 @@ __global__ void __launch_bounds__(POOL_THREADS, POOL_CTAS_PER_SM) pool_kernel(co
 #pragma unroll
     for (int e = 0; e < 8; ++e) red[r0][c * 8 + e] = acc[e];
     __syncthreads();
-    // the slot has been read (and, with a permutation, its bulk store has
-    // read it once thread 0 has waited): refill it
-    if (warp == 0) {
-      if (Xp0 && lane == 0) tc::bulk_wait_read_all();
-      __syncwarp();
-      if (k + POOL_STAGES < mine) issue(k + POOL_STAGES);
-    }
+    // the slot has been read: refill it
+    if (warp == 0 && k + POOL_STAGES < mine) issue(k + POOL_STAGES);
     if (tid < D) {
       float s = 0.f;
 #pragma unroll 8
@@ -164,7 +147,6 @@ __global__ void __launch_bounds__(POOL_THREADS, POOL_CTAS_PER_SM) pool_kernel(co
     for (int kk = issued > POOL_STAGES ? issued - POOL_STAGES : 0; kk < issued; ++kk)
       tc::mbar_drain(smem_u32(&fullb[kk % POOL_STAGES]), (uint32_t)(kk / POOL_STAGES) & 1u);
   }
-  if (tid == 0) tc::bulk_wait_all();   // permuted copies complete before exit
 }
 
 // Gather form for a permutation: rows are scattered, so each thread loads its
@@ -194,8 +176,16 @@ __global__ void __launch_bounds__(POOL_THREADS, POOL_CTAS_PER_SM) pool_gather_ke
     for (int it = 0; it < IT; ++it) {
       const int r = r0 + it * R;
       if (r < n) {
+        // a permutation entry outside [0, N) (possible only where the
+        // caller's device permutation is not checked on the host) is
+        // flagged and its row left out, never read through
         const int src = __ldg(a.perm + j * a.b + r);
-        v[it] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)src * D) + c);
+        if ((unsigned)src < (unsigned)a.N) {
+          v[it] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)src * D) + c);
+        } else {
+          v[it] = make_uint4(0u, 0u, 0u, 0u);
+          if (c == 0 && a.ctrl) flag_error(a.ctrl, DEV_BAD_INDEX, j * a.b + r);
+        }
       }
     }
   };

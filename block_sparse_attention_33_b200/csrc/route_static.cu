@@ -15,7 +15,11 @@
 // All calls share the array and it keeps the last call's contents, so every
 // call clears the words that must start at zero; calls that overlap on the GPU
 // (other streams, other host threads) race on it and must be serialised by
-// the caller.
+// the caller.  The cached address belongs to the device's current context: a
+// cudaDeviceReset invalidates it, so this entry point must not be used across
+// one.  Device-side errors (a permutation entry outside [0, N), which the
+// pooling skips without reading, or a bounded wait that gave up) are recorded
+// only in the array's control block and are not reported to the caller.
 #include <math.h>
 #include <mutex>
 #include <stdarg.h>
@@ -81,19 +85,42 @@ extern "C" spattn_status_t spattn_route_static(int B, int H, int N, int d, int b
   if (b != 64 && b != 128) return fail(SPATTN_ERR_UNSUPPORTED, "b must be 64 or 128");
   if (!isfinite(tau)) return fail(SPATTN_ERR_INVALID_ARG, "tau must be finite");
   if (kmin < 1 || kmax < kmin) return fail(SPATTN_ERR_INVALID_ARG, "need 1 <= kmin <= kmax");
+  const long long nb = (N + (long long)b - 1) / b;
+  if (nb > 2048) return fail(SPATTN_ERR_UNSUPPORTED, "nb = %lld blocks exceeds 2048", nb);
+  if ((long long)B * H > 65535) return fail(SPATTN_ERR_UNSUPPORTED, "B*H exceeds 65535");
+  const int kcap = kmax < nb ? kmax : (int)nb;
+
+  // scratch layout: control block, Qbar, Kbar (fp32), counts, padded lists,
+  // order; each region rounded up to 256 bytes.  The size is checked before
+  // the pointers, so that a caller can ask whether a shape fits without
+  // passing any buffer.
+  const size_t rows = (size_t)B * H * nb;
+  const size_t cen = rows * d * sizeof(float);
+  size_t off = 0;
+  const size_t o_ctrl = off; off += up256(spattn::CTRL_WORDS * 4);
+  const size_t o_qbar = off; off += up256(cen);
+  const size_t o_kbar = off; off += up256(cen);
+  const size_t o_counts = off; off += up256(rows * 4);
+  const size_t o_lists = off; off += up256(rows * kcap * 4);
+  const size_t o_order = off; off += up256(rows * 4);
+  if (off > kScratchBytes)
+    return fail(SPATTN_ERR_UNSUPPORTED,
+                "this problem needs %zu bytes of routing scratch; the static scratch holds %zu "
+                "bytes (use spattn_route with a caller workspace)", off, kScratchBytes);
+
   if (!Q || !K || !row_ptr || !col_idx)
     return fail(SPATTN_ERR_INVALID_ARG, "Q, K, row_ptr and col_idx must be non-NULL");
   if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K)) & 15)
     return fail(SPATTN_ERR_INVALID_ARG, "Q and K must be 16-byte aligned");
-  const long long nb = (N + (long long)b - 1) / b;
-  if (nb > 2048) return fail(SPATTN_ERR_UNSUPPORTED, "nb = %lld blocks exceeds 2048", nb);
-  if ((long long)B * H > 65535) return fail(SPATTN_ERR_UNSUPPORTED, "B*H exceeds 65535");
+  if ((reinterpret_cast<uintptr_t>(perm) | reinterpret_cast<uintptr_t>(row_ptr) |
+       reinterpret_cast<uintptr_t>(col_idx)) & 3)
+    return fail(SPATTN_ERR_INVALID_ARG, "perm, row_ptr and col_idx must be 4-byte aligned");
 
   spattn::Problem p;
   p.B = B; p.H = H; p.N = N; p.d = d; p.b = b;
   p.nb = (int)nb;
   p.n_last = N - (p.nb - 1) * b;
-  p.kcap = kmax < p.nb ? kmax : p.nb;
+  p.kcap = kcap;
   p.BH = B * H;
   p.tau = tau; p.kmin = kmin; p.kmax = kmax;
   p.residual = 0;
@@ -102,21 +129,6 @@ extern "C" spattn_status_t spattn_route_static(int B, int H, int N, int d, int b
   p.threshold = 0;
   p.test_stall = 0;
   p.perm = perm;
-
-  // scratch layout: Qbar, Kbar (fp32), counts, padded lists, order, control
-  const size_t rows = (size_t)p.BH * p.nb;
-  const size_t cen = rows * d * sizeof(float);
-  size_t off = 0;
-  const size_t o_qbar = off; off += up256(cen);
-  const size_t o_kbar = off; off += up256(cen);
-  const size_t o_counts = off; off += up256(rows * 4);
-  const size_t o_lists = off; off += up256(rows * p.kcap * 4);
-  const size_t o_order = off; off += up256(rows * 4);
-  const size_t o_ctrl = off; off += up256(spattn::CTRL_WORDS * 4);
-  if (off > kScratchBytes)
-    return fail(SPATTN_ERR_UNSUPPORTED,
-                "this problem needs %zu bytes of routing scratch; the static scratch holds %zu "
-                "bytes (use spattn_route with a caller workspace)", off, kScratchBytes);
 
   uint8_t* base = nullptr;
   if (spattn_status_t st = scratch_address(&base)) return st;

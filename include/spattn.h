@@ -285,21 +285,29 @@ spattn_status_t spattn_hilbert_perm(int T, int Hs, int W, int32_t* perm_host);
  * same shape and knobs (same kernels, bit-identical result), without a plan
  * or workspace:
  *   B, H, N, d, b, tau, kmin, kmax   as for spattn_plan;
- *   perm     NULL, or a DEVICE array of N int32 (perm[new] = old), which the
- *            caller guarantees to be a bijection (it is not checked here);
- *   Q, K     bf16 [B, H, N, d] device (V is not needed for routing);
+ *   perm     NULL, or a DEVICE array of N int32 (perm[new] = old), 4-byte
+ *            aligned, which the caller guarantees to be a bijection (it is not
+ *            checked on the host; an entry outside [0, N) is skipped by the
+ *            pooling, never read through, and the CSR is then unspecified);
+ *   Q, K     bf16 [B, H, N, d] device, 16-byte aligned (V is not needed);
  *   row_ptr  int32 [B*H*nb + 1] device, col_idx int32 [B*H*nb*min(kmax, nb)]
- *            device: the CSR, as written by spattn_route.
+ *            device, both 4-byte aligned: the CSR, as written by spattn_route.
  * Scratch lives in one file-scope device array of
  * SPATTN_ROUTE_STATIC_SCRATCH_BYTES, held by every GPU that loads the library
- * until the process exits.  A problem whose scratch (2*B*H*nb*d*4 bytes of
- * means + B*H*nb*(min(kmax,nb) + 2)*4 bytes of lists, each rounded up to 256)
- * exceeds it is rejected with SPATTN_ERR_UNSUPPORTED before anything runs.
+ * until the process exits.  A problem needs
+ *     256 + 2*up(R*d*4) + 2*up(R*4) + up(R*min(kmax, nb)*4)
+ * bytes of it, with R = B*H*nb and up() rounding up to a multiple of 256 (a
+ * control block, the fp32 means of Q and K, per-row budgets and work order,
+ * padded kept lists); a problem that needs more is rejected with
+ * SPATTN_ERR_UNSUPPORTED before any pointer is looked at or anything runs.
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  Every call shares the one array: calls that
- * overlap on the GPU (other streams or host threads) race and must be
- * serialised by the caller.  No cudaMalloc, cudaFree or allocating library
+ * (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ * first call before any stream capture, and do not use this entry point
+ * across a cudaDeviceReset (the kept address would be stale).  Every call
+ * shares the one array: calls that overlap on the GPU (other streams or host
+ * threads) race and must be serialised by the caller.  Device-side errors
+ * are not reported by this path (there is no workspace to hold them and no
+ * check call for it).  No cudaMalloc, cudaFree or allocating library
  * routine is called. */
 #define SPATTN_ROUTE_STATIC_SCRATCH_BYTES (32u << 20)
 spattn_status_t spattn_route_static(int B, int H, int N, int d, int b, float tau, int kmin,

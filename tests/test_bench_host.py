@@ -117,6 +117,7 @@ def test_default_arguments_are_one_gpu_and_a_short_run():
     sys.path.insert(0, ROOT)
     import bench
     a = bench.parse_args([])
-    assert a.gpus == 1 and a.impl == "ours" and a.workload == "medium"
+    # the headline: the largest configuration that fits one GPU
+    assert a.gpus == 1 and a.impl == "ours" and a.workload == "hunyuan"
     assert a.warmup >= 3 and 1 <= a.steps <= 100
     assert a.selection == "top_p" and a.routing == "centroid"

@@ -77,3 +77,61 @@ def test_probe_index_out_of_range_is_flagged():
     *_, o_sparse, o_corr, status = _run(w, 4, 100.0, 8, bad_probe=True)
     assert status == sp.ERR_DEVICE
     assert np.isfinite(o_corr).all()
+
+
+# The composed path against the oracle run on its own: the library's routing,
+# routed attention, exact probe rows, ridge fit, subspace and correction on
+# one side; oracle.probe_residual.forward_probe (its own routing, its own
+# sparse output, its own exact rows) on the other.  Routing may differ only on
+# marginal blocks; the corrected outputs must agree within the output bounds
+# (every row, or a seeded sample of rows at the Wan-like size).
+E2E_CASES = [
+    ("tiny d=64, r=16", "tiny", dict(kmax=2), 16, 100.0, 16, 0),
+    ("medium 2 heads, r=8", "medium", dict(H=2, tau=0.8), 4, 100.0, 8, 0),
+    ("medium 2 heads, r=d", "medium", dict(H=2), 4, 10.0, 128, 0),
+    ("wan 2 heads, 384 sampled rows, r=8", "wan", dict(H=2), 1, 100.0, 8, 384),
+]
+
+
+@pytest.mark.parametrize("desc,name,ov,per_block,lam,r,sample", E2E_CASES,
+                         ids=[c[0] for c in E2E_CASES])
+def test_composed_path_against_oracle_forward_probe(desc, name, ov, per_block, lam, r, sample):
+    import torch
+    import block_sparse_attention_33_b200 as sp
+    from tests.harness import compare_routing, csr_to_kept
+    w = get_config(name, **ov)
+    Q, K, V = make_qkv(w)
+    probes = np.stack([np.stack([probe_rows(w.N, w.b, (6, bi, hi), per_block)
+                                 for hi in range(w.H)]) for bi in range(w.B)]).astype(np.int32)
+    plan = sp.Plan(w.B, w.H, w.N, w.d, w.b, w.tau, w.kmin, w.kmax, w.residual)
+    try:
+        q, k, v = to_dev(Q), to_dev(K), to_dev(V)
+        o = torch.zeros_like(q)
+        row_ptr = torch.zeros(w.B * w.H * plan.nb + 1, dtype=torch.int32, device="cuda")
+        col_idx = torch.zeros(max(plan.col_capacity, 1), dtype=torch.int32, device="cuda")
+        plan.route(q, k, v, row_ptr, col_idx)
+        plan.attend(q, k, v, o)
+        plan.probe_correct(q, k, v, o, torch.from_numpy(probes).cuda(), lam, r)
+        assert plan.check() == sp.OK
+        got = from_dev(o)
+        gpu_kept = csr_to_kept(row_ptr.cpu().numpy(), col_idx.cpu().numpy(), w.B, w.H, plan.nb)
+    finally:
+        plan.close()
+    rows = None
+    if sample:
+        rng = np.random.default_rng(17)
+        rows = {(bi, hi): np.sort(np.concatenate([rng.choice(w.N, sample - 8, replace=False),
+                                                  probes[bi, hi][:8]]))
+                for bi in range(w.B) for hi in range(w.H)}
+    ref = P.forward_probe(Q, K, V, w.b, w.tau, w.kmin, w.kmax, w.residual, probes, lam, r,
+                          rows=rows)
+    bad, marginal, _ = compare_routing(ref["route"], gpu_kept)
+    assert bad == 0, f"{bad} non-marginal kept-set disagreements ({marginal} marginal)"
+    for bi in range(w.B):
+        for hi in range(w.H):
+            if rows is None:
+                g, want = got[bi, hi], ref["O"][bi, hi]
+            else:
+                g, want = got[bi, hi][rows[(bi, hi)]], ref["O"][(bi, hi)]
+            max_abs, rel = compare_outputs(g, want)
+            assert max_abs < MAX_ABS and rel < REL_L2, (bi, hi, max_abs, rel, marginal)

@@ -146,3 +146,26 @@ def test_forward_probe_keeps_probes_exact_and_shrinks_the_error():
         e_sparse = np.linalg.norm(res["O_sparse"][0, hi][rest] - dense[rest])
         e_corr = np.linalg.norm(res["O"][0, hi][rest] - dense[rest])
         assert e_corr < 0.99 * e_sparse
+
+
+def test_row_subset_evaluation_equals_the_full_evaluation():
+    """forward_probe(rows=...) evaluates the routed output only at the probes
+    and the requested rows; the corrected rows (probe rows among them) equal
+    those of the full evaluation, and the routing is the same."""
+    w = get_config("tiny", kmax=2)
+    Q, K, V = make_qkv(w)
+    B, H, N, d = Q.shape
+    probes = np.stack([np.stack([probe_rows(N, w.b, (5, bi, hi), 4) for hi in range(H)])
+                       for bi in range(B)])
+    full = P.forward_probe(Q, K, V, w.b, w.tau, w.kmin, w.kmax, w.residual, probes, 100.0, 8)
+    rng = np.random.default_rng(2)
+    rows = {(0, hi): np.sort(np.concatenate([rng.choice(N, 30, replace=False), probes[0, hi][:3]]))
+            for hi in range(H)}
+    sub = P.forward_probe(Q, K, V, w.b, w.tau, w.kmin, w.kmax, w.residual, probes, 100.0, 8,
+                          rows=rows)
+    for hi in range(H):
+        np.testing.assert_array_equal(sub["O"][(0, hi)], full["O"][0, hi][rows[(0, hi)]])
+        np.testing.assert_array_equal(sub["O_sparse"][(0, hi)],
+                                      full["O_sparse"][0, hi][rows[(0, hi)]])
+        for a, b in zip(sub["route"][(0, hi)]["kept"], full["route"][(0, hi)]["kept"]):
+            np.testing.assert_array_equal(a, b)

@@ -73,3 +73,49 @@ def test_static_route_rejects_problems_beyond_the_scratch():
     st = L.spattn_route_static(w.B, w.H, w.N, w.d, w.b, 0.9, 1, w.kmax, None, 16, 16, 16, 16, None)
     assert st == sp.ERR_UNSUPPORTED
     assert "static scratch" in sp.spattn_last_error()
+
+
+def _scratch_need(B, H, N, d, b, kmax):
+    """The scratch size spattn_route_static documents in include/spattn.h."""
+    up = lambda x: (x + 255) // 256 * 256
+    nb = -(-N // b)
+    R = B * H * nb
+    return 256 + 2 * up(R * d * 4) + 2 * up(R * 4) + up(R * min(kmax, nb) * 4)
+
+
+def test_static_route_size_check_follows_the_documented_formula():
+    """Shapes on both sides of the limit: the size check comes before the
+    pointer checks, so a call with NULL buffers is refused for its size
+    (UNSUPPORTED) or, when it fits, for its pointers (INVALID_ARG); nothing
+    reaches the device either way."""
+    L = sp.lib()
+    limit = 32 << 20
+    N, d, b, kmax = 32760, 128, 128, 256
+    for H in range(60, 68):
+        st = L.spattn_route_static(1, H, N, d, b, 0.9, 1, kmax, None, None, None, None, None, None)
+        fits = _scratch_need(1, H, N, d, b, kmax) <= limit
+        assert st == (sp.ERR_INVALID_ARG if fits else sp.ERR_UNSUPPORTED), (H, st)
+    assert _scratch_need(1, 63, N, d, b, kmax) <= limit < _scratch_need(1, 64, N, d, b, kmax)
+
+
+def test_static_route_path_calls_no_device_allocator():
+    """The routing path of spattn_route_static (its own file, the pooling and
+    routing launchers and the shared-memory attribute helper) names no device
+    allocator, so a later edit that adds one fails here."""
+    import os
+    import re
+    csrc = os.path.join(os.path.dirname(sp.__file__), "csrc")
+
+    def code(path):
+        s = open(os.path.join(csrc, path)).read()
+        s = re.sub(r"/\*.*?\*/", "", s, flags=re.S)
+        return re.sub(r"//[^\n]*", "", s)
+
+    api = code("api.cu")
+    start = api.index("cudaError_t ensure_dyn_smem(")
+    helper = api[start:api.index("\n}\n", start)]
+    alloc = re.compile(r"\b(cudaMalloc\w*|cudaFree\w*|cudaHostAlloc|cuMemAlloc\w*|cuMemCreate|"
+                       r"cudaMemPool\w*|cudaMallocAsync)\b")
+    for name, text in (("route_static.cu", code("route_static.cu")), ("pool.cu", code("pool.cu")),
+                       ("route.cu", code("route.cu")), ("api.cu:ensure_dyn_smem", helper)):
+        assert not alloc.findall(text), (name, alloc.findall(text))
