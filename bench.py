@@ -667,6 +667,27 @@ def run_ours(args):
                       "attn_tflops": (t_exact + t_resid) / (t_attend * 1e-3) / 1e12,
                       "unit": "TFLOP/s",
                       "what": "per-block threshold p >= theta in the route kernel, same attention"}
+            # the same threshold selected inside the attention pass: pooling
+            # + attention, no routing launch and no kept lists
+            if routing == sp.ROUTING_CENTROID:
+                fplan = sp.Plan(B, H, N, d, w.b, args.theta, w.kmin, w.kmax, w.residual, perm,
+                                device=dev,
+                                routing=routing | sp.SELECT_THRESHOLD | sp.SELECT_INLINE)
+                n_graphs = len(graphs)
+                tf = timed([as_graph(lambda: fplan.pool(q, k, v)),
+                            as_graph(lambda: fplan.attend(q, k, v, o))], max(3, args.steps // 3), 2)
+                f_pool = float(np.mean([x[0] for x in tf]))
+                f_attend = float(np.mean([x[1] for x in tf]))
+                fstatus = fplan.check()
+                del graphs[n_graphs:]
+                fplan.close()
+                thresh["inline"] = {
+                    "ms_per_step": f_pool + f_attend, "pool_ms": f_pool, "attend_ms": f_attend,
+                    "value": (t_exact + t_resid) / ((f_pool + f_attend) * 1e-3) / 1e12,
+                    "unit": "TFLOP/s", "status": int(fstatus),
+                    "speedup_vs_route_attend": (t_route + t_attend) / (f_pool + f_attend),
+                    "what": "the same threshold selected inside the attention kernel "
+                            "(SPATTN_SELECT_INLINE): pooling + attention, no routing launch"}
         except Exception as ex:   # reported in the line; the measurements above stand
             thresh = {"error": f"{type(ex).__name__}: {ex}"[:300], "theta": args.theta}
 

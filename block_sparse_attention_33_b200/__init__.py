@@ -24,6 +24,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: 
 
 ROUTING_CENTROID, ROUTING_PAMA = 0, 1
 SELECT_THRESHOLD = 16   # OR into routing: tau is the per-block threshold theta on p
+SELECT_INLINE = 32      # OR into routing: the attention kernel selects (no routing launch)
 
 EXPORTS = ("spattn_plan", "spattn_plan_ex", "spattn_plan_destroy", "spattn_plan_info", "spattn_pool",
            "spattn_route", "spattn_attend", "spattn_forward", "spattn_means", "spattn_check",

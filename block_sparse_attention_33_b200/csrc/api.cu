@@ -209,9 +209,11 @@ spattn_status_t spattn_plan_ex(spattn_plan_t* out, int B, int H, int N, int d, i
                                int routing, size_t* workspace_bytes) {
   g_err[0] = 0;
   if (!out) return fail(SPATTN_ERR_INVALID_ARG, "out is NULL");
-  const int estimate = routing & ~SPATTN_SELECT_THRESHOLD;
+  const int estimate = routing & ~(SPATTN_SELECT_THRESHOLD | SPATTN_SELECT_INLINE);
   if (estimate != SPATTN_ROUTING_CENTROID && estimate != SPATTN_ROUTING_PAMA)
-    return fail(SPATTN_ERR_INVALID_ARG, "routing must be SPATTN_ROUTING_CENTROID or SPATTN_ROUTING_PAMA, optionally | SPATTN_SELECT_THRESHOLD (got %d)", routing);
+    return fail(SPATTN_ERR_INVALID_ARG, "routing must be SPATTN_ROUTING_CENTROID or SPATTN_ROUTING_PAMA, optionally | SPATTN_SELECT_THRESHOLD | SPATTN_SELECT_INLINE (got %d)", routing);
+  if ((routing & SPATTN_SELECT_INLINE) && estimate != SPATTN_ROUTING_CENTROID)
+    return fail(SPATTN_ERR_INVALID_ARG, "routing: SPATTN_SELECT_INLINE needs the centroid estimate");
   *out = nullptr;
   if (B < 1 || H < 1 || N < 1) return fail(SPATTN_ERR_INVALID_ARG, "need B, H, N >= 1 (got %d, %d, %d)", B, H, N);
   if (d != 64 && d != 128) return fail(SPATTN_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
@@ -250,12 +252,15 @@ spattn_status_t spattn_plan_ex(spattn_plan_t* out, int B, int H, int N, int d, i
   p.perm = nullptr;
   p.routing = estimate == SPATTN_ROUTING_PAMA ? spattn::ROUTING_PAMA : spattn::ROUTING_CENTROID;
   p.threshold = (routing & SPATTN_SELECT_THRESHOLD) ? 1 : 0;
+  p.inline_sel = (routing & SPATTN_SELECT_INLINE) ? 1 : 0;
   {
-    // tcgen05/TMEM kernel for 128-token blocks; the warp-MMA kernel serves
-    // b = 64 and, with SPATTN_ATTN=mma in the environment when the plan is
-    // made, any shape (used to cross-check the two GPU paths).
+    // tcgen05/TMEM kernel for every supported shape; with SPATTN_ATTN=mma in
+    // the environment when the plan is made, the warp-MMA kernel instead
+    // (kept only to cross-check the two GPU paths in the tests).
     const char* env = getenv("SPATTN_ATTN");
     p.use_tc = spattn::attend_tc_supported(p) && !(env && strcmp(env, "mma") == 0);
+    // the inline selection lives in the tcgen05 kernel
+    if (p.inline_sel && !p.use_tc) { delete P; return fail(SPATTN_ERR_UNSUPPORTED, "SPATTN_SELECT_INLINE needs the tcgen05 attention kernel"); }
     // Failure-path test: with SPATTN_TEST_WAIT_TIMEOUT=1 in the environment
     // when the plan is made, the tcgen05 attention's first CTA waits on an
     // mbarrier phase that nothing completes; the bounded wait gives up after
@@ -346,7 +351,13 @@ spattn_status_t spattn_attend(spattn_plan_t plan, const void* Q, const void* K, 
 spattn_status_t spattn_forward(spattn_plan_t plan, const void* Q, const void* K, const void* V,
                                void* O, void* workspace, void* stream) {
   Range range("spattn_forward");
-  if (spattn_status_t st = spattn_route(plan, Q, K, V, workspace, nullptr, nullptr, stream)) return st;
+  // with inline selection the attention kernel selects from the means: no
+  // routing launch
+  if (plan && plan->p.inline_sel) {
+    if (spattn_status_t st = spattn_pool(plan, Q, K, V, workspace, stream)) return st;
+  } else if (spattn_status_t st = spattn_route(plan, Q, K, V, workspace, nullptr, nullptr, stream)) {
+    return st;
+  }
   return spattn_attend(plan, Q, K, V, nullptr, nullptr, O, workspace, stream);
 }
 
@@ -420,7 +431,7 @@ spattn_status_t spattn_forward_host(spattn_plan_t plan, const void* Q_host, cons
     void* o = slot_buf(slot, 3);
     what = "pool kernel";
     e = spattn::launch_pool(ps, q, k, v, w, s0);
-    if (e == cudaSuccess) { what = "route kernels"; e = spattn::launch_route(ps, w, q, nullptr, nullptr, !ps.use_tc, s0); }
+    if (e == cudaSuccess && !ps.inline_sel) { what = "route kernels"; e = spattn::launch_route(ps, w, q, nullptr, nullptr, !ps.use_tc, s0); }
     if (e == cudaSuccess) { what = "attention kernel"; e = spattn::launch_attend(ps, q, k, v, w.row_ptr, w.col_idx, o, w, s0); }
     if (e == cudaSuccess && w.ctrl != ctrl) {
       what = "error merge";

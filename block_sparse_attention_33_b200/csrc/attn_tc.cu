@@ -35,6 +35,15 @@
 //              TMEM, V from shared memory), tcgen05.mma with fp32
 //              accumulation in TMEM.
 //
+// 64-token blocks use the same 128-row tiles: an item is the pair of query
+// blocks 2i and 2i + 1 (rows 0-63 and 64-127 of the Q tile), and its key
+// tiles walk the union of the two kept sets in ascending order, two blocks
+// per tile (two 64-row TMA boxes).  The softmax warps of lane quarters 0-1
+// belong to the first query block, those of quarters 2-3 to the second, and
+// each key half holds one key block, so a warp masks a whole half when its
+// query block did not keep that key block; the residual bias of a warp
+// likewise follows its own query block's kept set.
+//
 // Tasks of an item: its kept key blocks (one online-softmax sweep over the
 // selected blocks, as in the Sol-Attn abstract), then, in residual mode,
 // every 128-row tile of the bf16 block centroids Kbar/Vbar that holds a
@@ -53,6 +62,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "select.cuh"
 #include "tc.cuh"
 
 namespace spattn {
@@ -102,9 +112,23 @@ struct TcArgs {
   // (counts[item] entries at col_idx + item * kcap)
   const int32_t *row_ptr, *col_idx, *counts, *order, *perm;
   int kcap;
-  __nv_bfloat16* o;
+  __nv_bfloat16* o;           // bf16 output [BH, q_rows, D], scattered through perm
+  float* o32;                 // or, when set, fp32 output [BH, q_rows, D] in tile order
+  int q_rows;                 // query (and output) rows per (batch, head)
+  int dense;                  // every key tile of the N keys, no residual (exact rows)
   int32_t* ctrl;
   int N, nb, n_last, residual, items;
+  // inline selection (Sol-Attn abstract: blocks chosen inside the attention
+  // pass, no stored proxy map and no routing launch): the producer scores
+  // each query block against every key block from the fp32 means and cuts
+  // the row itself, with the routing kernel's arithmetic
+  int inline_sel;
+  const float *qbar, *kbar;  // fp32 means [BH, nb, d]
+  float tau;                 // Top-p mass, or the per-block threshold theta
+  int threshold, kmin;
+  int b64;         // 64-token blocks: a tile holds two query (key) blocks
+  int nq;          // query tiles per (batch, head): nb (b = 128) or ceil(nb / 2) (b = 64)
+  int blk;         // block size b
   int test_stall;  // failure-path test (see Problem::test_stall)
   float sl2;       // log2(e) / sqrt(d)
 };
@@ -113,13 +137,17 @@ struct TcArgs {
 // builds item n+1 (and starts its loads) while item n is still in the
 // softmax and epilogue.
 struct ItemInfo {
-  int item;            // bh * nb + i; -1 once the work is exhausted
-  int nkept;           // kept key blocks (CSR row length)
-  int T;               // tasks: the kept blocks, then residual centroid tiles
-  int tail_task;       // task index of the partial last key block, -1 if none
+  int item;            // bh * nq + query tile; -1 once the work is exhausted
+  int nkept;           // key-tile tasks (b = 128: the CSR row length)
+  int T;               // tasks: the key tiles, then residual centroid tiles
+  int tail_task;       // b = 128: task index of the partial last key block, -1 if none
+  int nunion;          // b = 64: blocks kept by either query block of the tile
   uint32_t res_tiles;  // bit c: centroid tile c holds a dropped block
-  uint32_t kept[64];   // kept-block bitmap (nb <= 2048)
-  uint32_t bad[64];    // tasks whose CSR block index is out of range (caller CSR)
+  uint32_t kept[2][64];  // kept-block bitmaps (nb <= 2048) of the tile's query block(s):
+                         // [1] is the second query block with b = 64
+  uint32_t bad[64];    // b = 128: tasks whose CSR block index is out of range (caller CSR)
+  uint16_t ublk[2048]; // b = 64: the union of both kept sets, ascending; key tile t
+                       // holds blocks ublk[2t] (rows 0-63) and ublk[2t + 1] (rows 64-127)
 };
 
 struct __align__(8) TcCtrl {
@@ -127,9 +155,63 @@ struct __align__(8) TcCtrl {
   uint32_t tmem_base;
   int abort;
   ItemInfo info[2];
+  float selp[2048];           // inline selection: the proxy / probability row
+  float selq[128];            // inline selection: the query block's mean
   float xm[2][2][TILE_ROWS];  // epilogue, per item slot: reference max of each key half
   float xl[2][2][TILE_ROWS];  // epilogue, per item slot: sum of each key half
 };
+
+// Inline selection of query row `row` (bh * nb + query block) into the kept
+// bitmap km (one whole warp; selp and selq are shared-memory scratch): the
+// centroid proxy logits against every key block, split over the lanes
+// exactly as the routing kernel splits them, the block softmax and the cut.
+// Kept out of line so that its registers do not add to the softmax warps'.
+struct SelArgs {
+  const float *qbar, *kbar;
+  int nb, n_last, blk, threshold, kmin, kcap;
+  float tau;
+};
+
+template <int D>
+__device__ __noinline__ void select_inline(const SelArgs a, int row, uint32_t* km, float* selp,
+                                           float* selq) {
+  const int lane = threadIdx.x & 31;
+  const float4* qrow = reinterpret_cast<const float4*>(a.qbar + (size_t)row * D);
+  for (int c4 = lane; c4 < D / 4; c4 += 32) reinterpret_cast<float4*>(selq)[c4] = __ldg(qrow + c4);
+  __syncwarp();
+  const float* kb = a.kbar + (size_t)(row / a.nb) * a.nb * D;
+  const float inv_sqrt_d = 1.0f / sqrtf((float)D);
+  const int tpj = sel::proxy_threads_per_block(a.nb);
+  const int sub = lane % tpj, grp = lane / tpj, ngrp = 32 / tpj;
+  for (int j0 = 0; j0 < a.nb; j0 += ngrp) {
+    const int j = j0 + grp;
+    const bool live = j < a.nb;
+    float acc = 0.f;
+    if (live) {
+      const float4* kr = reinterpret_cast<const float4*>(kb + (size_t)j * D);
+      for (int k4 = sub; k4 < D / 4; k4 += tpj) {
+        const float4 kv = __ldg(kr + k4);
+        const float4 q = reinterpret_cast<const float4*>(selq)[k4];
+        acc = fmaf(q.x, kv.x, acc);
+        acc = fmaf(q.y, kv.y, acc);
+        acc = fmaf(q.z, kv.z, acc);
+        acc = fmaf(q.w, kv.w, acc);
+      }
+    }
+    for (int o = 1; o < tpj; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (live && sub == 0) {
+      const int nj = (j == a.nb - 1) ? a.n_last : a.blk;
+      selp[j] = fmaf(acc, inv_sqrt_d, logf((float)nj));
+    }
+  }
+  __syncwarp();
+  sel::softmax_row(selp, a.nb);
+  const sel::Cut c = sel::cut_row(selp, a.nb, a.tau, a.threshold, a.kmin, a.kcap);
+  sel::walk_kept(selp, a.nb, c, [&](int j0, bool, unsigned w) {
+    if (lane == 0) km[j0 >> 5] = w;
+  });
+  __syncwarp();
+}
 
 template <int D>
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -212,26 +294,86 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       const int item = a.order ? __ldg(a.order + ticket) : ticket;
-      const int bh = item / a.nb, i = item % a.nb;
-      const int r_lo = a.counts ? item * a.kcap : __ldg(a.row_ptr + item);
-      const int nkept = a.counts ? __ldg(a.counts + item) : max(0, __ldg(a.row_ptr + item + 1) - r_lo);
-      inf.kept[lane] = 0u;
-      inf.kept[lane + 32] = 0u;
+      const int bh = item / a.nq, i = item % a.nq;
+      int r_lo = 0, nkept = 0;
+      inf.kept[0][lane] = 0u;
+      inf.kept[0][lane + 32] = 0u;
+      inf.kept[1][lane] = 0u;
+      inf.kept[1][lane + 32] = 0u;
       inf.bad[lane] = 0u;
       inf.bad[lane + 32] = 0u;
       if (lane == 0) inf.tail_task = -1;
       __syncwarp();
-      for (int t = lane; t < nkept; t += 32) {
-        const int j = __ldg(a.col_idx + r_lo + t);
-        if (j >= 0 && j < a.nb) {
-          atomicOr(&inf.kept[j >> 5], 1u << (j & 31));
-          if (j == a.nb - 1 && a.n_last < TILE_ROWS) inf.tail_task = t;
-        } else if (t < 2048) {
-          atomicOr(&inf.bad[t >> 5], 1u << (t & 31));
+      const bool pair2 = a.b64 && 2 * i + 1 < a.nb;   // the tile holds a second query block
+      if (a.dense) {
+        // exact rows: every key tile, in order
+        nkept = a.nb;
+        if (lane == 0 && a.n_last < TILE_ROWS) inf.tail_task = a.nb - 1;
+        __syncwarp();
+      } else if (a.inline_sel) {
+        const SelArgs sa{a.qbar, a.kbar, a.nb, a.n_last, a.blk, a.threshold, a.kmin, a.kcap, a.tau};
+        select_inline<D>(sa, a.b64 ? bh * a.nb + 2 * i : item, inf.kept[0], cs->selp, cs->selq);
+        if (pair2) select_inline<D>(sa, bh * a.nb + 2 * i + 1, inf.kept[1], cs->selp, cs->selq);
+      } else if (!a.b64) {
+        r_lo = a.counts ? item * a.kcap : __ldg(a.row_ptr + item);
+        nkept = a.counts ? __ldg(a.counts + item) : max(0, __ldg(a.row_ptr + item + 1) - r_lo);
+        for (int t = lane; t < nkept; t += 32) {
+          const int j = __ldg(a.col_idx + r_lo + t);
+          if (j >= 0 && j < a.nb) {
+            atomicOr(&inf.kept[0][j >> 5], 1u << (j & 31));
+            if (j == a.nb - 1 && a.n_last < TILE_ROWS) inf.tail_task = t;
+          } else if (t < 2048) {
+            atomicOr(&inf.bad[t >> 5], 1u << (t & 31));
+          }
         }
+        __syncwarp();
+      } else {
+        // 64-token blocks: query blocks 2i and 2i + 1 share the tile; their
+        // kept sets go into two bitmaps (a block index out of range is
+        // skipped and flagged), and the key tiles walk the union in
+        // ascending order, two blocks per tile
+        for (int qb = 0; qb < (pair2 ? 2 : 1); ++qb) {
+          const int row = bh * a.nb + 2 * i + qb;
+          const int lo = a.counts ? row * a.kcap : __ldg(a.row_ptr + row);
+          const int nk = a.counts ? __ldg(a.counts + row) : max(0, __ldg(a.row_ptr + row + 1) - lo);
+          uint32_t* km = inf.kept[qb];
+          for (int t = lane; t < nk; t += 32) {
+            const int j = __ldg(a.col_idx + lo + t);
+            if (j >= 0 && j < a.nb) atomicOr(&km[j >> 5], 1u << (j & 31));
+            else flag_error(a.ctrl, DEV_BAD_INDEX, row);
+          }
+        }
+        __syncwarp();
       }
-      __syncwarp();
-      // centroid tiles that hold at least one dropped block
+      if (a.b64 || a.inline_sel) {
+        // the kept blocks (the union of both bitmaps with b = 64) as an
+        // ascending list
+        const uint32_t w0 = inf.kept[0][2 * lane] | inf.kept[1][2 * lane];
+        const uint32_t w1 = inf.kept[0][2 * lane + 1] | inf.kept[1][2 * lane + 1];
+        const int c = __popc(w0) + __popc(w1);
+        int x = c;   // inclusive scan of the per-lane counts
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        int pos = x - c;
+        for (uint32_t m = w0; m; m &= m - 1u) inf.ublk[pos++] = (uint16_t)(64 * lane + __ffs(m) - 1);
+        for (uint32_t m = w1; m; m &= m - 1u) inf.ublk[pos++] = (uint16_t)(64 * lane + 32 + __ffs(m) - 1);
+        const int nunion = __shfl_sync(0xffffffffu, x, 31);
+        if (a.b64) {
+          nkept = (nunion + 1) / 2;
+        } else {
+          nkept = nunion;
+          // the partial last block, when kept, is the last entry
+          if (lane == 0 && a.n_last < TILE_ROWS && ((inf.kept[0][(a.nb - 1) >> 5] >> ((a.nb - 1) & 31)) & 1u))
+            inf.tail_task = nunion - 1;
+        }
+        if (lane == 0) inf.nunion = nunion;
+        __syncwarp();
+      }
+      // centroid tiles that hold at least one dropped block (of either query
+      // block of the tile, with b = 64)
       bool any = false;
       if (a.residual && lane < ntiles) {
         for (int q = 0; q < TILE_ROWS / 32; ++q) {
@@ -239,7 +381,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (j0 >= a.nb) break;
           const int cnt = min(32, a.nb - j0);
           const uint32_t valid = cnt == 32 ? 0xffffffffu : ((1u << cnt) - 1u);
-          any |= (~inf.kept[j0 >> 5] & valid) != 0u;
+          any |= (~inf.kept[0][j0 >> 5] & valid) != 0u;
+          if (pair2) any |= (~inf.kept[1][j0 >> 5] & valid) != 0u;
         }
       }
       const uint32_t res_tiles = __ballot_sync(0xffffffffu, any);
@@ -264,15 +407,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         auto issue = [&](int t, bool is_v) -> bool {
           const CUtensorMap* m;
-          int row;
+          int row, row2 = -1;   // row2: b = 64, first token of the tile's second key block
           if (t < nkept) {
-            int j = __ldg(a.col_idx + r_lo + t);
-            if (j < 0 || j >= a.nb) {
-              flag_error(a.ctrl, DEV_BAD_INDEX, item);
-              j = 0;  // load something valid; the softmax masks the whole task
-            }
             m = is_v ? &tmV : &tmK;
-            row = j * TILE_ROWS;
+            if (a.b64) {
+              // an absent second block repeats the first (valid data, masked
+              // by the softmax)
+              const int j0 = inf.ublk[2 * t];
+              const int j1 = 2 * t + 1 < inf.nunion ? inf.ublk[2 * t + 1] : j0;
+              row = j0 * 64;
+              row2 = j1 * 64;
+            } else if (a.dense) {
+              row = t * TILE_ROWS;
+            } else if (a.inline_sel) {
+              row = inf.ublk[t] * TILE_ROWS;
+            } else {
+              int j = __ldg(a.col_idx + r_lo + t);
+              if (j < 0 || j >= a.nb) {
+                flag_error(a.ctrl, DEV_BAD_INDEX, item);
+                j = 0;  // load something valid; the softmax masks the whole task
+              }
+              row = j * TILE_ROWS;
+            }
           } else {
             m = is_v ? &tmVb : &tmKb;
             row = res_tile(res_tiles, t - nkept) * TILE_ROWS;
@@ -282,8 +438,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             return false;
           tc::mbar_expect_tx(full(s), TILE_BYTES);
           const uint32_t dst = sRing + s * TILE_BYTES;
+          if (row2 < 0) {
 #pragma unroll
-          for (int c = 0; c < NCH; ++c) tc::tma_load_3d(dst + c * CHUNK_BYTES, m, full(s), c * 64, row, bh);
+            for (int c = 0; c < NCH; ++c) tc::tma_load_3d(dst + c * CHUNK_BYTES, m, full(s), c * 64, row, bh);
+          } else {
+            // two 64-row boxes: rows 0-63 and 64-127 of every 128-byte chunk
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+              tc::tma_load_3d(dst + c * CHUNK_BYTES, m, full(s), c * 64, row, bh);
+              tc::tma_load_3d(dst + c * CHUNK_BYTES + 64 * 128, m, full(s), c * 64, row2, bh);
+            }
+          }
           ++li;
           return true;
         };
@@ -406,7 +571,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int r = quarter * 32 + lane;                 // row / TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tOh = tmem + lane_off + COL_O + 128u * (uint32_t)half;  // this half's O
-    const float lg_b = log2f((float)TILE_ROWS), lg_last = log2f((float)a.n_last);
+    const float lg_b = log2f((float)a.blk), lg_last = log2f((float)a.n_last);
+    // b = 64: rows 0-63 of a tile are the first query block, rows 64-127 the
+    // second, so lane quarters 2 and 3 test the second block's kept set
+    const int qsel = a.b64 ? (quarter >> 1) : 0;
     int n = 0, qn = 0, gt = 0;  // items, items with tasks, tasks before this item
     bool ok = true;
 
@@ -430,8 +598,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (item < 0) break;
       const int T = inf.T, nkept = inf.nkept, tail_task = inf.tail_task;
       const uint32_t res_tiles = inf.res_tiles;
-      const int bh = item / a.nb, i = item % a.nb;
-      const int rows_valid = (i == a.nb - 1) ? a.n_last : TILE_ROWS;
+      const int bh = item / a.nq, i = item % a.nq;
       // m: reference maximum of this row's key half (log2 units); l: sum of
       // p at that reference; owe: factor O_h owes once PV(g-1) is done.
       float m = -INFINITY, l = 0.f, owe = 1.f;
@@ -445,30 +612,50 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (!(ok = wait_warp(bar(B_SFULL0 + b), (uint32_t)(g >> 1) & 1u, 7))) break;
         tc::tc_fence_after();
         // this warp's 64 columns of S(g).  Key tiles: columns past n_j of the
-        // partial last block (or a whole tile with a bad index) are set to
-        // -inf.  Centroid tiles: the log2-scaled logit plus the bias log2 n_j
-        // (dropped) / -inf (kept) is formed up front.
+        // partial last block (or a whole tile with a bad index; with b = 64,
+        // a whole half whose block this warp's query block did not keep) are
+        // set to -inf.  Centroid tiles: the log2-scaled logit plus the bias
+        // log2 n_j (dropped) / -inf (kept) is formed up front.
         uint32_t u[64];
         const uint32_t scol = tmem + lane_off + 128u * (uint32_t)b + 64u * (uint32_t)half;
         const float scale = t < nkept ? a.sl2 : 1.f;
+        // the task's mask, looked up before S is loaded (fewer live registers
+        // next to S): key tiles, the count of valid columns of this half;
+        // centroid tiles, the first block of this half and the kept bits of
+        // its 64 blocks
+        int nvalid = 64, jres = 0;
+        uint32_t kw0 = 0u, kw1 = 0u;
+        if (t < nkept) {
+          if (a.b64) {
+            const int e = 2 * t + half;
+            const int j = e < inf.nunion ? (int)inf.ublk[e] : -1;
+            const bool mine = j >= 0 && ((inf.kept[qsel][j >> 5] >> (j & 31)) & 1u);
+            nvalid = mine ? (j == a.nb - 1 ? a.n_last : 64) : 0;
+          } else {
+            const bool bad = t < 2048 && ((inf.bad[t >> 5] >> (t & 31)) & 1u);
+            nvalid = (bad ? 0 : (t == tail_task ? a.n_last : TILE_ROWS)) - 64 * half;
+          }
+        } else {
+          jres = res_tile(res_tiles, t - nkept) * TILE_ROWS + 64 * half;
+          if (jres < a.nb) kw0 = inf.kept[qsel][jres >> 5];
+          if (jres + 32 < a.nb) kw1 = inf.kept[qsel][(jres >> 5) + 1];
+        }
         auto load_s = [&]() {
           tc::tmem_ld32(scol, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
           tc::tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
           tc::tmem_wait_ld();
           if (t < nkept) {
-            const bool bad = t < 2048 && ((inf.bad[t >> 5] >> (t & 31)) & 1u);
-            const int nvalid = (bad ? 0 : (t == tail_task ? a.n_last : TILE_ROWS)) - 64 * half;
             if (nvalid < 64) {
 #pragma unroll
               for (int c = 0; c < 64; ++c)
                 if (c >= nvalid) u[c] = __float_as_uint(-INFINITY);
             }
           } else {
-            const int jres = res_tile(res_tiles, t - nkept) * TILE_ROWS + 64 * half;
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
               const int j = jres + c;
-              const bool dropped = j < a.nb && !((inf.kept[j >> 5] >> (j & 31)) & 1u);
+              const uint32_t kw = c < 32 ? kw0 : kw1;
+              const bool dropped = j < a.nb && !((kw >> (c & 31)) & 1u);
               const float bias = dropped ? (j == a.nb - 1 ? lg_last : lg_b) : -INFINITY;
               u[c] = __float_as_uint(fmaf(__uint_as_float(u[c]), a.sl2, bias));
             }
@@ -589,9 +776,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const float a1 = m1 == -INFINITY ? 0.f : tc::ex2(m1 - M);
         const float L = a0 * cs->xl[slot][0][r] + a1 * cs->xl[slot][1][r];
         const int tok = i * TILE_ROWS + r;
-        const bool store = r < rows_valid;
+        const bool store = tok < a.q_rows;   // rows past the last query are padding
         const int dst = store ? (a.perm ? __ldg(a.perm + tok) : tok) : 0;
-        uint4* orow = reinterpret_cast<uint4*>(a.o + ((size_t)bh * a.N + dst) * D + half * (D / 2));
+        const size_t obase = ((size_t)bh * a.q_rows + dst) * D + half * (D / 2);
         const float inv = L > 0.f ? 1.f / L : 0.f;
         const float w0 = a0 * inv, w1 = a1 * inv;
 #pragma unroll
@@ -613,12 +800,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
               for (int e = 0; e < 8; ++e)
                 v[e] = __uint_as_float(o0[8 * q + e]) * w0 + __uint_as_float(o1[8 * q + e]) * w1;
-              uint4 pv;
-              pv.x = pack_bf16x2(v[0], v[1]);
-              pv.y = pack_bf16x2(v[2], v[3]);
-              pv.z = pack_bf16x2(v[4], v[5]);
-              pv.w = pack_bf16x2(v[6], v[7]);
-              orow[c * 4 + q] = pv;
+              if (a.o32) {
+                float4* orow32 = reinterpret_cast<float4*>(a.o32 + obase);
+                orow32[c * 8 + 2 * q] = make_float4(v[0], v[1], v[2], v[3]);
+                orow32[c * 8 + 2 * q + 1] = make_float4(v[4], v[5], v[6], v[7]);
+              } else {
+                uint4 pv;
+                pv.x = pack_bf16x2(v[0], v[1]);
+                pv.y = pack_bf16x2(v[2], v[3]);
+                pv.z = pack_bf16x2(v[4], v[5]);
+                pv.w = pack_bf16x2(v[6], v[7]);
+                reinterpret_cast<uint4*>(a.o + obase)[c * 4 + q] = pv;
+              }
             }
           }
         }
@@ -660,25 +853,26 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [BH, rows, D] bf16 tensor, box = 64 channels x 128 rows x 1, 128-byte swizzle.
-bool encode_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH) {
+// [BH, rows, D] bf16 tensor, box = 64 channels x box_rows rows x 1, 128-byte
+// swizzle.
+bool encode_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)TILE_ROWS, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// A tensor map depends only on (pointer, D, rows, BH): the last few encoded
-// maps of each host thread are kept so repeated calls on the same buffers
-// skip the driver's encode.
+// A tensor map depends only on (pointer, D, rows, BH, box rows): the last few
+// encoded maps of each host thread are kept so repeated calls on the same
+// buffers skip the driver's encode.
 struct MapKey {
   const void* ptr;
-  int D, rows, BH;
+  int D, rows, BH, box;
 };
 struct MapEntry {
   MapKey k;
@@ -686,30 +880,34 @@ struct MapEntry {
   bool used;
 };
 
-bool make_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH) {
+bool make_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH, int box = TILE_ROWS) {
   constexpr int SLOTS = 16;
   thread_local MapEntry cache[SLOTS] = {};
   thread_local int next = 0;
   for (int c = 0; c < SLOTS; ++c) {
     const MapEntry& e = cache[c];
-    if (e.used && e.k.ptr == ptr && e.k.D == D && e.k.rows == rows && e.k.BH == BH) {
+    if (e.used && e.k.ptr == ptr && e.k.D == D && e.k.rows == rows && e.k.BH == BH &&
+        e.k.box == box) {
       *m = e.m;
       return true;
     }
   }
-  if (!encode_map(m, ptr, D, rows, BH)) return false;
+  if (!encode_map(m, ptr, D, rows, BH, box)) return false;
   MapEntry& e = cache[next];
   next = (next + 1) % SLOTS;
-  e.k = MapKey{ptr, D, rows, BH};
+  e.k = MapKey{ptr, D, rows, BH, box};
   e.m = *m;
   e.used = true;
   return true;
 }
 
 template <int D>
-size_t tc_smem_bytes() {
+constexpr size_t tc_smem_bytes() {
   return (size_t)(1 + TcCfg<D>::STAGES) * TcCfg<D>::TILE_BYTES + sizeof(TcCtrl) + 1024;
 }
+// 227 KB of shared memory per CTA at most
+static_assert(tc_smem_bytes<128>() <= 232448 && tc_smem_bytes<64>() <= 232448,
+              "attention tiles and control block exceed the shared memory of one CTA");
 
 template <int D>
 cudaError_t launch_tc(const CUtensorMap* maps, const TcArgs& a, cudaStream_t s) {
@@ -728,7 +926,9 @@ cudaError_t launch_tc(const CUtensorMap* maps, const TcArgs& a, cudaStream_t s) 
 
 }  // namespace
 
-bool attend_tc_supported(const Problem& p) { return p.b == TILE_ROWS && (p.d == 64 || p.d == 128); }
+bool attend_tc_supported(const Problem& p) {
+  return (p.b == TILE_ROWS || p.b == TILE_ROWS / 2) && (p.d == 64 || p.d == 128);
+}
 
 cudaError_t launch_attend_tc(const Problem& p, const void* Q, const void* K, const void* V,
                              const int32_t* row_ptr, const int32_t* col_idx, void* O,
@@ -736,26 +936,44 @@ cudaError_t launch_attend_tc(const Problem& p, const void* Q, const void* K, con
   const void* q = w.qp ? (const void*)w.qp : Q;
   const void* k = w.kp ? (const void*)w.kp : K;
   const void* v = w.vp ? (const void*)w.vp : V;
+  // K and V tiles: one 128-row box, or two 64-row boxes (one per block) with
+  // 64-token blocks
+  const bool b64 = p.b == TILE_ROWS / 2;
   CUtensorMap maps[5];
-  if (!make_map(&maps[0], q, p.d, p.N, p.BH) || !make_map(&maps[1], k, p.d, p.N, p.BH) ||
-      !make_map(&maps[2], v, p.d, p.N, p.BH) || !make_map(&maps[3], w.kbar16, p.d, p.nb, p.BH) ||
+  if (!make_map(&maps[0], q, p.d, p.N, p.BH) || !make_map(&maps[1], k, p.d, p.N, p.BH, p.b) ||
+      !make_map(&maps[2], v, p.d, p.N, p.BH, p.b) || !make_map(&maps[3], w.kbar16, p.d, p.nb, p.BH) ||
       !make_map(&maps[4], w.vbar16, p.d, p.nb, p.BH))
     return cudaErrorInvalidValue;
   TcArgs a;
-  if (row_ptr == w.row_ptr) {
+  a.inline_sel = (row_ptr == w.row_ptr && p.inline_sel) ? 1 : 0;
+  a.qbar = w.qbar; a.kbar = w.kbar;
+  a.tau = p.tau; a.threshold = p.threshold; a.kmin = p.kmin;
+  if (a.inline_sel) {
+    // the producer selects from the workspace means: no lists, plain order
+    a.row_ptr = nullptr; a.col_idx = nullptr; a.counts = nullptr; a.kcap = p.kcap;
+    a.order = nullptr;
+  } else if (row_ptr == w.row_ptr) {
     // the workspace's own routing result: padded lists, longest-first order
+    // (the order is per query block: with 64-token blocks the tiles run in
+    // plain order)
     a.row_ptr = nullptr; a.col_idx = w.lists; a.counts = w.counts; a.kcap = p.kcap;
-    a.order = w.order;
+    a.order = b64 ? nullptr : w.order;
   } else {
     a.row_ptr = row_ptr; a.col_idx = col_idx; a.counts = nullptr; a.kcap = 0;
     a.order = nullptr;
   }
   a.perm = p.perm;
   a.o = static_cast<__nv_bfloat16*>(O);
+  a.o32 = nullptr;
+  a.q_rows = p.N;
+  a.dense = 0;
   a.ctrl = w.ctrl;
   a.N = p.N; a.nb = p.nb; a.n_last = p.n_last; a.residual = p.residual;
+  a.b64 = b64 ? 1 : 0;
+  a.blk = p.b;
+  a.nq = b64 ? (p.nb + 1) / 2 : p.nb;
   a.sl2 = 1.4426950408889634f / sqrtf((float)p.d);
-  a.items = p.BH * p.nb;
+  a.items = p.BH * a.nq;
   a.test_stall = p.test_stall;
   // The work counter resets itself at the end of every launch; it starts
   // from zero after the routing call's control-block clear.  A caller CSR
@@ -767,6 +985,36 @@ cudaError_t launch_attend_tc(const Problem& p, const void* Q, const void* K, con
     cudaError_t e = cudaMemsetAsync(w.ctrl, 0, 4 * sizeof(int32_t), s);
     if (e != cudaSuccess) return e;
   }
+  return p.d == 128 ? launch_tc<128>(maps, a, s) : launch_tc<64>(maps, a, s);
+}
+
+// Exact (dense) softmax attention of gathered query rows, fp32 out: Qg holds
+// q_alloc rows per (batch, head) (a multiple of 128, zero past q_rows), every
+// one of the N keys of K and V is attended, and rows [0, q_rows) of each head
+// are written to out [BH, q_rows, d].  The probe correction's exact rows.
+cudaError_t launch_dense_rows_tc(const Problem& p, const void* Qg, int q_alloc, int q_rows,
+                                 const void* K, const void* V, float* out, int32_t* ctrl,
+                                 cudaStream_t s) {
+  const int nb = (p.N + TILE_ROWS - 1) / TILE_ROWS;
+  CUtensorMap maps[5];
+  if (!make_map(&maps[0], Qg, p.d, q_alloc, p.BH) || !make_map(&maps[1], K, p.d, p.N, p.BH) ||
+      !make_map(&maps[2], V, p.d, p.N, p.BH))
+    return cudaErrorInvalidValue;
+  maps[3] = maps[1];   // no residual tiles: the centroid maps are never read
+  maps[4] = maps[2];
+  TcArgs a{};
+  a.dense = 1;
+  a.o = nullptr;
+  a.o32 = out;
+  a.q_rows = q_rows;
+  a.ctrl = ctrl;
+  a.N = p.N; a.nb = nb; a.n_last = p.N - (nb - 1) * TILE_ROWS; a.residual = 0;
+  a.b64 = 0;
+  a.blk = TILE_ROWS;
+  a.nq = q_alloc / TILE_ROWS;
+  a.kcap = nb;
+  a.sl2 = 1.4426950408889634f / sqrtf((float)p.d);
+  a.items = p.BH * a.nq;
   return p.d == 128 ? launch_tc<128>(maps, a, s) : launch_tc<64>(maps, a, s);
 }
 

@@ -24,6 +24,7 @@ struct Problem {
   int use_tc;           // attention on the tcgen05 kernel (else warp MMA)
   int routing;          // ROUTING_CENTROID or ROUTING_PAMA
   int threshold;        // selection: 0 Top-p (tau = mass), 1 per-block p >= tau
+  int inline_sel;       // 1: the attention kernel selects (no routing launch)
   int test_stall;       // failure-path test: CTA 0 of the attention waits on a phase
                         // that never completes, so its bounded wait runs out
   const int32_t* perm;  // device, NULL if none
@@ -53,6 +54,13 @@ cudaError_t launch_route(const Problem& p, const Work& w, const void* Q, int32_t
 cudaError_t launch_attend(const Problem& p, const void* Q, const void* K, const void* V,
                           const int32_t* row_ptr, const int32_t* col_idx, void* O,
                           const Work& w, cudaStream_t s);
+
+// Exact softmax attention of gathered query rows (Qg: [BH, q_alloc, d] bf16,
+// q_alloc a multiple of 128) over all N keys of K and V, fp32 output rows
+// [BH, q_rows, d]; the tcgen05 attention kernel in its dense mode.
+cudaError_t launch_dense_rows_tc(const Problem& p, const void* Qg, int q_alloc, int q_rows,
+                                 const void* K, const void* V, float* out, int32_t* ctrl,
+                                 cudaStream_t s);
 
 // Probe-fitted residual correction (SparsePR page, section 2B) of the routed
 // output O in place; scratch of probe_scratch_bytes(p, M) bytes.

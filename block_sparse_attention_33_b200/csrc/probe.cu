@@ -9,9 +9,11 @@
 //
 // One head at a time (every (batch, head) pair is its own attention call):
 //
-//   probe_dense_kernel  exact softmax attention of the M probe rows over all
-//                       N keys, fp32 (one warp per row, K/V tiles of 64 keys
-//                       staged in shared memory, online softmax in base 2);
+//   probe_gather_kernel the probe queries into whole 128-row tiles, then the
+//                       tcgen05 attention kernel in its dense mode: exact
+//                       softmax attention of those rows over all N keys, fp32
+//                       output (bf16 operands, fp32 accumulation, as every
+//                       attention row of this library);
 //   probe_fit_kernel    normal equations of the ridge fit on [1, x]:
 //                       G = A^T A + lam * diag(0, 1, ..., 1), C = A^T R, then
 //                       a Cholesky factorisation of G and two triangular
@@ -36,8 +38,6 @@ namespace spattn {
 namespace {
 
 constexpr int PB_THREADS = 256;
-constexpr int PD_ROWS = PB_THREADS / 32;   // probe rows per dense CTA (one per warp)
-constexpr int PD_KEYS = 64;                // keys per staged tile
 constexpr int PF_CHUNK = 32;               // probe rows per accumulation chunk
 constexpr int PA_ROWS = 64;                // output rows per apply CTA
 constexpr int JACOBI_MAX_SWEEPS = 16;
@@ -72,76 +72,28 @@ __device__ __forceinline__ int probe_token(const ProbeArgs& a, int bh, int m) {
 }
 
 // ---- exact rows ------------------------------------------------------------
+// The probe queries are gathered into a [BH, Mpad, D] bf16 buffer (rows past M
+// zero); the tcgen05 attention kernel then runs them as dense query tiles over
+// all N keys with an fp32 output (launch_dense_rows_tc).
 
 template <int D>
-size_t dense_smem_bytes() {
-  return ((size_t)PD_KEYS * (D + 1) + (size_t)PD_KEYS * D + (size_t)PD_ROWS * D) * sizeof(float);
-}
-
-template <int D>
-__global__ void __launch_bounds__(PB_THREADS) probe_dense_kernel(const ProbeArgs a) {
-  constexpr int PER_LANE = D / 32;       // output channels per lane
-  constexpr int KS = D + 1;              // padded K row: lanes read different rows conflict-free
-  extern __shared__ float psm[];
-  float* sk = psm;                       // [PD_KEYS][KS]
-  float* sv = sk + PD_KEYS * KS;         // [PD_KEYS][D]
-  float* sq = sv + PD_KEYS * D;          // [PD_ROWS][D], scaled by log2(e) / sqrt(D)
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y, m = blockIdx.x * PD_ROWS + warp;
-  const int tok = m < a.M ? probe_token(a, bh, m) : -1;
-  if (m < a.M && tok < 0 && lane == 0) flag_error(a.ctrl, DEV_BAD_INDEX, bh * a.M + m);
-  const float qscale = 1.4426950408889634f / sqrtf((float)D);
-  const __nv_bfloat16* qrow = a.q + ((size_t)bh * a.N + (tok < 0 ? 0 : tok)) * D;
-  for (int c = lane; c < D; c += 32)
-    sq[warp * D + c] = tok < 0 ? 0.f : __bfloat162float(qrow[c]) * qscale;
-
-  float mrow = -INFINITY, l = 0.f, acc[PER_LANE];
-#pragma unroll
-  for (int e = 0; e < PER_LANE; ++e) acc[e] = 0.f;
-  const __nv_bfloat16* kh = a.k + (size_t)bh * a.N * D;
-  const __nv_bfloat16* vh = a.v + (size_t)bh * a.N * D;
-  for (int n0 = 0; n0 < a.N; n0 += PD_KEYS) {
-    __syncthreads();   // the previous tile is no longer read
-    for (int e = threadIdx.x; e < PD_KEYS * D; e += PB_THREADS) {
-      const int j = e / D, c = e % D, n = n0 + j;
-      const bool in = n < a.N;
-      sk[j * KS + c] = in ? __bfloat162float(kh[(size_t)n * D + c]) : 0.f;
-      sv[j * D + c] = in ? __bfloat162float(vh[(size_t)n * D + c]) : 0.f;
-    }
-    __syncthreads();
-    // lane owns keys lane and lane + 32 of the tile
-    float s[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int j = lane + 32 * h;
-      float dot = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) dot = fmaf(sq[warp * D + c], sk[j * KS + c], dot);
-      s[h] = (n0 + j < a.N) ? dot : -INFINITY;
-    }
-    const float mt = warp_max_f(fmaxf(s[0], s[1]));     // finite: the tile holds key n0
-    const float mn = fmaxf(mrow, mt);
-    const float corr = exp2f(mrow - mn);                 // 0 on the first tile
-    const float p0 = exp2f(s[0] - mn), p1 = exp2f(s[1] - mn);
-    l = l * corr + warp_sum_f(p0 + p1);
-#pragma unroll
-    for (int e = 0; e < PER_LANE; ++e) acc[e] *= corr;
-    for (int j = 0; j < 32; ++j) {
-      const float pa = __shfl_sync(0xffffffffu, p0, j), pb = __shfl_sync(0xffffffffu, p1, j);
-#pragma unroll
-      for (int e = 0; e < PER_LANE; ++e) {
-        acc[e] = fmaf(pa, sv[j * D + lane + 32 * e], acc[e]);
-        acc[e] = fmaf(pb, sv[(j + 32) * D + lane + 32 * e], acc[e]);
-      }
-    }
-    mrow = mn;
-  }
+__global__ void __launch_bounds__(PB_THREADS) probe_gather_kernel(const ProbeArgs a, int m_alloc,
+                                                                  __nv_bfloat16* qg) {
+  constexpr int CH = D / 8;   // 16-byte chunks per row
+  const int bh = blockIdx.y;
+  const int e = blockIdx.x * PB_THREADS + threadIdx.x;
+  const int m = e / CH, c = e % CH;
+  if (m >= m_alloc) return;
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
   if (m < a.M) {
-    float* out = a.od + ((size_t)bh * a.M + m) * D;
-    const float inv = (tok >= 0 && l > 0.f) ? 1.f / l : 0.f;
-#pragma unroll
-    for (int e = 0; e < PER_LANE; ++e) out[lane + 32 * e] = acc[e] * inv;
+    const int tok = probe_token(a, bh, m);
+    if (tok >= 0) {
+      v = __ldg(reinterpret_cast<const uint4*>(a.q + ((size_t)bh * a.N + tok) * D) + c);
+    } else if (c == 0) {
+      flag_error(a.ctrl, DEV_BAD_INDEX, bh * a.M + m);
+    }
   }
+  reinterpret_cast<uint4*>(qg + ((size_t)bh * m_alloc + m) * D)[c] = v;
 }
 
 // ---- ridge fit -------------------------------------------------------------
@@ -437,14 +389,16 @@ __global__ void __launch_bounds__(D) probe_set_kernel(const ProbeArgs a) {
 }
 
 template <int D>
-cudaError_t launch_probe_d(const ProbeArgs& a, cudaStream_t s) {
+cudaError_t launch_probe_d(const Problem& p, const ProbeArgs& a, int m_alloc, __nv_bfloat16* qg,
+                           cudaStream_t s) {
   cudaError_t e;
-  if ((e = ensure_dyn_smem((const void*)probe_dense_kernel<D>, dense_smem_bytes<D>())) != cudaSuccess) return e;
   if ((e = ensure_dyn_smem((const void*)probe_fit_kernel<D>, fit_smem_bytes<D>())) != cudaSuccess) return e;
   if ((e = ensure_dyn_smem((const void*)probe_eig_kernel<D>, eig_smem_bytes<D>())) != cudaSuccess) return e;
   if ((e = ensure_dyn_smem((const void*)probe_apply_kernel<D>, apply_smem_bytes<D>())) != cudaSuccess) return e;
-  probe_dense_kernel<D><<<dim3((a.M + PD_ROWS - 1) / PD_ROWS, a.BH), PB_THREADS, dense_smem_bytes<D>(), s>>>(a);
+  const int gather_blocks = (m_alloc * (D / 8) + PB_THREADS - 1) / PB_THREADS;
+  probe_gather_kernel<D><<<dim3(gather_blocks, a.BH), PB_THREADS, 0, s>>>(a, m_alloc, qg);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_dense_rows_tc(p, qg, m_alloc, a.M, a.k, a.v, a.od, a.ctrl, s)) != cudaSuccess) return e;
   probe_fit_kernel<D><<<a.BH, PB_THREADS, fit_smem_bytes<D>(), s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   probe_eig_kernel<D><<<a.BH, PB_THREADS, eig_smem_bytes<D>(), s>>>(a);
@@ -457,10 +411,14 @@ cudaError_t launch_probe_d(const ProbeArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+// Probe queries are gathered into whole 128-row tiles.
+inline int probe_rows_alloc(int M) { return (M + 127) / 128 * 128; }
+
 size_t probe_scratch_bytes(const Problem& p, int M) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t BH = (size_t)p.BH, d = (size_t)p.d;
-  return up(BH * M * d * 4) + up(BH * (d + 1) * d * 4) + up(BH * d * d * 4) + up(BH * d * 4);
+  return up(BH * M * d * 4) + up(BH * (d + 1) * d * 4) + up(BH * d * d * 4) + up(BH * d * 4) +
+         up(BH * probe_rows_alloc(M) * d * 2);
 }
 
 cudaError_t launch_probe_correct(const Problem& p, const void* Q, const void* K, const void* V,
@@ -479,10 +437,13 @@ cudaError_t launch_probe_correct(const Problem& p, const void* Q, const void* K,
   a.od = reinterpret_cast<float*>(b + off); off += up(BH * M * d * 4);
   a.w = reinterpret_cast<float*>(b + off);  off += up(BH * (d + 1) * d * 4);
   a.wp = reinterpret_cast<float*>(b + off); off += up(BH * d * d * 4);
-  a.cp = reinterpret_cast<float*>(b + off);
+  a.cp = reinterpret_cast<float*>(b + off); off += up(BH * d * 4);
+  __nv_bfloat16* qg = reinterpret_cast<__nv_bfloat16*>(b + off);
   a.ctrl = ctrl;
   a.N = p.N; a.M = M; a.BH = p.BH; a.r = r; a.lam = lam;
-  return p.d == 128 ? launch_probe_d<128>(a, s) : launch_probe_d<64>(a, s);
+  const int m_alloc = probe_rows_alloc(M);
+  return p.d == 128 ? launch_probe_d<128>(p, a, m_alloc, qg, s)
+                    : launch_probe_d<64>(p, a, m_alloc, qg, s);
 }
 
 }  // namespace spattn

@@ -10,18 +10,9 @@
 // attention-mass aggregation (PARK page 5.1) and shares the selection.
 //
 // With a threshold instead (Sol-Attn abstract: blocks are selected by comparing
-// their proxy scores with a threshold; read as p_ij >= theta), the cut is
-// bits(theta) - 1 and only a binding clamp needs the search below.
-//
-// Selection without a sort: with p >= 0 the float bit pattern orders p, and
-// the mass G(u) = sum of p_j whose bits exceed u is monotone in u.  The kept
-// prefix is {p_j > v} plus the first few blocks with p_j == v (ascending j),
-// where v is the smallest value whose strictly-larger mass is < tau.  A
-// search over the bit patterns finds v: 32-way for rows of at most 128
-// blocks (each lane evaluates one candidate over the whole row), binary with
-// one warp reduction per step otherwise.  The same search on the count
-// #{p_j > u} yields the top-k set when the clamp binds.  Kept blocks are then
-// emitted in ascending j with warp ballots.
+// their proxy scores with a threshold; read as p_ij >= theta).  The selection
+// itself (a sort-free search on the float bits of p) is in select.cuh, shared
+// with the attention kernel's inline selection.
 //
 // route_kernel: one CTA per (ROWS query blocks, head), ROWS = 4, 8 or 16 by
 // the number of blocks so that small problems still fill the GPU; 8 warps.
@@ -33,6 +24,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "select.cuh"
 
 namespace spattn {
 namespace {
@@ -52,167 +44,19 @@ struct RouteArgs {
   int threshold;  // 1: keep p_ij >= tau (Sol-Attn on-the-fly thresholding)
 };
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-__device__ __forceinline__ int warp_sum_i(int v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
-// Mass of the blocks whose probability bits exceed u.
-__device__ __forceinline__ float mass_above(const float* p, int nb, uint32_t u) {
-  float s = 0.f;
-  for (int j = threadIdx.x & 31; j < nb; j += 32) {
-    const float x = p[j];
-    if (__float_as_uint(x) > u) s += x;
-  }
-  return warp_sum(s);
-}
-__device__ __forceinline__ int count_above(const float* p, int nb, uint32_t u) {
-  int c = 0;
-  for (int j = threadIdx.x & 31; j < nb; j += 32) c += (__float_as_uint(p[j]) > u) ? 1 : 0;
-  return warp_sum_i(c);
-}
-__device__ __forceinline__ int count_equal(const float* p, int nb, uint32_t u) {
-  int c = 0;
-  for (int j = threadIdx.x & 31; j < nb; j += 32) c += (__float_as_uint(p[j]) == u) ? 1 : 0;
-  return warp_sum_i(c);
-}
-
-// Smallest u in [lo, hi] with pred(u) true, for pred monotone in u (false
-// ... false true ... true) and pred(hi) true; warp-uniform result.  Each
-// round the 32 lanes test 32 evenly spaced candidates and the range shrinks
-// 32-fold, so 2^30 candidates need 6 rounds.  pred is evaluated by one lane
-// alone (a full pass over the row), which suits short rows.
-template <typename Pred>
-__device__ __forceinline__ uint32_t search32(uint32_t lo, uint32_t hi, Pred pred) {
-  const int lane = threadIdx.x & 31;
-  while (lo < hi) {
-    const uint32_t span = hi - lo;                    // candidates lo .. hi - 1 undecided
-    const uint32_t step = span / 32 + 1;
-    const uint32_t u = lo + (uint32_t)lane * step;
-    const bool in = u < hi;
-    const unsigned yes = __ballot_sync(0xffffffffu, in && pred(u));
-    const unsigned cand = __ballot_sync(0xffffffffu, in);
-    if (yes == 0u) {
-      // every tested candidate is false: the answer is above the last one
-      const int last = 31 - __clz(cand);
-      lo = lo + (uint32_t)last * step + 1;
-    } else {
-      const int first = __ffs(yes) - 1;
-      const uint32_t uf = lo + (uint32_t)first * step;
-      if (first == 0) return uf;                      // pred(lo) holds
-      lo = lo + (uint32_t)(first - 1) * step + 1;
-      hi = uf;
-    }
-  }
-  return lo;
-}
-
-// Mass / count of the blocks whose probability bits exceed u, by one lane.
-__device__ __forceinline__ float mass_above_1(const float* p, int nb, uint32_t u) {
-  float s = 0.f;
-  for (int j = 0; j < nb; ++j) {
-    const float x = p[j];
-    s += (__float_as_uint(x) > u) ? x : 0.f;
-  }
-  return s;
-}
-__device__ __forceinline__ int count_above_1(const float* p, int nb, uint32_t u) {
-  int c = 0;
-  for (int j = 0; j < nb; ++j) c += (__float_as_uint(p[j]) > u) ? 1 : 0;
-  return c;
-}
-
-// rows with at most this many blocks use the 32-way search
-constexpr int SEARCH32_MAX_NB = 128;
-
-// One warp: the Top-p selection and clamp on a probability row p[0..nb) in
-// shared memory, then the kept blocks of query row `row` emitted in
-// ascending j into the padded lists, and their count.
+// One warp: the selection of probability row p[0..nb) (shared memory), then
+// the kept blocks of query row `row` emitted in ascending j into the padded
+// lists, and their count.
 __device__ void select_emit(const float* p, const RouteArgs& a, int row) {
   const int lane = threadIdx.x & 31;
-  // kept set = {bits(p) > thr} + first `ties` blocks with bits(p) == thr
-  uint32_t thr = 0;
-  int ties = 0, kstar = 0;
-  bool by_mass = false;
-  if (a.threshold) {
-    // p >= theta: for theta > 0 the bits order p, so the critical set is
-    // {bits(p) > bits(theta) - 1}, a prefix of the (p desc, j asc) order;
-    // theta <= 0 keeps every block
-    if (a.tau <= 0.0f) {
-      kstar = a.nb;
-    } else {
-      thr = __float_as_uint(a.tau) - 1u;
-      kstar = count_above(p, a.nb, thr);
-      by_mass = true;  // the cut is set: the clamp search runs only if it binds
-    }
-  } else if (a.tau >= 1.0f) {
-    kstar = a.nb;               // tau >= 1 keeps every block
-  } else if (a.tau > 0.0f) {
-    if (a.nb <= SEARCH32_MAX_NB) {
-      thr = search32(0u, 0x3F800000u, [&](uint32_t u) { return mass_above_1(p, a.nb, u) < a.tau; });
-    } else {
-      uint32_t lo = 0, hi = 0x3F800000u;  // p <= 1, so nothing is above hi
-      while (lo < hi) {
-        const uint32_t mid = lo + ((hi - lo) >> 1);
-        if (mass_above(p, a.nb, mid) < a.tau) hi = mid; else lo = mid + 1;
-      }
-      thr = lo;
-    }
-    // the same summation as the search's predicate
-    const float g = a.nb <= SEARCH32_MAX_NB ? mass_above_1(p, a.nb, thr) : mass_above(p, a.nb, thr);
-    const int gt = count_above(p, a.nb, thr);
-    const int eq = count_equal(p, a.nb, thr);
-    const float v = __uint_as_float(thr);
-    float e = g;
-    int keep = 0;
-    while (keep < eq && e < a.tau) { e += v; ++keep; }
-    ties = keep;
-    kstar = gt + keep;
-    by_mass = true;
-  }
-  const int k = min(max(kstar, a.kmin), a.kcap);
-  const bool all = (k >= a.nb);
-  if (!all && !(by_mass && k == kstar)) {
-    // the clamp binds (or tau <= 0): top-k in (p desc, j asc) order
-    if (a.nb <= SEARCH32_MAX_NB) {
-      thr = search32(0u, 0x3F800000u, [&](uint32_t u) { return count_above_1(p, a.nb, u) < k; });
-    } else {
-      uint32_t lo = 0, hi = 0x3F800000u;
-      while (lo < hi) {
-        const uint32_t mid = lo + ((hi - lo) >> 1);
-        if (count_above(p, a.nb, mid) < k) hi = mid; else lo = mid + 1;
-      }
-      thr = lo;
-    }
-    ties = k - count_above(p, a.nb, thr);
-  }
+  const sel::Cut c = sel::cut_row(p, a.nb, a.tau, a.threshold, a.kmin, a.kcap);
   int32_t* out = a.lists + (size_t)row * a.kcap;
-  int base = 0, seen_eq = 0;
-  for (int j0 = 0; j0 < a.nb; j0 += 32) {
-    const int j = j0 + lane;
-    const bool valid = j < a.nb;
-    const uint32_t u = valid ? __float_as_uint(p[j]) : 0u;
-    const bool eq = valid && !all && u == thr;
-    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-    const int eq_rank = seen_eq + __popc(eqm & ((1u << lane) - 1u));
-    seen_eq += __popc(eqm);
-    const bool keep = valid && (all || u > thr || (eq && eq_rank < ties));
-    const unsigned km = __ballot_sync(0xffffffffu, keep);
-    if (keep) out[base + __popc(km & ((1u << lane) - 1u))] = j;
+  int base = 0;
+  sel::walk_kept(p, a.nb, c, [&](int j0, bool keep, unsigned km) {
+    if (keep) out[base + __popc(km & ((1u << lane) - 1u))] = j0 + lane;
     base += __popc(km);
-  }
-  if (lane == 0) a.counts[row] = k;
+  });
+  if (lane == 0) a.counts[row] = c.k;
 }
 
 
@@ -235,7 +79,7 @@ __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
   // each thread a strided share of the channels, reduced with shuffles;
   // TPJ = 256 / nb (at most 32) keeps every thread busy when nb is small
   const float inv_sqrt_d = 1.0f / sqrtf((float)D);
-  const int tpj = a.nb >= RT_THREADS ? 1 : (a.nb >= 128 ? 2 : (a.nb >= 64 ? 4 : (a.nb >= 32 ? 8 : 16)));
+  const int tpj = sel::proxy_threads_per_block(a.nb);
   const int sub = threadIdx.x % tpj, grp = threadIdx.x / tpj, ngrp = RT_THREADS / tpj;
   for (int j0 = 0; j0 < a.nb; j0 += ngrp) {
     const int j = j0 + grp;
@@ -275,18 +119,7 @@ __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int r = warp; r < rows; r += RT_THREADS / 32) {
     float* p = S + r * nbp;
-    float mx = -INFINITY;
-    for (int j = lane; j < a.nb; j += 32) mx = fmaxf(mx, p[j]);
-    mx = warp_max(mx);
-    float sum = 0.f;
-    for (int j = lane; j < a.nb; j += 32) {
-      const float e = expf(p[j] - mx);
-      p[j] = e;
-      sum += e;
-    }
-    sum = warp_sum(sum);
-    for (int j = lane; j < a.nb; j += 32) p[j] = p[j] / sum;
-    __syncwarp();
+    sel::softmax_row(p, a.nb);
     select_emit(p, a, bh * a.nb + i0 + r);
   }
 }

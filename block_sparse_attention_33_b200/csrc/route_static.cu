@@ -127,6 +127,7 @@ extern "C" spattn_status_t spattn_route_static(int B, int H, int N, int d, int b
   p.use_tc = 0;
   p.routing = spattn::ROUTING_CENTROID;
   p.threshold = 0;
+  p.inline_sel = 0;
   p.test_stall = 0;
   p.perm = perm;
 

@@ -116,9 +116,30 @@ enum {
  * before. */
 enum { SPATTN_SELECT_THRESHOLD = 16 };
 
+/* Selection flag, OR'ed into the routing argument of spattn_plan_ex (with
+ * the centroid estimate, optionally with SPATTN_SELECT_THRESHOLD): the
+ * attention kernel selects the blocks itself, inside the attention pass
+ * (Sol-Attn abstract, thelatestinai page: critical blocks are chosen by
+ * comparing proxy scores with a threshold during the online softmax, without
+ * materialising the proxy map).  Per work item the kernel scores its query
+ * block against every key block from the fp32 means, forms the block softmax
+ * and cuts the row (threshold theta = tau, or Top-p mass tau, with the same
+ * clamp), in on-chip memory only, with the same arithmetic as the routing
+ * kernel, so it keeps exactly the blocks spattn_route would list.  With it:
+ *   spattn_forward  is spattn_pool + the attention: no routing launch, no
+ *                   kept lists, no CSR;
+ *   spattn_attend   with NULL row_ptr / col_idx selects from the means the
+ *                   last spattn_pool or spattn_route left in the workspace
+ *                   (a caller CSR is used as given);
+ *   spattn_route    still writes the CSR of the same selection, for callers
+ *                   that want to see it.
+ * The budget of every query block is found per work item, so the work runs
+ * in plain (batch, head, block) order rather than longest-first. */
+enum { SPATTN_SELECT_INLINE = 32 };
+
 /* spattn_plan with a choice of routing estimate (one of the values above,
- * optionally | SPATTN_SELECT_THRESHOLD; anything else is
- * SPATTN_ERR_INVALID_ARG).  spattn_plan is
+ * optionally | SPATTN_SELECT_THRESHOLD and, with the centroid estimate,
+ * | SPATTN_SELECT_INLINE; anything else is SPATTN_ERR_INVALID_ARG).  spattn_plan is
  * spattn_plan_ex(..., SPATTN_ROUTING_CENTROID, ...).  spattn_route_static
  * always uses the centroid estimate and the Top-p selection. */
 spattn_status_t spattn_plan_ex(spattn_plan_t* out, int B, int H, int N, int d, int b,
@@ -165,7 +186,9 @@ spattn_status_t spattn_route(spattn_plan_t plan, const void* Q, const void* K, c
  *                     and a col_idx that holds every entry row_ptr
  *                     points at: the library cannot see the size of a device
  *                     buffer and reads col_idx[row_ptr[r] .. row_ptr[r+1]).
- *                     A block listed twice is attended twice.  Block
+ *                     With b = 128 a block listed twice is attended twice;
+ *                     with b = 64 two query blocks share their key tiles
+ *                     and a block listed twice counts once.  Block
  *                     indices outside [0, nb) are skipped and flagged
  *                     (SPATTN_ERR_DEVICE from spattn_check).  With a
  *                     caller CSR the call first clears the workspace's
@@ -241,9 +264,11 @@ spattn_status_t spattn_probe_scratch_bytes(spattn_plan_t plan, int M, size_t* by
  *   workspace the plan's workspace (its device error word only);
  *   scratch   device, spattn_probe_scratch_bytes(plan, M) bytes, 256-byte
  *             aligned.
- * Everything is fp32 on the device: the exact probe rows, the (d+1) x (d+1)
- * normal equations solved by Cholesky factorisation, the eigenvectors of
- * R^T R by cyclic Jacobi rotations, and one pass O += O (B P) + b P.  Normal
+ * The exact probe rows run on the tensor cores, as the attention does (bf16
+ * operands, fp32 accumulation), with an fp32 output; the rest is fp32 on the
+ * device: the (d+1) x (d+1) normal equations solved by Cholesky
+ * factorisation, the eigenvectors of R^T R by cyclic Jacobi rotations, and
+ * one pass O += O (B P) + b P.  Normal
  * equations that are not positive definite (lam = 0 with fewer than d + 1
  * independent probe rows, for instance) leave that head uncorrected and are
  * flagged (spattn_check: SPATTN_ERR_DEVICE).  B*H <= 65535. */

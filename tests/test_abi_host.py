@@ -115,13 +115,18 @@ def test_hilbert_rejects_bad_grid(L):
 
 def test_plan_ex_routing_argument(L):
     """spattn_plan_ex accepts the two routing estimates, each with or without
-    the threshold selection flag (no CUDA needed without a permutation), and
-    rejects anything else before any CUDA call."""
-    T = sp.SELECT_THRESHOLD
+    the threshold selection flag, and the inline selection flag with the
+    centroid estimate (no CUDA needed without a permutation); it rejects
+    anything else, the inline flag with PAMA among them, before any CUDA
+    call."""
+    T, I = sp.SELECT_THRESHOLD, sp.SELECT_INLINE
     for routing, code in ((sp.ROUTING_CENTROID, sp.OK), (sp.ROUTING_PAMA, sp.OK),
                           (sp.ROUTING_CENTROID | T, sp.OK), (sp.ROUTING_PAMA | T, sp.OK),
+                          (sp.ROUTING_CENTROID | I, sp.OK), (sp.ROUTING_CENTROID | T | I, sp.OK),
+                          (sp.ROUTING_PAMA | I, sp.ERR_INVALID_ARG),
+                          (sp.ROUTING_PAMA | T | I, sp.ERR_INVALID_ARG),
                           (2, sp.ERR_INVALID_ARG), (-1, sp.ERR_INVALID_ARG), (2 | T, sp.ERR_INVALID_ARG),
-                          (32, sp.ERR_INVALID_ARG)):
+                          (64, sp.ERR_INVALID_ARG)):
         h = ctypes.c_void_p()
         ws = ctypes.c_size_t()
         st = L.spattn_plan_ex(ctypes.byref(h), 1, 2, 1000, 64, 64, 0.9, 1, 8, 1, None, routing,
@@ -226,8 +231,9 @@ def test_binding_checks_host_tensors_of_the_host_forward(L):
 
 
 def test_probe_correct_argument_checks(L):
-    """spattn_probe_scratch_bytes sizes the exact rows, the fit, B P and b P;
-    spattn_probe_correct refuses bad arguments before any CUDA call."""
+    """spattn_probe_scratch_bytes sizes the exact rows, the fit, B P, b P and
+    the gathered probe queries (whole 128-row tiles); spattn_probe_correct
+    refuses bad arguments before any CUDA call."""
     B, H, N, d = 1, 3, 1000, 64
     st, h, ws = plan_status(B, H, N, d, 64, 0.9, 1, 4, 1)
     assert st == sp.OK
@@ -236,7 +242,7 @@ def test_probe_correct_argument_checks(L):
     M = 48
     assert L.spattn_probe_scratch_bytes(h, M, ctypes.byref(n)) == sp.OK
     assert n.value == (up(B * H * M * d * 4) + up(B * H * (d + 1) * d * 4) + up(B * H * d * d * 4)
-                       + up(B * H * d * 4))
+                       + up(B * H * d * 4) + up(B * H * 128 * d * 2))
     assert L.spattn_probe_scratch_bytes(h, 0, ctypes.byref(n)) == sp.ERR_INVALID_ARG
     f = L.spattn_probe_correct
     ok = dict(Q=16, K=16, V=16, O=16, probes=16, M=M, lam=100.0, r=8, ws=256, scratch=256)

@@ -1,0 +1,109 @@
+"""Inline selection (Sol-Attn abstract, thelatestinai page: critical blocks are
+chosen by comparing proxy scores with a threshold during the online softmax,
+without materialising the proxy map): with SPATTN_SELECT_INLINE the attention
+kernel scores and cuts every query block itself, and spattn_forward is the
+pooling plus the attention alone.
+
+The kernel uses the routing kernel's arithmetic, so its output must equal,
+bit for bit, the output of route + attend with the same knobs (the same kept
+sets in the same order through the same attention kernel).  The routing
+kernel's CSR of that selection is compared with the oracle (route_threshold /
+route_rows; marginal blocks only may differ), and the fused output with the
+oracle's attention on those kept sets, within the output bounds."""
+import numpy as np
+import pytest
+
+from tests.harness import (MAX_ABS, REL_L2, compare_outputs, from_dev, oracle_check, run_library,
+                           to_dev)
+from workloads import get_config, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu(gpu_required):
+    import block_sparse_attention_33_b200 as sp
+    sp.lib()
+
+
+def _fused_forward(w, Q, K, V, routing, perm=None):
+    import torch
+    import block_sparse_attention_33_b200 as sp
+    plan = sp.Plan(w.B, w.H, w.N, w.d, w.b, w.tau, w.kmin, w.kmax, w.residual, perm,
+                   routing=routing | sp.SELECT_INLINE)
+    try:
+        q, k, v = to_dev(Q), to_dev(K), to_dev(V)
+        o = torch.full_like(q, float("nan"))
+        plan.forward(q, k, v, o)
+        status = plan.check()
+        torch.cuda.synchronize()
+        return status, from_dev(o)
+    finally:
+        plan.close()
+
+
+# (description, workload, overrides, threshold selection?)
+CASES = [
+    ("tiny b=64 theta 0.05", "tiny", dict(tau=0.05), True),
+    ("tiny b=64 theta 0.1, kmin 2 binds", "tiny", dict(tau=0.1, kmin=2, kmax=4), True),
+    ("tiny b=64 top-p 0.8", "tiny", dict(tau=0.8), False),
+    ("b=128 partial tail, theta 0.05", "tiny", dict(grid=(1, 5, 100), d=128, b=128, H=2, kmax=8,
+                                                     tau=0.05), True),
+    ("medium theta 0.01", "medium", dict(H=2, tau=0.01), True),
+    ("medium theta 0.02, no residual", "medium", dict(H=2, tau=0.02, residual=0), True),
+    ("medium top-p 0.9", "medium", dict(H=2), False),
+    ("medium top-p 0.9, kmax 8 binds", "medium", dict(H=2, kmax=8), False),
+    ("medium d=64 b=64 top-p 0.85", "medium", dict(H=2, d=64, b=64, tau=0.85), False),
+]
+
+
+@pytest.mark.parametrize("desc,name,ov,threshold", CASES, ids=[c[0] for c in CASES])
+def test_inline_selection_equals_route_and_attend(desc, name, ov, threshold):
+    import block_sparse_attention_33_b200 as sp
+    w = get_config(name, **ov)
+    Q, K, V = make_qkv(w)
+    routing = sp.ROUTING_CENTROID | (sp.SELECT_THRESHOLD if threshold else 0)
+    res = run_library(w, Q, K, V, routing=routing)
+    assert res["status"] == 0
+    status, o = _fused_forward(w, Q, K, V, routing)
+    assert status == sp.OK
+    assert np.array_equal(o, res["O"]), "fused output differs from route + attend"
+    fig = oracle_check(w, Q, K, V, res, selection="threshold" if threshold else "top_p")
+    assert fig["bad"] == 0, fig
+    max_abs, rel = compare_outputs(o, fig["ref"]["O"])
+    assert max_abs < MAX_ABS and rel < REL_L2, (max_abs, rel)
+
+
+@pytest.mark.parametrize("tau,kmax,threshold", [(0.005, 256, True), (0.002, 64, True),
+                                                 (0.9, 256, False)],
+                         ids=["wan theta 0.005", "wan theta 0.002, kmax 64 (every row clamped)",
+                              "wan top-p 0.9"])
+def test_inline_selection_at_wan_size(tau, kmax, threshold):
+    """nb = 256: the mass search and the clamp's top-k take the binary search
+    over 256-wide rows; the fused output still equals route + attend."""
+    import block_sparse_attention_33_b200 as sp
+    from tests.test_gpu_full_size import sample_rows
+    w = get_config("wan", H=2, tau=tau, kmax=kmax)
+    Q, K, V = make_qkv(w)
+    routing = sp.ROUTING_CENTROID | (sp.SELECT_THRESHOLD if threshold else 0)
+    res = run_library(w, Q, K, V, routing=routing)
+    assert res["status"] == 0
+    status, o = _fused_forward(w, Q, K, V, routing)
+    assert status == sp.OK
+    assert np.array_equal(o, res["O"])
+    rows = sample_rows(w, res, None)
+    fig = oracle_check(w, Q, K, V, res, rows=rows, selection="threshold" if threshold else "top_p")
+    assert fig["bad"] == 0 and fig["max_abs"] < MAX_ABS and fig["rel_l2"] < REL_L2, fig
+
+
+def test_inline_selection_with_hilbert_permutation():
+    import block_sparse_attention_33_b200 as sp
+    w = get_config("stress", H=2, tau=0.01)
+    Q, K, V = make_qkv(w)
+    perm = sp.spattn_hilbert_perm(*w.grid)
+    routing = sp.ROUTING_CENTROID | sp.SELECT_THRESHOLD
+    res = run_library(w, Q, K, V, perm=perm, routing=routing)
+    status, o = _fused_forward(w, Q, K, V, routing, perm=perm)
+    assert res["status"] == 0 and status == sp.OK
+    assert np.array_equal(o, res["O"])
+

@@ -39,6 +39,14 @@ SMALL = [
     ("d=64 b=128", dict(grid=(2, 8, 64), d=64, b=128, H=2, tau=0.85)),
     ("no residual", dict(grid=(2, 8, 64), d=128, b=128, H=2, tau=0.6, residual=0)),
     ("tau=1 dense", dict(grid=(2, 8, 64), d=128, b=128, H=2, tau=1.0)),
+    # 64-token blocks: two query blocks per 128-row tile, two key blocks per
+    # key tile (union of the two kept sets)
+    ("b=64 d=64", dict()),
+    ("b=64 d=128", dict(d=128, H=2, tau=0.8)),
+    ("b=64 no residual", dict(residual=0, kmax=3, tau=0.6)),
+    ("b=64 odd nb, one token in the last block", dict(grid=(1, 5, 13), kmax=2)),
+    ("b=64 three blocks, last tile single", dict(grid=(1, 3, 64), kmax=2, tau=0.5)),
+    ("b=64 partial last block of 20", dict(grid=(1, 7, 12), d=128, kmax=3, tau=0.7)),
 ]
 
 
