@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (lane == 0) ticket = atomicAdd(a.ctrl + CTRL_WORK, 1);
       ticket = __shfl_sync(0xffffffffu, ticket, 0);
       ItemInfo& inf = cs->info[slot];
-      if (ticket >= a.items) {
+      if ((unsigned)ticket >= (unsigned)a.items) {   // also a counter left invalid
         if (lane == 0) inf.item = -1;
         __syncwarp();
         tc::mbar_arrive(bar(B_INFO_FULL0 + slot));
@@ -1015,6 +1015,11 @@ cudaError_t launch_dense_rows_tc(const Problem& p, const void* Qg, int q_alloc, 
   a.kcap = nb;
   a.sl2 = 1.4426950408889634f / sqrtf((float)p.d);
   a.items = p.BH * a.nq;
+  // the work ticket and retirement count start from zero (the workspace may
+  // never have run an attention); the error word is left as it is
+  static_assert(CTRL_DONE == CTRL_WORK + 1, "ticket words cleared together");
+  cudaError_t e = cudaMemsetAsync(ctrl + CTRL_WORK, 0, 2 * sizeof(int32_t), s);
+  if (e != cudaSuccess) return e;
   return p.d == 128 ? launch_tc<128>(maps, a, s) : launch_tc<64>(maps, a, s);
 }
 

@@ -38,7 +38,6 @@ namespace spattn {
 namespace {
 
 constexpr int PB_THREADS = 256;
-constexpr int PF_CHUNK = 32;               // probe rows per accumulation chunk
 constexpr int PA_ROWS = 64;                // output rows per apply CTA
 constexpr int JACOBI_MAX_SWEEPS = 16;
 
@@ -50,6 +49,7 @@ struct ProbeArgs {
   float* w;                        // [BH, D + 1, D] ridge solution, row 0 = b
   float* wp;                       // [BH, D, D] B P
   float* cp;                       // [BH, D] b P
+  float* pu;                       // [BH, D, D] leading eigenvectors of R^T R (first r columns)
   int32_t* ctrl;                   // error word
   int N, M, BH, r;
   float lam;
@@ -96,184 +96,187 @@ __global__ void __launch_bounds__(PB_THREADS) probe_gather_kernel(const ProbeArg
   reinterpret_cast<uint4*>(qg + ((size_t)bh * m_alloc + m) * D)[c] = v;
 }
 
-// ---- ridge fit -------------------------------------------------------------
+// ---- Gram matrix of the probe rows -----------------------------------------
+// Every quantity of the fit comes from the Gram matrix of the rows
+// Z = [1, x, R] (x the sparse output of a probe row, R = exact - x): with
+// A = [1, x], G = A^T A, C = A^T R and S = R^T R are its blocks.  The rows of
+// one head are cut into slabs of GR_ROWS; one CTA per (slab, head) adds up
+// the upper-triangle 4 x 4 tiles of its slab's Gram matrix (register tiles,
+// rows staged in shared memory 32 at a time) and writes them to its own
+// partial buffer; the solve kernel adds the partials in slab order.
+
+constexpr int GR_ROWS = 128;      // probe rows per Gram CTA
+constexpr int GR_THREADS = 768;
+constexpr int GR_CHUNK = 32;      // rows staged at a time
+constexpr int SV_THREADS = 1024;  // solve kernel
+constexpr int SUB_ITERS = 24;     // subspace iterations
+constexpr int SUB_EXTRA = 16;     // subspace columns beyond r
+constexpr int SUB_MAXQ = 64;      // subspace iteration for r + SUB_EXTRA <= 64, else Jacobi
 
 template <int D>
-size_t fit_smem_bytes() {
-  constexpr int DA = D + 1;
-  return ((size_t)DA * DA + (size_t)DA * D + (size_t)PF_CHUNK * DA + (size_t)PF_CHUNK * D + 4) *
-         sizeof(float);
+struct GramGeom {
+  static constexpr int ZC = 1 + 2 * D;                // columns of Z
+  static constexpr int NT = (ZC + 3) / 4;             // 4-wide column tiles
+  static constexpr int ZW = 4 * NT;                   // padded row width
+  static constexpr int TILES = NT * (NT + 1) / 2;     // upper-triangle tiles
+  static constexpr int PER = (TILES + GR_THREADS - 1) / GR_THREADS;
+};
+
+inline int gram_slabs(int M) { return (M + GR_ROWS - 1) / GR_ROWS; }
+
+// tile index e (row-major over the upper triangle, ti <= tj) -> (ti, tj)
+__device__ __forceinline__ void upper_tile(int e, int nt, int& ti, int& tj) {
+  int i = 0, rowlen = nt;
+  while (e >= rowlen) { e -= rowlen; ++i; --rowlen; }
+  ti = i;
+  tj = i + e;
 }
 
-// Rows m0 .. m0 + PF_CHUNK - 1 of A = [1, x] and R = x_exact - x into shared
-// memory (rows past M, or with a bad probe index, are zero and add nothing).
 template <int D>
-__device__ void load_probe_chunk(const ProbeArgs& a, int bh, int m0, float* xa, float* rc) {
-  constexpr int DA = D + 1;
-  for (int e = threadIdx.x; e < PF_CHUNK * D; e += PB_THREADS) {
-    const int rr = e / D, c = e % D, m = m0 + rr;
-    const int tok = m < a.M ? probe_token(a, bh, m) : -1;
-    float x = 0.f, res = 0.f;
-    if (tok >= 0) {
-      x = __bfloat162float(a.o[((size_t)bh * a.N + tok) * D + c]);
-      res = a.od[((size_t)bh * a.M + m) * D + c] - x;
+__global__ void __launch_bounds__(GR_THREADS) probe_gram_kernel(const ProbeArgs a, float* gp,
+                                                                int slabs) {
+  using G = GramGeom<D>;
+  __shared__ __align__(16) float Zs[GR_CHUNK][G::ZW];
+  const int slab = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  int ti[G::PER], tj[G::PER];
+  float acc[G::PER][16];
+#pragma unroll
+  for (int u = 0; u < G::PER; ++u) {
+    const int e = tid + u * GR_THREADS;
+    if (e < G::TILES) upper_tile(e, G::NT, ti[u], tj[u]); else ti[u] = tj[u] = -1;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) acc[u][k] = 0.f;
+  }
+  const int m_lo = slab * GR_ROWS, m_hi = min(a.M, m_lo + GR_ROWS);
+  for (int m0 = m_lo; m0 < m_hi; m0 += GR_CHUNK) {
+    __syncthreads();
+    // Z rows m0 .. m0 + 31 (zero past the slab, or for a bad probe index)
+    for (int e = tid; e < GR_CHUNK * G::ZW; e += GR_THREADS) {
+      const int rr = e / G::ZW, c = e % G::ZW, m = m0 + rr;
+      const int tok = m < m_hi ? probe_token(a, bh, m) : -1;
+      float z = 0.f;
+      if (tok >= 0) {
+        if (c == 0) {
+          z = 1.f;
+        } else if (c <= D) {
+          z = __bfloat162float(a.o[((size_t)bh * a.N + tok) * D + c - 1]);
+        } else if (c <= 2 * D) {
+          const int cc = c - D - 1;
+          z = a.od[((size_t)bh * a.M + m) * D + cc] -
+              __bfloat162float(a.o[((size_t)bh * a.N + tok) * D + cc]);
+        }
+      }
+      Zs[rr][c] = z;
     }
-    xa[rr * DA + 1 + c] = x;
-    rc[rr * D + c] = res;
-    if (c == 0) xa[rr * DA] = tok >= 0 ? 1.f : 0.f;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < G::PER; ++u) {
+      if (ti[u] < 0) continue;
+      for (int rr = 0; rr < GR_CHUNK; ++rr) {
+        const float4 x = *reinterpret_cast<const float4*>(&Zs[rr][4 * ti[u]]);
+        const float4 y = *reinterpret_cast<const float4*>(&Zs[rr][4 * tj[u]]);
+        const float xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[u][4 * p + q] = fmaf(xs[p], ys[q], acc[u][4 * p + q]);
+      }
+    }
+  }
+  float* out = gp + ((size_t)bh * slabs + slab) * G::ZW * G::ZW;
+#pragma unroll
+  for (int u = 0; u < G::PER; ++u) {
+    if (ti[u] < 0) continue;
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+      *reinterpret_cast<float4*>(out + (size_t)(4 * ti[u] + p) * G::ZW + 4 * tj[u]) =
+          make_float4(acc[u][4 * p], acc[u][4 * p + 1], acc[u][4 * p + 2], acc[u][4 * p + 3]);
   }
 }
 
+// Entry (i, j) of a head's Gram matrix: the slabs' partials added in order
+// (only upper-triangle tiles are stored, so (i, j) is read from the tile side).
 template <int D>
-__global__ void __launch_bounds__(PB_THREADS) probe_fit_kernel(const ProbeArgs a) {
-  constexpr int DA = D + 1;
-  extern __shared__ float psm[];
-  float* G = psm;                  // [DA][DA]
-  float* C = G + DA * DA;          // [DA][D], then the solution W
-  float* xa = C + DA * D;          // [PF_CHUNK][DA]
-  float* rc = xa + PF_CHUNK * DA;  // [PF_CHUNK][D]
-  int* bad = reinterpret_cast<int*>(rc + PF_CHUNK * D);
-  const int bh = blockIdx.x, tid = threadIdx.x;
-  for (int e = tid; e < DA * DA; e += PB_THREADS) G[e] = 0.f;
-  for (int e = tid; e < DA * D; e += PB_THREADS) C[e] = 0.f;
-  if (tid == 0) *bad = 0;
-  for (int m0 = 0; m0 < a.M; m0 += PF_CHUNK) {
-    __syncthreads();
-    load_probe_chunk<D>(a, bh, m0, xa, rc);
-    __syncthreads();
-    for (int e = tid; e < DA * DA; e += PB_THREADS) {
-      const int i = e / DA, j = e % DA;
-      float s = G[e];
-      for (int rr = 0; rr < PF_CHUNK; ++rr) s = fmaf(xa[rr * DA + i], xa[rr * DA + j], s);
-      G[e] = s;
-    }
-    for (int e = tid; e < DA * D; e += PB_THREADS) {
-      const int i = e / D, c = e % D;
-      float s = C[e];
-      for (int rr = 0; rr < PF_CHUNK; ++rr) s = fmaf(xa[rr * DA + i], rc[rr * D + c], s);
-      C[e] = s;
-    }
-  }
-  __syncthreads();
-  for (int i = 1 + tid; i < DA; i += PB_THREADS) G[i * DA + i] += a.lam;   // the bias is not penalised
-  __syncthreads();
-  // Cholesky, lower triangle in place: G = L L^T
-  for (int k = 0; k < DA; ++k) {
+__device__ __forceinline__ float gram_at(const float* gph, int slabs, int i, int j) {
+  using G = GramGeom<D>;
+  if ((i >> 2) > (j >> 2)) { const int t = i; i = j; j = t; }
+  float s = 0.f;
+  for (int k = 0; k < slabs; ++k) s += gph[(size_t)k * G::ZW * G::ZW + (size_t)i * G::ZW + j];
+  return s;
+}
+
+// ---- solve: ridge fit (role 0) and residual subspace (role 1) ---------------
+
+template <int D>
+constexpr size_t solve_smem_bytes() {
+  constexpr size_t DA = D + 1;
+  constexpr size_t fit = (DA * DA + DA * D + 8) * sizeof(float);
+  constexpr size_t jac = (2 * (size_t)D * (D + 1) + 4 * (size_t)D + 8) * sizeof(float);
+  constexpr size_t sub = ((size_t)D * (D + 1) + 2 * (size_t)D * SUB_MAXQ +
+                          2 * (size_t)SUB_MAXQ * (SUB_MAXQ + 1) + 4 * (size_t)SUB_MAXQ + 8) *
+                         sizeof(float);
+  return fit > jac ? (fit > sub ? fit : sub) : (jac > sub ? jac : sub);
+}
+
+// In-place Cholesky of the n x n matrix A (row stride ld, lower triangle
+// used) by the whole CTA; a pivot that is not positive and finite sets *bad
+// (and is replaced by a tiny one so the factorisation still completes).
+__device__ void cholesky_cta(float* A, int n, int ld, int* bad) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  for (int k = 0; k < n; ++k) {
     if (tid == 0) {
-      const float dkk = G[k * DA + k];
+      const float dkk = A[k * ld + k];
       if (!(dkk > 0.f) || !isfinite(dkk)) *bad = 1;
-      G[k * DA + k] = sqrtf(fmaxf(dkk, 1e-30f));
+      A[k * ld + k] = sqrtf(fmaxf(dkk, 1e-30f));
     }
     __syncthreads();
-    const float lkk = G[k * DA + k];
-    for (int i = k + 1 + tid; i < DA; i += PB_THREADS) G[i * DA + k] /= lkk;
+    const float lkk = A[k * ld + k];
+    for (int i = k + 1 + tid; i < n; i += nt) A[i * ld + k] /= lkk;
     __syncthreads();
-    const int n = DA - k - 1;   // trailing block (k, DA) x (k, DA), lower part
-    for (int e = tid; e < n * n; e += PB_THREADS) {
-      const int i = k + 1 + e / n, j = k + 1 + e % n;
-      if (j <= i) G[i * DA + j] = fmaf(-G[i * DA + k], G[j * DA + k], G[i * DA + j]);
+    const int m = n - k - 1;   // trailing block, lower part
+    for (int e = tid; e < m * m; e += nt) {
+      const int i = k + 1 + e / m, j = k + 1 + e % m;
+      if (j <= i) A[i * ld + j] = fmaf(-A[i * ld + k], A[j * ld + k], A[i * ld + j]);
     }
     __syncthreads();
   }
-  // L Y = C, then L^T W = Y: one right-hand side (output channel) per thread
-  for (int c = tid; c < D; c += PB_THREADS) {
-    for (int i = 0; i < DA; ++i) {
-      float s = C[i * D + c];
-      for (int k = 0; k < i; ++k) s = fmaf(-G[i * DA + k], C[k * D + c], s);
-      C[i * D + c] = s / G[i * DA + i];
-    }
-    for (int i = DA - 1; i >= 0; --i) {
-      float s = C[i * D + c];
-      for (int k = i + 1; k < DA; ++k) s = fmaf(-G[k * DA + i], C[k * D + c], s);
-      C[i * D + c] = s / G[i * DA + i];
-    }
-  }
-  __syncthreads();
-  const bool failed = *bad != 0;
-  if (failed && tid == 0) flag_error(a.ctrl, DEV_NUMERIC, bh);
-  float* w = a.w + (size_t)bh * DA * D;
-  for (int e = tid; e < DA * D; e += PB_THREADS) w[e] = failed ? 0.f : C[e];
 }
 
-// ---- residual subspace and the folded correction --------------------------
-
-template <int D>
-size_t eig_smem_bytes() {
-  return ((size_t)2 * D * (D + 1) + (size_t)PF_CHUNK * D + (size_t)PF_CHUNK * (D + 1) +
-          (size_t)2 * (D / 2) + 2 * D + 4) * sizeof(float);
-}
-
-template <int D>
-__global__ void __launch_bounds__(PB_THREADS) probe_eig_kernel(const ProbeArgs a) {
-  constexpr int DP = D + 1;        // padded row: column updates hit distinct banks
-  constexpr int H = D / 2;
-  extern __shared__ float psm[];
-  float* S = psm;                  // [D][DP]: R^T R, rotated towards diagonal; later P
-  float* V = S + D * DP;           // [D][DP]: eigenvectors (columns); later B
-  float* xa = V + D * DP;          // [PF_CHUNK][D + 1]
-  float* rc = xa + PF_CHUNK * (D + 1);   // [PF_CHUNK][D]
-  float* rot_c = rc + PF_CHUNK * D;      // [H]
-  float* rot_s = rot_c + H;              // [H]
-  float* lam = rot_s + H;                // [D] eigenvalues
-  float* sel = lam + D;                  // [D] 1 for the r largest, else 0
-  int* flags = reinterpret_cast<int*>(sel + D);
-  __shared__ int pp[H], qq[H];
-  const int bh = blockIdx.x, tid = threadIdx.x;
-  const float* wfit = a.w + (size_t)bh * (D + 1) * D;
-  float* wp = a.wp + (size_t)bh * D * D;
-  float* cp = a.cp + (size_t)bh * D;
-
-  if (a.r <= 0 || a.r >= D) {
-    // P = 0 (no correction) or P = I (the whole output space)
-    const bool full = a.r >= D;
-    for (int e = tid; e < D * D; e += PB_THREADS) wp[e] = full ? wfit[D + e] : 0.f;
-    for (int c = tid; c < D; c += PB_THREADS) cp[c] = full ? wfit[c] : 0.f;
-    return;
-  }
-  for (int e = tid; e < D * DP; e += PB_THREADS) S[e] = 0.f;
-  for (int m0 = 0; m0 < a.M; m0 += PF_CHUNK) {
-    __syncthreads();
-    load_probe_chunk<D>(a, bh, m0, xa, rc);
-    __syncthreads();
-    for (int e = tid; e < D * D; e += PB_THREADS) {
-      const int i = e / D, j = e % D;
-      float s = S[i * DP + j];
-      for (int rr = 0; rr < PF_CHUNK; ++rr) s = fmaf(rc[rr * D + i], rc[rr * D + j], s);
-      S[i * DP + j] = s;
-    }
-  }
-  for (int e = tid; e < D * DP; e += PB_THREADS) V[e] = (e % DP == e / DP) ? 1.f : 0.f;
+// Cyclic Jacobi on the symmetric n x n matrix S (row stride ld, n even),
+// round-robin pairing (n / 2 disjoint rotations per step; every pair meets
+// once in a sweep of n - 1 steps), accumulating the rotations into V (row
+// stride ld, starts at the identity).  Stops when the off-diagonal mass is
+// negligible against the diagonal.  rc, rs: n / 2 floats; pq: n ints; flag: 1.
+__device__ void jacobi_cta(float* S, float* V, int n, int ld, float* rc, float* rs, int* pq,
+                           int* flag) {
+  const int tid = threadIdx.x, nt = blockDim.x, h = n / 2;
+  for (int e = tid; e < n * ld; e += nt) V[e] = (e % ld == e / ld) ? 1.f : 0.f;
   __syncthreads();
-
-  // cyclic Jacobi, round-robin pairing: in step t of a sweep, pair 0 is
-  // (t, D - 1) and pair k > 0 is ((t + k) mod (D - 1), (t - k) mod (D - 1));
-  // every unordered pair meets once per sweep of D - 1 steps
   for (int sweep = 0; sweep < JACOBI_MAX_SWEEPS; ++sweep) {
-    // stop when the off-diagonal mass is negligible against the diagonal
     if (tid < 32) {
       float off = 0.f, dia = 0.f;
-      for (int e = tid; e < D * D; e += 32) {
-        const int i = e / D, j = e % D;
-        const float x = S[i * DP + j];
+      for (int e = tid; e < n * n; e += 32) {
+        const int i = e / n, j = e % n;
+        const float x = S[i * ld + j];
         if (i == j) dia += x * x; else off += x * x;
       }
       off = warp_sum_f(off);
       dia = warp_sum_f(dia);
-      if (tid == 0) flags[0] = off <= 1e-12f * dia ? 1 : 0;
+      if (tid == 0) *flag = off <= 1e-12f * dia ? 1 : 0;
     }
     __syncthreads();
-    if (flags[0]) break;
-    for (int t = 0; t < D - 1; ++t) {
-      if (tid < H) {
+    if (*flag) break;
+    for (int t = 0; t < n - 1; ++t) {
+      if (tid < h) {
         int p, q;
         if (tid == 0) {
-          p = t; q = D - 1;
+          p = t; q = n - 1;
         } else {
-          p = (t + tid) % (D - 1);
-          q = (t - tid + (D - 1)) % (D - 1);
+          p = (t + tid) % (n - 1);
+          q = (t - tid + (n - 1)) % (n - 1);
         }
         if (p > q) { const int x = p; p = q; q = x; }
-        const float apq = S[p * DP + q], app = S[p * DP + p], aqq = S[q * DP + q];
+        const float apq = S[p * ld + q], app = S[p * ld + p], aqq = S[q * ld + q];
         float c = 1.f, s = 0.f;
         if (fabsf(apq) > 1e-30f) {
           const float theta = (aqq - app) / (2.f * apq);
@@ -281,64 +284,285 @@ __global__ void __launch_bounds__(PB_THREADS) probe_eig_kernel(const ProbeArgs a
           c = rsqrtf(fmaf(tt, tt, 1.f));
           s = tt * c;
         }
-        pp[tid] = p; qq[tid] = q; rot_c[tid] = c; rot_s[tid] = s;
+        pq[2 * tid] = p; pq[2 * tid + 1] = q; rc[tid] = c; rs[tid] = s;
       }
       __syncthreads();
-      // columns: S <- S J, V <- V J
-      for (int e = tid; e < H * D; e += PB_THREADS) {
-        const int k = e / D, i = e % D;
-        const int p = pp[k], q = qq[k];
-        const float c = rot_c[k], s = rot_s[k];
-        const float sp = S[i * DP + p], sq = S[i * DP + q];
-        S[i * DP + p] = c * sp - s * sq;
-        S[i * DP + q] = s * sp + c * sq;
-        const float vp = V[i * DP + p], vq = V[i * DP + q];
-        V[i * DP + p] = c * vp - s * vq;
-        V[i * DP + q] = s * vp + c * vq;
+      for (int e = tid; e < h * n; e += nt) {   // columns: S <- S J, V <- V J
+        const int k = e / n, i = e % n;
+        const int p = pq[2 * k], q = pq[2 * k + 1];
+        const float c = rc[k], s = rs[k];
+        const float sp = S[i * ld + p], sq = S[i * ld + q];
+        S[i * ld + p] = c * sp - s * sq;
+        S[i * ld + q] = s * sp + c * sq;
+        const float vp = V[i * ld + p], vq = V[i * ld + q];
+        V[i * ld + p] = c * vp - s * vq;
+        V[i * ld + q] = s * vp + c * vq;
       }
       __syncthreads();
-      // rows: S <- J^T S
-      for (int e = tid; e < H * D; e += PB_THREADS) {
-        const int k = e / D, j = e % D;
-        const int p = pp[k], q = qq[k];
-        const float c = rot_c[k], s = rot_s[k];
-        const float sp = S[p * DP + j], sq = S[q * DP + j];
-        S[p * DP + j] = c * sp - s * sq;
-        S[q * DP + j] = s * sp + c * sq;
+      for (int e = tid; e < h * n; e += nt) {   // rows: S <- J^T S
+        const int k = e / n, j = e % n;
+        const int p = pq[2 * k], q = pq[2 * k + 1];
+        const float c = rc[k], s = rs[k];
+        const float sp = S[p * ld + j], sq = S[q * ld + j];
+        S[p * ld + j] = c * sp - s * sq;
+        S[q * ld + j] = s * sp + c * sq;
       }
       __syncthreads();
     }
   }
-  // eigenvalues; the r largest (ties: lower index) span the subspace
-  for (int i = tid; i < D; i += PB_THREADS) lam[i] = S[i * DP + i];
-  __syncthreads();
-  for (int i = tid; i < D; i += PB_THREADS) {
-    int rank = 0;
-    for (int j = 0; j < D; ++j) rank += (lam[j] > lam[i] || (lam[j] == lam[i] && j < i)) ? 1 : 0;
-    sel[i] = rank < a.r ? 1.f : 0.f;
+}
+
+// Columns of the r largest eigenvalues (diagonal of S after jacobi_cta; ties
+// to the lower index), copied from V into U (row stride D) in rank order.
+__device__ void top_vectors(const float* S, const float* V, int n, int ld, int r, float* U,
+                            int D, int* rank) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  for (int i = tid; i < n; i += nt) {
+    const float li = S[i * ld + i];
+    int k = 0;
+    for (int j = 0; j < n; ++j) {
+      const float lj = S[j * ld + j];
+      k += (lj > li || (lj == li && j < i)) ? 1 : 0;
+    }
+    rank[i] = k;
   }
   __syncthreads();
-  // P = V diag(sel) V^T into S
-  for (int e = tid; e < D * D; e += PB_THREADS) {
+  for (int e = tid; e < n * n; e += nt) {
+    const int row = e / n, col = e % n;
+    if (rank[col] < r) U[row * D + rank[col]] = V[row * ld + col];
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(SV_THREADS) probe_solve_kernel(const ProbeArgs a, const float* gp,
+                                                                 int slabs) {
+  using G = GramGeom<D>;
+  constexpr int DA = D + 1;
+  extern __shared__ __align__(16) float psm[];
+  const int bh = blockIdx.x, role = blockIdx.y, tid = threadIdx.x, nt = blockDim.x;
+  const float* gph = gp + (size_t)bh * slabs * G::ZW * G::ZW;
+  if (role == 0) {
+    // ---- ridge fit: (A^T A + lam diag(0, 1, ..., 1)) W = A^T R, W = [b; B]
+    float* Gm = psm;               // [DA][DA]
+    float* Cm = Gm + DA * DA;      // [DA][D], then Y, then W
+    int* bad = reinterpret_cast<int*>(Cm + DA * D);
+    for (int e = tid; e < DA * DA; e += nt) {
+      const int i = e / DA, j = e % DA;
+      Gm[e] = gram_at<D>(gph, slabs, i, j) + ((i == j && i > 0) ? a.lam : 0.f);
+    }
+    for (int e = tid; e < DA * D; e += nt) Cm[e] = gram_at<D>(gph, slabs, e / D, DA + e % D);
+    if (tid == 0) *bad = 0;
+    __syncthreads();
+    cholesky_cta(Gm, DA, DA, bad);
+    // L Y = C, then L^T W = Y, one row at a time; (column c, part) threads
+    // add strided parts of each row's sum, reduced over 8 lanes
+    const int c = tid >> 3, part = tid & 7;
+    const bool live = c < D;
+    for (int i = 0; i < DA; ++i) {
+      float s = 0.f;
+      if (live)
+        for (int k = part; k < i; k += 8) s = fmaf(Gm[i * DA + k], Cm[k * D + c], s);
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      s += __shfl_xor_sync(0xffffffffu, s, 4);
+      if (live && part == 0) Cm[i * D + c] = (Cm[i * D + c] - s) / Gm[i * DA + i];
+      __syncthreads();
+    }
+    for (int i = DA - 1; i >= 0; --i) {
+      float s = 0.f;
+      if (live)
+        for (int k = i + 1 + part; k < DA; k += 8) s = fmaf(Gm[k * DA + i], Cm[k * D + c], s);
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      s += __shfl_xor_sync(0xffffffffu, s, 4);
+      if (live && part == 0) Cm[i * D + c] = (Cm[i * D + c] - s) / Gm[i * DA + i];
+      __syncthreads();
+    }
+    const bool failed = *bad != 0;
+    if (failed && tid == 0) flag_error(a.ctrl, DEV_NUMERIC, bh);
+    float* w = a.w + (size_t)bh * DA * D;
+    for (int e = tid; e < DA * D; e += nt) w[e] = failed ? 0.f : Cm[e];
+    return;
+  }
+  // ---- residual subspace: the r leading eigenvectors of S = R^T R (the
+  // leading right singular vectors of R) into U [D][D] (first r columns)
+  const int r = a.r;
+  if (r <= 0 || r >= D) return;   // P = 0 or P = I: the fold needs no U
+  float* U = a.pu + (size_t)bh * D * D;
+  constexpr int DP = D + 1;
+  const int q = r + SUB_EXTRA;
+  if (q > SUB_MAXQ || q >= D) {
+    // Jacobi on the whole D x D matrix
+    float* S = psm;               // [D][DP]
+    float* V = S + D * DP;        // [D][DP]
+    float* rc = V + D * DP;       // [D / 2]
+    float* rs = rc + D / 2;       // [D / 2]
+    int* pq = reinterpret_cast<int*>(rs + D / 2);   // [D]
+    int* rank = pq + D;                              // [D]
+    int* flag = rank + D;
+    for (int e = tid; e < D * D; e += nt) S[(e / D) * DP + e % D] = gram_at<D>(gph, slabs, DA + e / D, DA + e % D);
+    __syncthreads();
+    jacobi_cta(S, V, D, DP, rc, rs, pq, flag);
+    top_vectors(S, V, D, DP, r, U, D, rank);
+    return;
+  }
+  // block subspace iteration with a Rayleigh-Ritz step: X (D x q, orthonormal
+  // columns) <- orth(S X), SUB_ITERS times from a fixed +-1 start; then the
+  // q x q matrix T = X^T S X is diagonalised by Jacobi and the r leading Ritz
+  // vectors X W are the basis.  The subspace error decays like
+  // (lambda_{q+1} / lambda_r)^SUB_ITERS.
+  constexpr int QM = SUB_MAXQ, QP = SUB_MAXQ + 1;
+  float* S = psm;                 // [D][DP]
+  float* X = S + D * DP;          // [D][QM]
+  float* Y = X + D * QM;          // [D][QM]
+  float* T = Y + D * QM;          // [QM][QP]: Gram of Y / Rayleigh quotient
+  float* W = T + QM * QP;         // [QM][QP]: Jacobi vectors
+  float* rc = W + QM * QP;        // [QM / 2]
+  float* rs = rc + QM / 2;        // [QM / 2]
+  int* pq = reinterpret_cast<int*>(rs + QM / 2);  // [QM]
+  int* rank = pq + QM;                             // [QM]
+  int* flag = rank + QM;
+  for (int e = tid; e < D * D; e += nt) S[(e / D) * DP + e % D] = gram_at<D>(gph, slabs, DA + e / D, DA + e % D);
+  for (int e = tid; e < D * q; e += nt) {
+    const int i = e / q, c = e % q;
+    // a fixed +-1 pattern from a multiplicative hash of (i, c): full column
+    // rank (an xor of per-row and per-column bits would give rank 1)
+    unsigned h = (unsigned)i * 0x9E3779B1u + (unsigned)c * 0x85EBCA77u;
+    h ^= h >> 15;
+    h *= 0x2C1B3C6Du;
+    h ^= h >> 12;
+    X[i * QM + c] = (h >> 31) ? 1.f : -1.f;
+  }
+  __syncthreads();
+  // Y <- S X
+  auto mul = [&]() {
+    for (int e = tid; e < D * q; e += nt) {
+      const int i = e / q, c = e % q;
+      float s0 = 0.f, s1 = 0.f;
+      for (int j = 0; j < D; j += 2) {
+        s0 = fmaf(S[i * DP + j], X[j * QM + c], s0);
+        s1 = fmaf(S[i * DP + j + 1], X[(j + 1) * QM + c], s1);
+      }
+      Y[i * QM + c] = s0 + s1;
+    }
+    __syncthreads();
+  };
+  // X <- Y L^-T with Y^T Y = L L^T (Cholesky QR); a column that has become
+  // dependent (tiny pivot) is set to zero
+  auto orth = [&]() {
+    for (int e = tid; e < q * q; e += nt) {
+      const int i = e / q, j = e % q;
+      float s = 0.f;
+      for (int k = 0; k < D; ++k) s = fmaf(Y[k * QM + i], Y[k * QM + j], s);
+      T[i * QP + j] = s;
+    }
+    __syncthreads();
+    if (tid < 32) {   // one warp: q x q Cholesky, lanes share each column update
+      float scale = 0.f;
+      for (int k = tid; k < q; k += 32) scale = fmaxf(scale, T[k * QP + k]);
+      scale = warp_max_f(scale);
+      for (int k = 0; k < q; ++k) {
+        float dkk = T[k * QP + k];
+        const bool dead = !(dkk > 1e-12f * fmaxf(scale, 1e-30f));
+        const float lkk = dead ? 0.f : sqrtf(dkk);
+        __syncwarp();
+        for (int i = k + 1 + tid; i < q; i += 32) T[i * QP + k] = dead ? 0.f : T[i * QP + k] / lkk;
+        if (tid == 0) T[k * QP + k] = lkk;
+        __syncwarp();
+        for (int e = tid; e < (q - k - 1) * (q - k - 1); e += 32) {
+          const int i = k + 1 + e / (q - k - 1), j = k + 1 + e % (q - k - 1);
+          if (j <= i) T[i * QP + j] = fmaf(-T[i * QP + k], T[j * QP + k], T[i * QP + j]);
+        }
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < D; i += nt) {   // row i: x L^T = y, forward substitution
+      for (int c = 0; c < q; ++c) {
+        float s = Y[i * QM + c];
+        for (int k = 0; k < c; ++k) s = fmaf(-X[i * QM + k], T[c * QP + k], s);
+        const float lcc = T[c * QP + c];
+        X[i * QM + c] = lcc > 0.f ? s / lcc : 0.f;
+      }
+    }
+    __syncthreads();
+  };
+  for (int it = 0; it < SUB_ITERS; ++it) {
+    mul();
+    orth();
+  }
+  mul();   // Y = S X; T = X^T Y
+  for (int e = tid; e < q * q; e += nt) {
+    const int i = e / q, j = e % q;
+    float s = 0.f;
+    for (int k = 0; k < D; ++k) s = fmaf(X[k * QM + i], Y[k * QM + j], s);
+    T[i * QP + j] = s;
+  }
+  __syncthreads();
+  // symmetrise, pad to an even size for the round-robin pairing
+  const int qe = (q + 1) & ~1;
+  for (int e = tid; e < qe * qe; e += nt) {
+    const int i = e / qe, j = e % qe;
+    if (i >= q || j >= q) T[i * QP + j] = (i == j) ? -1.f : 0.f;   // below every Ritz value (>= 0)
+    else if (i < j) { const float v = 0.5f * (T[i * QP + j] + T[j * QP + i]); T[i * QP + j] = v; T[j * QP + i] = v; }
+  }
+  __syncthreads();
+  jacobi_cta(T, W, qe, QP, rc, rs, pq, flag);
+  __syncthreads();
+  // rank the Ritz values; U[:, k] = X W[:, col of rank k], k < r
+  for (int i = tid; i < qe; i += nt) {
+    const float li = T[i * QP + i];
+    int k = 0;
+    for (int j = 0; j < qe; ++j) {
+      const float lj = T[j * QP + j];
+      k += (lj > li || (lj == li && j < i)) ? 1 : 0;
+    }
+    rank[i] = k;
+  }
+  __syncthreads();
+  for (int e = tid; e < D * qe; e += nt) {
+    const int row = e / qe, col = e % qe;
+    if (rank[col] < r && col < q) {
+      float s = 0.f;
+      for (int k = 0; k < q; ++k) s = fmaf(X[row * QM + k], W[k * QP + col], s);
+      U[row * D + rank[col]] = s;
+    }
+  }
+}
+
+// B P and b P with P = U U^T (U: the first r columns), or P = 0 / I for
+// r = 0 / r >= D; one CTA per head.
+template <int D>
+__global__ void __launch_bounds__(PB_THREADS) probe_fold_kernel(const ProbeArgs a) {
+  extern __shared__ __align__(16) float psm[];
+  const int bh = blockIdx.x, tid = threadIdx.x;
+  const int r = a.r;
+  const float* wfit = a.w + (size_t)bh * (D + 1) * D;   // row 0 = b, rows 1.. = B
+  float* wp = a.wp + (size_t)bh * D * D;
+  float* cp = a.cp + (size_t)bh * D;
+  if (r <= 0 || r >= D) {
+    const bool full = r >= D;
+    for (int e = tid; e < D * D; e += PB_THREADS) wp[e] = full ? wfit[D + e] : 0.f;
+    for (int c = tid; c < D; c += PB_THREADS) cp[c] = full ? wfit[c] : 0.f;
+    return;
+  }
+  float* Us = psm;                 // [D][r]
+  float* BU = Us + D * r;          // [D + 1][r]: row 0 = b U, rows 1.. = B U
+  const float* U = a.pu + (size_t)bh * D * D;
+  for (int e = tid; e < D * r; e += PB_THREADS) Us[e] = U[(e / r) * D + e % r];
+  __syncthreads();
+  for (int e = tid; e < (D + 1) * r; e += PB_THREADS) {
+    const int i = e / r, k = e % r;
+    float s = 0.f;
+    for (int j = 0; j < D; ++j) s = fmaf(wfit[i * D + j], Us[j * r + k], s);
+    BU[e] = s;
+  }
+  __syncthreads();
+  for (int e = tid; e < (D + 1) * D; e += PB_THREADS) {
     const int i = e / D, j = e % D;
     float s = 0.f;
-    for (int k = 0; k < D; ++k) s = fmaf(sel[k] * V[i * DP + k], V[j * DP + k], s);
-    S[i * DP + j] = s;
-  }
-  __syncthreads();
-  // B into V's space, then B P and b P
-  for (int e = tid; e < D * D; e += PB_THREADS) V[(e / D) * DP + e % D] = wfit[D + e];
-  __syncthreads();
-  for (int e = tid; e < D * D; e += PB_THREADS) {
-    const int i = e / D, j = e % D;
-    float s = 0.f;
-    for (int k = 0; k < D; ++k) s = fmaf(V[i * DP + k], S[k * DP + j], s);
-    wp[e] = s;
-  }
-  for (int j = tid; j < D; j += PB_THREADS) {
-    float s = 0.f;
-    for (int k = 0; k < D; ++k) s = fmaf(wfit[k], S[k * DP + j], s);
-    cp[j] = s;
+    for (int k = 0; k < r; ++k) s = fmaf(BU[i * r + k], Us[j * r + k], s);
+    if (i == 0) cp[j] = s; else wp[(i - 1) * D + j] = s;
   }
 }
 
@@ -389,19 +613,28 @@ __global__ void __launch_bounds__(D) probe_set_kernel(const ProbeArgs a) {
 }
 
 template <int D>
+size_t fold_smem_bytes() {
+  return ((size_t)D * (D - 1) + (size_t)(D + 1) * (D - 1)) * sizeof(float);
+}
+
+template <int D>
 cudaError_t launch_probe_d(const Problem& p, const ProbeArgs& a, int m_alloc, __nv_bfloat16* qg,
-                           cudaStream_t s) {
+                           float* gp, cudaStream_t s) {
   cudaError_t e;
-  if ((e = ensure_dyn_smem((const void*)probe_fit_kernel<D>, fit_smem_bytes<D>())) != cudaSuccess) return e;
-  if ((e = ensure_dyn_smem((const void*)probe_eig_kernel<D>, eig_smem_bytes<D>())) != cudaSuccess) return e;
+  if ((e = ensure_dyn_smem((const void*)probe_solve_kernel<D>, solve_smem_bytes<D>())) != cudaSuccess) return e;
+  if ((e = ensure_dyn_smem((const void*)probe_fold_kernel<D>, fold_smem_bytes<D>())) != cudaSuccess) return e;
   if ((e = ensure_dyn_smem((const void*)probe_apply_kernel<D>, apply_smem_bytes<D>())) != cudaSuccess) return e;
   const int gather_blocks = (m_alloc * (D / 8) + PB_THREADS - 1) / PB_THREADS;
   probe_gather_kernel<D><<<dim3(gather_blocks, a.BH), PB_THREADS, 0, s>>>(a, m_alloc, qg);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = launch_dense_rows_tc(p, qg, m_alloc, a.M, a.k, a.v, a.od, a.ctrl, s)) != cudaSuccess) return e;
-  probe_fit_kernel<D><<<a.BH, PB_THREADS, fit_smem_bytes<D>(), s>>>(a);
+  const int slabs = gram_slabs(a.M);
+  probe_gram_kernel<D><<<dim3(slabs, a.BH), GR_THREADS, 0, s>>>(a, gp, slabs);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  probe_eig_kernel<D><<<a.BH, PB_THREADS, eig_smem_bytes<D>(), s>>>(a);
+  probe_solve_kernel<D><<<dim3(a.BH, 2), SV_THREADS, solve_smem_bytes<D>(), s>>>(a, gp, slabs);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t fold_smem = a.r > 0 && a.r < D ? ((size_t)D * a.r + (size_t)(D + 1) * a.r) * sizeof(float) : 0;
+  probe_fold_kernel<D><<<a.BH, PB_THREADS, fold_smem, s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   probe_apply_kernel<D><<<dim3((a.N + PA_ROWS - 1) / PA_ROWS, a.BH), PB_THREADS, apply_smem_bytes<D>(), s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -414,11 +647,15 @@ cudaError_t launch_probe_d(const Problem& p, const ProbeArgs& a, int m_alloc, __
 // Probe queries are gathered into whole 128-row tiles.
 inline int probe_rows_alloc(int M) { return (M + 127) / 128 * 128; }
 
+// Padded width of a head's Gram matrix of [1, x, R] (a multiple of 4).
+inline size_t gram_width(int d) { return (size_t)(1 + 2 * d + 3) / 4 * 4; }
+
 size_t probe_scratch_bytes(const Problem& p, int M) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-  const size_t BH = (size_t)p.BH, d = (size_t)p.d;
+  const size_t BH = (size_t)p.BH, d = (size_t)p.d, zw = gram_width(p.d);
   return up(BH * M * d * 4) + up(BH * (d + 1) * d * 4) + up(BH * d * d * 4) + up(BH * d * 4) +
-         up(BH * probe_rows_alloc(M) * d * 2);
+         up(BH * probe_rows_alloc(M) * d * 2) + up(BH * d * d * 4) +
+         up(BH * (size_t)gram_slabs(M) * zw * zw * 4);
 }
 
 cudaError_t launch_probe_correct(const Problem& p, const void* Q, const void* K, const void* V,
@@ -438,12 +675,14 @@ cudaError_t launch_probe_correct(const Problem& p, const void* Q, const void* K,
   a.w = reinterpret_cast<float*>(b + off);  off += up(BH * (d + 1) * d * 4);
   a.wp = reinterpret_cast<float*>(b + off); off += up(BH * d * d * 4);
   a.cp = reinterpret_cast<float*>(b + off); off += up(BH * d * 4);
-  __nv_bfloat16* qg = reinterpret_cast<__nv_bfloat16*>(b + off);
+  const int m_alloc = probe_rows_alloc(M);
+  __nv_bfloat16* qg = reinterpret_cast<__nv_bfloat16*>(b + off); off += up(BH * m_alloc * d * 2);
+  a.pu = reinterpret_cast<float*>(b + off); off += up(BH * d * d * 4);
+  float* gp = reinterpret_cast<float*>(b + off);
   a.ctrl = ctrl;
   a.N = p.N; a.M = M; a.BH = p.BH; a.r = r; a.lam = lam;
-  const int m_alloc = probe_rows_alloc(M);
-  return p.d == 128 ? launch_probe_d<128>(p, a, m_alloc, qg, s)
-                    : launch_probe_d<64>(p, a, m_alloc, qg, s);
+  return p.d == 128 ? launch_probe_d<128>(p, a, m_alloc, qg, gp, s)
+                    : launch_probe_d<64>(p, a, m_alloc, qg, gp, s);
 }
 
 }  // namespace spattn
