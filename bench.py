@@ -88,6 +88,9 @@ def parse_args(argv=None):
     ap.add_argument("--selection", choices=["top_p", "threshold"], default="top_p",
                     help="Top-p on the cumulative mass (tau), or a per-block threshold on p "
                          "(Sol-Attn on-the-fly thresholding; the knob is --theta)")
+    ap.add_argument("--inline", action="store_true",
+                    help="select inside the attention kernel (SPATTN_SELECT_INLINE): the step is "
+                         "pooling + attention, with the same kept blocks")
     ap.add_argument("--theta", type=float, default=0.01,
                     help="per-block probability threshold with --selection threshold")
     ap.add_argument("--no-probe", action="store_true",
@@ -343,7 +346,8 @@ def run_reference(args):
         "ms_per_step": 1e3 * float(np.mean(times)), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         # the GPU arm's config, so that the two lines describe the same workload
-        "config": dict(config_of(w, L2_NOTE), routing=args.routing, selection=args.selection),
+        "config": dict(config_of(w, L2_NOTE), routing=args.routing, selection=args.selection,
+                       inline_selection=bool(args.inline)),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": "each step: " + desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -468,6 +472,10 @@ def run_ours(args):
     routing = sp.ROUTING_PAMA if args.routing == "pama" else sp.ROUTING_CENTROID
     if args.selection == "threshold":
         routing |= sp.SELECT_THRESHOLD
+    if args.inline:
+        if args.routing == "pama":
+            raise SystemExit("--inline selects from the centroid estimate")
+        routing |= sp.SELECT_INLINE
     plan = sp.Plan(B, H, N, d, w.b, w.tau, w.kmin, w.kmax, w.residual, perm, device=dev,
                    routing=routing)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -538,7 +546,11 @@ def run_ours(args):
 
     clocks = ClockSampler(local)
     clocks.start()
-    t = timed([as_graph(lambda: plan.route(q, k, v)), as_graph(lambda: plan.attend(q, k, v, o))],
+    # the step: routing (pooling, proxy, selection, work order) then the
+    # attention; with --inline, pooling then the attention, which selects
+    # the same blocks itself
+    first = (lambda: plan.pool(q, k, v)) if args.inline else (lambda: plan.route(q, k, v))
+    t = timed([as_graph(first), as_graph(lambda: plan.attend(q, k, v, o))],
               args.steps, args.warmup)
     clk = clocks.stop()
     route_ms = float(np.mean([x[0] for x in t]))
@@ -751,7 +763,8 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": dict(config_of(w, L2_NOTE),
-                           routing=args.routing, selection=args.selection),
+                           routing=args.routing, selection=args.selection,
+                           inline_selection=bool(args.inline)),
             "dense_equiv_tflops": dense_flops * world / (step_ms * 1e-3) / 1e12,
             "attn_tflops": attn_tflops,
             "pct_of_bf16_peak": 100.0 * attn_tflops / bf16_peak,
@@ -787,7 +800,8 @@ def run_ours(args):
             "per_config": per_config,
             "threshold_selection": thresh,
             "probe_correction": probe,
-            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            # pool, route, scan, attend; pool and attend with --inline
+            "gpu_launches": (2 if args.inline else KERNELS_PER_STEP) * args.steps,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

@@ -58,6 +58,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstddef>
 #include <type_traits>
 
 #include "common.cuh"
@@ -71,6 +72,16 @@ namespace {
 // SPATTN_EXP_EMU of every 8 pairs of exponentials run on the FMA pipe
 // (tc::ex2_fma2) instead of the MUFU unit (0: all on MUFU, the fastest
 // setting measured for this kernel).
+// The two softmax warps that share a scheduler (same lane quarter, key
+// halves 0 and 1) would otherwise load S, wait and store P in lockstep, with
+// the MUFU idle meanwhile.  With SPATTN_STAGGER = 1 the half-1 warp starts
+// loading S(g) only once its half-0 partner has loaded its own columns, so
+// that one warp's TMEM traffic overlaps the other's exponentials (0: no
+// handoff).  The arithmetic is the same either way.
+#ifndef SPATTN_STAGGER
+#define SPATTN_STAGGER 1
+#endif
+
 #ifndef SPATTN_EXP_EMU
 #define SPATTN_EXP_EMU 0
 #endif
@@ -103,7 +114,8 @@ enum : int {
   B_INFO_FULL0, B_INFO_FULL1,    // item slot s described by the producer warp
   B_INFO_EMPTY0, B_INFO_EMPTY1,  // item slot s released by the MMA and softmax warps
   B_XREADY,                // + 4 * slot + quarter: both key halves of a lane quarter merged
-  B_RING = B_XREADY + 8,   // full[s] at B_RING + s, empty[s] at B_RING + STAGES + s
+  B_HAND = B_XREADY + 8,   // + 4 * (g & 1) + quarter: the half-0 warp has loaded S(g)
+  B_RING = B_HAND + 8,     // full[s] at B_RING + s, empty[s] at B_RING + STAGES + s
 };
 
 struct TcArgs {
@@ -155,8 +167,8 @@ struct __align__(8) TcCtrl {
   uint32_t tmem_base;
   int abort;
   ItemInfo info[2];
-  float selp[2048];           // inline selection: the proxy / probability row
-  float selq[128];            // inline selection: the query block's mean
+  alignas(16) float selp[2048];  // inline selection: the proxy / probability row
+  alignas(16) float selq[128];   // inline selection: the query block's mean (float4 access)
   float xm[2][2][TILE_ROWS];  // epilogue, per item slot: reference max of each key half
   float xl[2][2][TILE_ROWS];  // epilogue, per item slot: sum of each key half
 };
@@ -254,6 +266,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc::mbar_init(bar(B_INFO_EMPTY0 + s), 1 + NUM_SOFTMAX_WARPS);
     }
     for (int q = 0; q < 8; ++q) tc::mbar_init(bar(B_XREADY + q), 64);
+    for (int q = 0; q < 8; ++q) tc::mbar_init(bar(B_HAND + q), 1);
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(full(s), 1);
       tc::mbar_init(empty(s), 1);
@@ -661,7 +674,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
           }
         };
+        // staggered start (SPATTN_STAGGER): the handoff barrier of task g has
+        // two slots (g & 1), so its phase parity (g >> 1) & 1 names task g
+        // alone: the half-0 warp cannot be two tasks ahead, because S(g + 2)
+        // needs P(g) from both halves first
+        if (SPATTN_STAGGER && half == 1 &&
+            !(ok = wait_warp(bar(B_HAND + 4 * b + quarter), (uint32_t)(g >> 1) & 1u, 16)))
+          break;
         load_s();
+        if (SPATTN_STAGGER && half == 0) {
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(bar(B_HAND + 4 * b + quarter));
+        }
         auto tile_max = [&]() {
           float mx[8];
 #pragma unroll
@@ -900,6 +924,11 @@ bool make_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH, int box 
   e.used = true;
   return true;
 }
+
+// the control block starts 1024-byte aligned (after the tiles); the members
+// read or written as float4 must sit on 16-byte offsets inside it
+static_assert(offsetof(TcCtrl, selq) % 16 == 0 && offsetof(TcCtrl, selp) % 16 == 0,
+              "float4 scratch of the inline selection must be 16-byte aligned");
 
 template <int D>
 constexpr size_t tc_smem_bytes() {
