@@ -66,6 +66,10 @@ struct Layout {
       ctrl, total;
 };
 
+// Permuted copies of Q, K and V are made only for the warp-MMA cross-check
+// kernel; the tcgen05 kernel gathers rows through the permutation itself.
+bool keeps_copies(const Problem& p) { return p.perm != nullptr && !p.use_tc; }
+
 Layout make_layout(const Problem& p) {
   Layout L;
   size_t off = 0;
@@ -73,7 +77,7 @@ Layout make_layout(const Problem& p) {
   const size_t tok = (size_t)p.BH * p.N * p.d;
   const size_t cen = (size_t)p.BH * p.nb * p.d;
   const size_t rows = (size_t)p.BH * p.nb;
-  const bool perm = p.perm != nullptr;
+  const bool perm = keeps_copies(p);
   L.qp = perm ? take(tok * 2) : 0;
   L.kp = perm ? take(tok * 2) : 0;
   L.vp = perm ? take(tok * 2) : 0;
@@ -95,7 +99,7 @@ Layout make_layout(const Problem& p) {
 Work bind(const Problem& p, const Layout& L, void* ws) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   Work w;
-  const bool perm = p.perm != nullptr;
+  const bool perm = keeps_copies(p);
   w.qp = perm ? reinterpret_cast<__nv_bfloat16*>(b + L.qp) : nullptr;
   w.kp = perm ? reinterpret_cast<__nv_bfloat16*>(b + L.kp) : nullptr;
   w.vp = perm ? reinterpret_cast<__nv_bfloat16*>(b + L.vp) : nullptr;
@@ -261,6 +265,12 @@ spattn_status_t spattn_plan_ex(spattn_plan_t* out, int B, int H, int N, int d, i
     p.use_tc = spattn::attend_tc_supported(p) && !(env && strcmp(env, "mma") == 0);
     // the inline selection lives in the tcgen05 kernel
     if (p.inline_sel && !p.use_tc) { delete P; return fail(SPATTN_ERR_UNSUPPORTED, "SPATTN_SELECT_INLINE needs the tcgen05 attention kernel"); }
+    // with a permutation the tcgen05 kernel gathers rows of the [B*H*N, d]
+    // matrices by int32 row index
+    if (perm_host && p.use_tc && (long long)B * H * N > 0x7FFFFFFFLL) {
+      delete P;
+      return fail(SPATTN_ERR_UNSUPPORTED, "with a permutation B*H*N must stay below 2^31");
+    }
     // Failure-path test: with SPATTN_TEST_WAIT_TIMEOUT=1 in the environment
     // when the plan is made, the tcgen05 attention's first CTA waits on an
     // mbarrier phase that nothing completes; the bounded wait gives up after

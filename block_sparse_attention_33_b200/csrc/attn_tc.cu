@@ -72,16 +72,6 @@ namespace {
 // SPATTN_EXP_EMU of every 8 pairs of exponentials run on the FMA pipe
 // (tc::ex2_fma2) instead of the MUFU unit (0: all on MUFU, the fastest
 // setting measured for this kernel).
-// The two softmax warps that share a scheduler (same lane quarter, key
-// halves 0 and 1) would otherwise load S, wait and store P in lockstep, with
-// the MUFU idle meanwhile.  With SPATTN_STAGGER = 1 the half-1 warp starts
-// loading S(g) only once its half-0 partner has loaded its own columns, so
-// that one warp's TMEM traffic overlaps the other's exponentials (0: no
-// handoff).  The arithmetic is the same either way.
-#ifndef SPATTN_STAGGER
-#define SPATTN_STAGGER 1
-#endif
-
 #ifndef SPATTN_EXP_EMU
 #define SPATTN_EXP_EMU 0
 #endif
@@ -114,8 +104,7 @@ enum : int {
   B_INFO_FULL0, B_INFO_FULL1,    // item slot s described by the producer warp
   B_INFO_EMPTY0, B_INFO_EMPTY1,  // item slot s released by the MMA and softmax warps
   B_XREADY,                // + 4 * slot + quarter: both key halves of a lane quarter merged
-  B_HAND = B_XREADY + 8,   // + 4 * (g & 1) + quarter: the half-0 warp has loaded S(g)
-  B_RING = B_HAND + 8,     // full[s] at B_RING + s, empty[s] at B_RING + STAGES + s
+  B_RING = B_XREADY + 8,   // full[s] at B_RING + s, empty[s] at B_RING + STAGES + s
 };
 
 struct TcArgs {
@@ -138,6 +127,8 @@ struct TcArgs {
   const float *qbar, *kbar;  // fp32 means [BH, nb, d]
   float tau;                 // Top-p mass, or the per-block threshold theta
   int threshold, kmin;
+  int gather;      // a token permutation: Q, K and V rows are gathered through perm
+                   // (tmQ, tmK, tmV are then 2-D row maps [BH * N, D], box 64 x 1)
   int b64;         // 64-token blocks: a tile holds two query (key) blocks
   int nq;          // query tiles per (batch, head): nb (b = 128) or ceil(nb / 2) (b = 64)
   int blk;         // block size b
@@ -195,25 +186,36 @@ __device__ __noinline__ void select_inline(const SelArgs a, int row, uint32_t* k
   const float inv_sqrt_d = 1.0f / sqrtf((float)D);
   const int tpj = sel::proxy_threads_per_block(a.nb);
   const int sub = lane % tpj, grp = lane / tpj, ngrp = 32 / tpj;
-  for (int j0 = 0; j0 < a.nb; j0 += ngrp) {
-    const int j = j0 + grp;
-    const bool live = j < a.nb;
-    float acc = 0.f;
-    if (live) {
-      const float4* kr = reinterpret_cast<const float4*>(kb + (size_t)j * D);
-      for (int k4 = sub; k4 < D / 4; k4 += tpj) {
-        const float4 kv = __ldg(kr + k4);
-        const float4 q = reinterpret_cast<const float4*>(selq)[k4];
-        acc = fmaf(q.x, kv.x, acc);
-        acc = fmaf(q.y, kv.y, acc);
-        acc = fmaf(q.z, kv.z, acc);
-        acc = fmaf(q.w, kv.w, acc);
-      }
+  // two key blocks per lane at a time and an unrolled channel loop, so that
+  // a lane keeps many independent loads of Kbar in flight (one warp reads the
+  // whole Kbar of the head); each block's sum keeps the routing kernel's order
+  const float4* q4 = reinterpret_cast<const float4*>(selq);
+  for (int j0 = 0; j0 < a.nb; j0 += 2 * ngrp) {
+    const int ja = j0 + grp, jb = ja + ngrp;
+    const bool la = ja < a.nb, lb = jb < a.nb;
+    const float4* ka = reinterpret_cast<const float4*>(kb + (size_t)(la ? ja : 0) * D);
+    const float4* kc = reinterpret_cast<const float4*>(kb + (size_t)(lb ? jb : 0) * D);
+    float acc_a = 0.f, acc_b = 0.f;
+#pragma unroll 8
+    for (int k4 = sub; k4 < D / 4; k4 += tpj) {
+      const float4 va = __ldg(ka + k4), vb = __ldg(kc + k4);
+      const float4 q = q4[k4];
+      acc_a = fmaf(q.x, va.x, acc_a);
+      acc_a = fmaf(q.y, va.y, acc_a);
+      acc_a = fmaf(q.z, va.z, acc_a);
+      acc_a = fmaf(q.w, va.w, acc_a);
+      acc_b = fmaf(q.x, vb.x, acc_b);
+      acc_b = fmaf(q.y, vb.y, acc_b);
+      acc_b = fmaf(q.z, vb.z, acc_b);
+      acc_b = fmaf(q.w, vb.w, acc_b);
     }
-    for (int o = 1; o < tpj; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (live && sub == 0) {
-      const int nj = (j == a.nb - 1) ? a.n_last : a.blk;
-      selp[j] = fmaf(acc, inv_sqrt_d, logf((float)nj));
+    for (int o = 1; o < tpj; o <<= 1) {
+      acc_a += __shfl_xor_sync(0xffffffffu, acc_a, o);
+      acc_b += __shfl_xor_sync(0xffffffffu, acc_b, o);
+    }
+    if (sub == 0) {
+      if (la) selp[ja] = fmaf(acc_a, inv_sqrt_d, logf((float)(ja == a.nb - 1 ? a.n_last : a.blk)));
+      if (lb) selp[jb] = fmaf(acc_b, inv_sqrt_d, logf((float)(jb == a.nb - 1 ? a.n_last : a.blk)));
     }
   }
   __syncwarp();
@@ -266,7 +268,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc::mbar_init(bar(B_INFO_EMPTY0 + s), 1 + NUM_SOFTMAX_WARPS);
     }
     for (int q = 0; q < 8; ++q) tc::mbar_init(bar(B_XREADY + q), 64);
-    for (int q = 0; q < 8; ++q) tc::mbar_init(bar(B_HAND + q), 1);
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(full(s), 1);
       tc::mbar_init(empty(s), 1);
@@ -409,48 +410,74 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       __syncwarp();
       tc::mbar_arrive(bar(B_INFO_FULL0 + slot));   // every lane: releases its own writes
       if (T == 0) continue;
-      if (lane == 0) {
-        if (qn > 0)
-          ok = tc::mbar_wait_fast(bar(B_QEMPTY), (uint32_t)(qn - 1) & 1u, abort, a.ctrl, 12);
-        if (ok) {
-          tc::mbar_expect_tx(bar(B_QFULL), TILE_BYTES);
+      // Loads.  Lane 0 makes every wait and sets every transaction count;
+      // the tile loads are TMA boxes issued by lane 0, or, with a token
+      // permutation, row gathers through it issued by all lanes (lane l: tile
+      // rows 4l .. 4l + 3; a row past the last token repeats token N - 1).
+      auto gather_tile = [&](uint32_t dst, const CUtensorMap* m, uint32_t fb, int tok0, int tok1) {
+        // tok0: first token (permuted order) of tile rows 0-63, tok1: of rows 64-127
+        const int r0 = 4 * lane;
+        const int tok = (r0 < 64 ? tok0 : tok1) + (r0 & 63);
+        int rows[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) rows[k] = bh * a.N + __ldg(a.perm + min(tok + k, a.N - 1));
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
+          tc::tma_gather4(dst + c * CHUNK_BYTES + r0 * 128, m, fb, c * 64, rows[0], rows[1], rows[2], rows[3]);
+      };
+      if (lane == 0 && qn > 0)
+        ok = tc::mbar_wait_fast(bar(B_QEMPTY), (uint32_t)(qn - 1) & 1u, abort, a.ctrl, 12);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (ok) {
+        if (lane == 0) tc::mbar_expect_tx(bar(B_QFULL), TILE_BYTES);
+        if (a.gather) {
+          __syncwarp();
+          gather_tile(sQ, &tmQ, bar(B_QFULL), i * TILE_ROWS, i * TILE_ROWS + 64);
+        } else if (lane == 0) {
 #pragma unroll
           for (int c = 0; c < NCH; ++c)
             tc::tma_load_3d(sQ + c * CHUNK_BYTES, &tmQ, bar(B_QFULL), c * 64, i * TILE_ROWS, bh);
         }
-        auto issue = [&](int t, bool is_v) -> bool {
-          const CUtensorMap* m;
-          int row, row2 = -1;   // row2: b = 64, first token of the tile's second key block
-          if (t < nkept) {
-            m = is_v ? &tmV : &tmK;
-            if (a.b64) {
-              // an absent second block repeats the first (valid data, masked
-              // by the softmax)
-              const int j0 = inf.ublk[2 * t];
-              const int j1 = 2 * t + 1 < inf.nunion ? inf.ublk[2 * t + 1] : j0;
-              row = j0 * 64;
-              row2 = j1 * 64;
-            } else if (a.dense) {
-              row = t * TILE_ROWS;
-            } else if (a.inline_sel) {
-              row = inf.ublk[t] * TILE_ROWS;
-            } else {
-              int j = __ldg(a.col_idx + r_lo + t);
-              if (j < 0 || j >= a.nb) {
-                flag_error(a.ctrl, DEV_BAD_INDEX, item);
-                j = 0;  // load something valid; the softmax masks the whole task
-              }
-              row = j * TILE_ROWS;
-            }
+      }
+      auto issue = [&](int t, bool is_v) -> bool {
+        const CUtensorMap* m;
+        int row, row2 = -1;   // first token of tile rows 0-.. and, with b = 64, of rows 64-127
+        if (t < nkept) {
+          m = is_v ? &tmV : &tmK;
+          if (a.b64) {
+            // an absent second block repeats the first (valid data, masked
+            // by the softmax)
+            const int j0 = inf.ublk[2 * t];
+            const int j1 = 2 * t + 1 < inf.nunion ? inf.ublk[2 * t + 1] : j0;
+            row = j0 * 64;
+            row2 = j1 * 64;
+          } else if (a.dense) {
+            row = t * TILE_ROWS;
+          } else if (a.inline_sel) {
+            row = inf.ublk[t] * TILE_ROWS;
           } else {
-            m = is_v ? &tmVb : &tmKb;
-            row = res_tile(res_tiles, t - nkept) * TILE_ROWS;
+            int j = __ldg(a.col_idx + r_lo + t);
+            if (j < 0 || j >= a.nb) {
+              if (lane == 0) flag_error(a.ctrl, DEV_BAD_INDEX, item);
+              j = 0;  // load something valid; the softmax masks the whole task
+            }
+            row = j * TILE_ROWS;
           }
-          const int s = li % STAGES;
-          if (!tc::mbar_wait_fast(empty(s), ((uint32_t)(li / STAGES) & 1u) ^ 1u, abort, a.ctrl, 1))
-            return false;
-          tc::mbar_expect_tx(full(s), TILE_BYTES);
-          const uint32_t dst = sRing + s * TILE_BYTES;
+        } else {
+          m = is_v ? &tmVb : &tmKb;
+          row = res_tile(res_tiles, t - nkept) * TILE_ROWS;
+        }
+        const int s = li % STAGES;
+        bool free_slot = true;
+        if (lane == 0)
+          free_slot = tc::mbar_wait_fast(empty(s), ((uint32_t)(li / STAGES) & 1u) ^ 1u, abort, a.ctrl, 1);
+        if (!__shfl_sync(0xffffffffu, free_slot, 0)) return false;
+        if (lane == 0) tc::mbar_expect_tx(full(s), TILE_BYTES);
+        const uint32_t dst = sRing + s * TILE_BYTES;
+        if (a.gather && t < nkept) {
+          __syncwarp();
+          gather_tile(dst, m, full(s), row, row2 < 0 ? row + 64 : row2);
+        } else if (lane == 0) {
           if (row2 < 0) {
 #pragma unroll
             for (int c = 0; c < NCH; ++c) tc::tma_load_3d(dst + c * CHUNK_BYTES, m, full(s), c * 64, row, bh);
@@ -462,18 +489,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               tc::tma_load_3d(dst + c * CHUNK_BYTES + 64 * 128, m, full(s), c * 64, row2, bh);
             }
           }
-          ++li;
-          return true;
-        };
-        if (ok) ok = issue(0, false);
-        if (ok && T > 1) ok = issue(1, false);
-        for (int t = 0; ok && t < T; ++t) {
-          ok = issue(t, true);
-          if (ok && t + 2 < T) ok = issue(t + 2, false);
         }
+        ++li;
+        return true;
+      };
+      if (ok) ok = issue(0, false);
+      if (ok && T > 1) ok = issue(1, false);
+      for (int t = 0; ok && t < T; ++t) {
+        ok = issue(t, true);
+        if (ok && t + 2 < T) ok = issue(t + 2, false);
       }
       ++qn;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
     }
     if (lane == 0) {
@@ -674,18 +700,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
           }
         };
-        // staggered start (SPATTN_STAGGER): the handoff barrier of task g has
-        // two slots (g & 1), so its phase parity (g >> 1) & 1 names task g
-        // alone: the half-0 warp cannot be two tasks ahead, because S(g + 2)
-        // needs P(g) from both halves first
-        if (SPATTN_STAGGER && half == 1 &&
-            !(ok = wait_warp(bar(B_HAND + 4 * b + quarter), (uint32_t)(g >> 1) & 1u, 16)))
-          break;
         load_s();
-        if (SPATTN_STAGGER && half == 0) {
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(bar(B_HAND + 4 * b + quarter));
-        }
         auto tile_max = [&]() {
           float mx[8];
 #pragma unroll
@@ -891,6 +906,20 @@ bool encode_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH, int bo
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows, D] bf16 matrix as a 2-D map for row gathers: box = 64 channels x 1
+// row, 128-byte swizzle (rows land as consecutive 128-byte box rows).
+bool encode_rows_map(CUtensorMap* m, const void* ptr, int D, long long rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // A tensor map depends only on (pointer, D, rows, BH, box rows): the last few
 // encoded maps of each host thread are kept so repeated calls on the same
 // buffers skip the driver's encode.
@@ -904,6 +933,7 @@ struct MapEntry {
   bool used;
 };
 
+// box = 0 asks for the 2-D row-gather map of [BH * rows, D].
 bool make_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH, int box = TILE_ROWS) {
   constexpr int SLOTS = 16;
   thread_local MapEntry cache[SLOTS] = {};
@@ -916,7 +946,8 @@ bool make_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH, int box 
       return true;
     }
   }
-  if (!encode_map(m, ptr, D, rows, BH, box)) return false;
+  if (!(box == 0 ? encode_rows_map(m, ptr, D, (long long)rows * BH) : encode_map(m, ptr, D, rows, BH, box)))
+    return false;
   MapEntry& e = cache[next];
   next = (next + 1) % SLOTS;
   e.k = MapKey{ptr, D, rows, BH, box};
@@ -962,15 +993,18 @@ bool attend_tc_supported(const Problem& p) {
 cudaError_t launch_attend_tc(const Problem& p, const void* Q, const void* K, const void* V,
                              const int32_t* row_ptr, const int32_t* col_idx, void* O,
                              const Work& w, cudaStream_t s) {
-  const void* q = w.qp ? (const void*)w.qp : Q;
-  const void* k = w.kp ? (const void*)w.kp : K;
-  const void* v = w.vp ? (const void*)w.vp : V;
   // K and V tiles: one 128-row box, or two 64-row boxes (one per block) with
-  // 64-token blocks
+  // 64-token blocks; with a permutation, rows gathered through it from the
+  // caller's tensors (no permuted copies)
   const bool b64 = p.b == TILE_ROWS / 2;
+  const bool gather = p.perm != nullptr;
   CUtensorMap maps[5];
-  if (!make_map(&maps[0], q, p.d, p.N, p.BH) || !make_map(&maps[1], k, p.d, p.N, p.BH, p.b) ||
-      !make_map(&maps[2], v, p.d, p.N, p.BH, p.b) || !make_map(&maps[3], w.kbar16, p.d, p.nb, p.BH) ||
+  const bool ok_maps =
+      gather ? (make_map(&maps[0], Q, p.d, p.N, p.BH, 0) && make_map(&maps[1], K, p.d, p.N, p.BH, 0) &&
+                make_map(&maps[2], V, p.d, p.N, p.BH, 0))
+             : (make_map(&maps[0], Q, p.d, p.N, p.BH) && make_map(&maps[1], K, p.d, p.N, p.BH, p.b) &&
+                make_map(&maps[2], V, p.d, p.N, p.BH, p.b));
+  if (!ok_maps || !make_map(&maps[3], w.kbar16, p.d, p.nb, p.BH) ||
       !make_map(&maps[4], w.vbar16, p.d, p.nb, p.BH))
     return cudaErrorInvalidValue;
   TcArgs a;
@@ -992,6 +1026,7 @@ cudaError_t launch_attend_tc(const Problem& p, const void* Q, const void* K, con
     a.order = nullptr;
   }
   a.perm = p.perm;
+  a.gather = gather ? 1 : 0;
   a.o = static_cast<__nv_bfloat16*>(O);
   a.o32 = nullptr;
   a.q_rows = p.N;
