@@ -1052,6 +1052,139 @@ cudaError_t launch_attend_tc(const Problem& p, const void* Q, const void* K, con
   return p.d == 128 ? launch_tc<128>(maps, a, s) : launch_tc<64>(maps, a, s);
 }
 
+// ---- probe correction apply on the tensor cores ----------------------------
+// O <- O + O (B P) + b P for every row of a head (SparsePR page, section 2B),
+// one CTA per 128-row tile: the O tile and W^T = (B P)^T (bf16 [d][d], row n
+// holds column n of B P, i.e. a K-major operand) come in by TMA, one group of
+// tcgen05 MMAs puts O W into TMEM, and four warps add O (read back from the
+// swizzled shared tile) and b P in fp32 and store bf16.
+
+constexpr int AP_THREADS = 128;
+
+template <int D>
+constexpr size_t apply_tc_smem_bytes() {
+  return (size_t)2 * TILE_ROWS * D * 2 + 64 + 1024;
+}
+
+template <int D>
+__global__ void __launch_bounds__(AP_THREADS) probe_apply_tc_kernel(
+    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmW,
+    __nv_bfloat16* o, const float* cp, int N, int32_t* ctrl) {
+  constexpr int NCH = D / 64;
+  constexpr int CHUNK_A = TILE_ROWS * 128;   // bytes of one 64-channel chunk of the O tile
+  constexpr int CHUNK_B = D * 128;           // of W^T (D rows)
+  constexpr int TILE_A = TILE_ROWS * D * 2, TILE_B = D * D * 2;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sA = base, sB = base + TILE_A;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + TILE_A + TILE_B);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t bar_load = smem_u32(&bars[0]), bar_mma = smem_u32(&bars[1]);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, bh = blockIdx.y;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(bar_load, 1);
+    tc::mbar_init(bar_mma, 1);
+    *abort = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(smem_u32(tmem_slot), D < 32 ? 32 : D);
+    tc::tc_fence_before();
+  }
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    tc::mbar_expect_tx(bar_load, TILE_A + TILE_B);
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      tc::tma_load_3d(sA + c * CHUNK_A, &tmO, bar_load, c * 64, tile * TILE_ROWS, bh);
+      tc::tma_load_3d(sB + c * CHUNK_B, &tmW, bar_load, c * 64, 0, bh);
+    }
+    ok = tc::mbar_wait(bar_load, 0, abort, ctrl, 30);
+    if (ok) {
+      tc::tc_fence_after();
+      const uint64_t dA = tc::sdesc_sw128(sA, 16, 1024), dB = tc::sdesc_sw128(sB, 16, 1024);
+      constexpr uint32_t idesc = tc::idesc_bf16_f32(128, D, false);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t offA = ((kk >> 2) * CHUNK_A + (kk & 3) * 32) >> 4;
+        const uint32_t offB = ((kk >> 2) * CHUNK_B + (kk & 3) * 32) >> 4;
+        tc::umma_ss(tmem, dA + offA, dB + offB, idesc, kk > 0);
+      }
+      tc::umma_commit(bar_mma);
+    }
+  }
+  ok = __syncthreads_and(ok);
+  if (ok) ok = __syncthreads_and(tc::mbar_wait(bar_mma, 0, abort, ctrl, 31));
+  if (ok) {
+    tc::tc_fence_after();
+    const int r = warp * 32 + lane;              // tile row = TMEM lane
+    const int tok = tile * TILE_ROWS + r;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const float* cph = cp + (size_t)bh * D;
+    uint4* orow = reinterpret_cast<uint4*>(o + ((size_t)bh * N + (tok < N ? tok : 0)) * D);
+#pragma unroll
+    for (int c32 = 0; c32 < D / 32; ++c32) {
+      uint32_t acc[32];
+      tc::tmem_ld32(tmem + lane_off + 32u * c32, acc);
+      tc::tmem_wait_ld();
+      if (tok < N) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {   // 8 channels per 16-byte piece
+          const int ch = c32 * 32 + q * 8;
+          const int chunk = ch >> 6, piece = (ch & 63) >> 3;
+          const uint4 xv = *reinterpret_cast<const uint4*>(
+              gbase + chunk * CHUNK_A + r * 128 + ((piece ^ (r & 7)) << 4));
+          const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xv);
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 x2 = __bfloat1622float2(xh[e]);
+            v[2 * e] = x2.x + (__uint_as_float(acc[q * 8 + 2 * e]) + __ldg(cph + ch + 2 * e));
+            v[2 * e + 1] = x2.y + (__uint_as_float(acc[q * 8 + 2 * e + 1]) + __ldg(cph + ch + 2 * e + 1));
+          }
+          uint4 pv;
+          pv.x = pack_bf16x2(v[0], v[1]);
+          pv.y = pack_bf16x2(v[2], v[3]);
+          pv.z = pack_bf16x2(v[4], v[5]);
+          pv.w = pack_bf16x2(v[6], v[7]);
+          orow[ch / 8] = pv;
+        }
+      }
+    }
+  } else if (threadIdx.x == 0) {
+    // let copies and MMAs in flight land before the CTA can exit
+    tc::mbar_drain(bar_load, 0);
+    tc::mbar_drain(bar_mma, 0);
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, D < 32 ? 32 : D);
+  }
+}
+
+template <int D>
+cudaError_t launch_apply_tc_d(const Problem& p, void* O, const void* Wt, const float* cp,
+                              int32_t* ctrl, cudaStream_t s) {
+  CUtensorMap mo, mw;
+  if (!make_map(&mo, O, D, p.N, p.BH) || !make_map(&mw, Wt, D, D, p.BH, D)) return cudaErrorInvalidValue;
+  constexpr size_t smem = apply_tc_smem_bytes<D>();
+  cudaError_t e = ensure_dyn_smem((const void*)probe_apply_tc_kernel<D>, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((p.N + TILE_ROWS - 1) / TILE_ROWS, p.BH);
+  probe_apply_tc_kernel<D><<<grid, AP_THREADS, smem, s>>>(mo, mw, static_cast<__nv_bfloat16*>(O), cp,
+                                                         p.N, ctrl);
+  return cudaGetLastError();
+}
+
 // Exact (dense) softmax attention of gathered query rows, fp32 out: Qg holds
 // q_alloc rows per (batch, head) (a multiple of 128, zero past q_rows), every
 // one of the N keys of K and V is attended, and rows [0, q_rows) of each head
@@ -1085,6 +1218,14 @@ cudaError_t launch_dense_rows_tc(const Problem& p, const void* Qg, int q_alloc, 
   cudaError_t e = cudaMemsetAsync(ctrl + CTRL_WORK, 0, 2 * sizeof(int32_t), s);
   if (e != cudaSuccess) return e;
   return p.d == 128 ? launch_tc<128>(maps, a, s) : launch_tc<64>(maps, a, s);
+}
+
+// O <- O + O W + c per head on the tensor cores (the probe correction's
+// folded apply); Wt: bf16 [BH, d, d] with row n = column n of W; c: fp32 [BH, d].
+cudaError_t launch_probe_apply_tc(const Problem& p, void* O, const void* Wt, const float* c,
+                                  int32_t* ctrl, cudaStream_t s) {
+  return p.d == 128 ? launch_apply_tc_d<128>(p, O, Wt, c, ctrl, s)
+                    : launch_apply_tc_d<64>(p, O, Wt, c, ctrl, s);
 }
 
 }  // namespace spattn

@@ -62,6 +62,11 @@ cudaError_t launch_dense_rows_tc(const Problem& p, const void* Qg, int q_alloc, 
                                  const void* K, const void* V, float* out, int32_t* ctrl,
                                  cudaStream_t s);
 
+// O <- O + O W + c for every row of every head, on the tensor cores: Wt is
+// bf16 [BH, d, d] holding W transposed (row n = column n of W), c fp32 [BH, d].
+cudaError_t launch_probe_apply_tc(const Problem& p, void* O, const void* Wt, const float* c,
+                                  int32_t* ctrl, cudaStream_t s);
+
 // Probe-fitted residual correction (SparsePR page, section 2B) of the routed
 // output O in place; scratch of probe_scratch_bytes(p, M) bytes.
 size_t probe_scratch_bytes(const Problem& p, int M);

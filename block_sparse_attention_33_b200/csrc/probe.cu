@@ -7,28 +7,32 @@
 // leading right singular vectors of the probe residuals and added to every
 // row's sparse output.  Probe rows take their exact output.
 //
-// One head at a time (every (batch, head) pair is its own attention call):
+// Per (batch, head) pair (every pair is its own attention call):
 //
 //   probe_gather_kernel the probe queries into whole 128-row tiles, then the
 //                       tcgen05 attention kernel in its dense mode: exact
 //                       softmax attention of those rows over all N keys, fp32
 //                       output (bf16 operands, fp32 accumulation, as every
 //                       attention row of this library);
-//   probe_fit_kernel    normal equations of the ridge fit on [1, x]:
-//                       G = A^T A + lam * diag(0, 1, ..., 1), C = A^T R, then
-//                       a Cholesky factorisation of G and two triangular
-//                       solves for W = [b; B] (one CTA per head);
-//   probe_eig_kernel    R^T R, its eigenvectors by the cyclic Jacobi method
-//                       with a round-robin pairing (d/2 disjoint rotations per
-//                       step), the projector P = V_r V_r^T on the r largest
-//                       eigenvalues (the r leading right singular vectors of
-//                       R), and B P, b P (one CTA per head);
-//   probe_apply_kernel  O <- O + O (B P) + b P for every row, bf16 out;
+//   probe_gram_kernel   the Gram matrix of the probe rows [1, x, R] (one CTA
+//                       per 128 probe rows and head, partial sums per slab):
+//                       its blocks are A^T A, A^T R and R^T R for A = [1, x];
+//   probe_solve_kernel  role 0, the ridge fit: G = A^T A + lam diag(0, 1,
+//                       ..., 1), C = A^T R, Cholesky and two triangular solves
+//                       for W = [b; B]; role 1, the r leading eigenvectors of
+//                       R^T R (the leading right singular vectors of R) by
+//                       block subspace iteration with a Rayleigh-Ritz step, or
+//                       cyclic Jacobi on the whole matrix for large r;
+//   probe_fold_kernel   B P and b P with P = U U^T;
+//   then the tcgen05 apply (launch_probe_apply_tc): O <- O + O (B P) + b P
+//                       for every row, bf16 out;
 //   probe_set_kernel    probe rows <- their exact output.
 //
-// All arithmetic is fp32.  A probe index outside [0, N) is skipped and
-// flagged (DEV_BAD_INDEX); normal equations that are not positive definite
-// leave that head uncorrected and are flagged (DEV_NUMERIC).
+// The fit and the subspace are fp32; B P enters the tensor-core apply in
+// bf16 (the correction it makes is about a thousandth of the output).  A
+// probe index outside [0, N) is skipped and flagged (DEV_BAD_INDEX); normal
+// equations that are not positive definite leave that head uncorrected and
+// are flagged (DEV_NUMERIC).
 #include <math.h>
 
 #include "common.cuh"
@@ -38,7 +42,6 @@ namespace spattn {
 namespace {
 
 constexpr int PB_THREADS = 256;
-constexpr int PA_ROWS = 64;                // output rows per apply CTA
 constexpr int JACOBI_MAX_SWEEPS = 16;
 
 struct ProbeArgs {
@@ -47,7 +50,7 @@ struct ProbeArgs {
   const int32_t* probes;           // [BH, M] token indices
   float* od;                       // [BH, M, D] exact probe rows
   float* w;                        // [BH, D + 1, D] ridge solution, row 0 = b
-  float* wp;                       // [BH, D, D] B P
+  __nv_bfloat16* wt;               // [BH, D, D] (B P)^T, bf16
   float* cp;                       // [BH, D] b P
   float* pu;                       // [BH, D, D] leading eigenvectors of R^T R (first r columns)
   int32_t* ctrl;                   // error word
@@ -212,7 +215,7 @@ constexpr size_t solve_smem_bytes() {
   constexpr size_t DA = D + 1;
   constexpr size_t fit = (DA * DA + DA * D + 8) * sizeof(float);
   constexpr size_t jac = (2 * (size_t)D * (D + 1) + 4 * (size_t)D + 8) * sizeof(float);
-  constexpr size_t sub = ((size_t)D * (D + 1) + 2 * (size_t)D * SUB_MAXQ +
+  constexpr size_t sub = ((size_t)D * (D + 4) + 2 * (size_t)D * SUB_MAXQ +
                           2 * (size_t)SUB_MAXQ * (SUB_MAXQ + 1) + 4 * (size_t)SUB_MAXQ + 8) *
                          sizeof(float);
   return fit > jac ? (fit > sub ? fit : sub) : (jac > sub ? jac : sub);
@@ -391,7 +394,7 @@ __global__ void __launch_bounds__(SV_THREADS) probe_solve_kernel(const ProbeArgs
   float* U = a.pu + (size_t)bh * D * D;
   constexpr int DP = D + 1;
   const int q = r + SUB_EXTRA;
-  if (q > SUB_MAXQ || q >= D) {
+  if (((q + 7) & ~7) > SUB_MAXQ || q >= D) {
     // Jacobi on the whole D x D matrix
     float* S = psm;               // [D][DP]
     float* V = S + D * DP;        // [D][DP]
@@ -410,21 +413,24 @@ __global__ void __launch_bounds__(SV_THREADS) probe_solve_kernel(const ProbeArgs
   // columns) <- orth(S X), SUB_ITERS times from a fixed +-1 start; then the
   // q x q matrix T = X^T S X is diagonalised by Jacobi and the r leading Ritz
   // vectors X W are the basis.  The subspace error decays like
-  // (lambda_{q+1} / lambda_r)^SUB_ITERS.
-  constexpr int QM = SUB_MAXQ, QP = SUB_MAXQ + 1;
-  float* S = psm;                 // [D][DP]
-  float* X = S + D * DP;          // [D][QM]
+  // (lambda_{q+1} / lambda_r)^SUB_ITERS.  q = r + SUB_EXTRA rounded up to a
+  // multiple of 8, so that the products run on 4 x 4 register tiles of
+  // float4 rows (S is symmetric: row j of S is column j).
+  constexpr int QM = SUB_MAXQ, QP = SUB_MAXQ + 1, DS = D + 4;
+  const int qn = (q + 7) & ~7;   // q > SUB_MAXQ was sent to Jacobi above; qn <= SUB_MAXQ
+  float* S = psm;                 // [D][DS]
+  float* X = S + D * DS;          // [D][QM]
   float* Y = X + D * QM;          // [D][QM]
-  float* T = Y + D * QM;          // [QM][QP]: Gram of Y / Rayleigh quotient
-  float* W = T + QM * QP;         // [QM][QP]: Jacobi vectors
+  float* T = Y + D * QM;          // [QM][QP]: Gram of Y, L^-1, Rayleigh quotient
+  float* W = T + QM * QP;         // [QM][QP]: Cholesky factor, Jacobi vectors
   float* rc = W + QM * QP;        // [QM / 2]
   float* rs = rc + QM / 2;        // [QM / 2]
   int* pq = reinterpret_cast<int*>(rs + QM / 2);  // [QM]
   int* rank = pq + QM;                             // [QM]
   int* flag = rank + QM;
-  for (int e = tid; e < D * D; e += nt) S[(e / D) * DP + e % D] = gram_at<D>(gph, slabs, DA + e / D, DA + e % D);
-  for (int e = tid; e < D * q; e += nt) {
-    const int i = e / q, c = e % q;
+  for (int e = tid; e < D * D; e += nt) S[(e / D) * DS + e % D] = gram_at<D>(gph, slabs, DA + e / D, DA + e % D);
+  for (int e = tid; e < D * qn; e += nt) {
+    const int i = e / qn, c = e % qn;
     // a fixed +-1 pattern from a multiplicative hash of (i, c): full column
     // rank (an xor of per-row and per-column bits would give rank 1)
     unsigned h = (unsigned)i * 0x9E3779B1u + (unsigned)c * 0x85EBCA77u;
@@ -434,174 +440,209 @@ __global__ void __launch_bounds__(SV_THREADS) probe_solve_kernel(const ProbeArgs
     X[i * QM + c] = (h >> 31) ? 1.f : -1.f;
   }
   __syncthreads();
-  // Y <- S X
-  auto mul = [&]() {
-    for (int e = tid; e < D * q; e += nt) {
-      const int i = e / q, c = e % q;
-      float s0 = 0.f, s1 = 0.f;
-      for (int j = 0; j < D; j += 2) {
-        s0 = fmaf(S[i * DP + j], X[j * QM + c], s0);
-        s1 = fmaf(S[i * DP + j + 1], X[(j + 1) * QM + c], s1);
+  const int qb = qn / 4;          // 4-column blocks
+  // C (D x qn) = A (D x D, rows of stride lda, symmetric) x Bm (D x qn)
+  auto mul_tiles = [&](const float* A, int lda, const float* Bm, float* C) {
+    for (int t = tid; t < (D / 4) * qb; t += nt) {
+      const int ib = t / qb, cb = t % qb;
+      float acc[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+      for (int j = 0; j < D; ++j) {
+        const float4 a4 = *reinterpret_cast<const float4*>(A + j * lda + 4 * ib);   // A[4ib..][j]
+        const float4 b4 = *reinterpret_cast<const float4*>(Bm + j * QM + 4 * cb);
+        const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
       }
-      Y[i * QM + c] = s0 + s1;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<float4*>(C + (4 * ib + u) * QM + 4 * cb) =
+            make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+    }
+    __syncthreads();
+  };
+  // T (qn x qn) = A^T Bm for A, Bm (D x qn)
+  auto gram_tiles = [&](const float* A, const float* Bm) {
+    for (int t = tid; t < qb * qb; t += nt) {
+      const int ib = t / qb, cb = t % qb;
+      float acc[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+      for (int k = 0; k < D; ++k) {
+        const float4 a4 = *reinterpret_cast<const float4*>(A + k * QM + 4 * ib);
+        const float4 b4 = *reinterpret_cast<const float4*>(Bm + k * QM + 4 * cb);
+        const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) T[(4 * ib + u) * QP + 4 * cb + v] = acc[u][v];
     }
     __syncthreads();
   };
   // X <- Y L^-T with Y^T Y = L L^T (Cholesky QR); a column that has become
   // dependent (tiny pivot) is set to zero
   auto orth = [&]() {
-    for (int e = tid; e < q * q; e += nt) {
-      const int i = e / q, j = e % q;
-      float s = 0.f;
-      for (int k = 0; k < D; ++k) s = fmaf(Y[k * QM + i], Y[k * QM + j], s);
-      T[i * QP + j] = s;
-    }
-    __syncthreads();
-    if (tid < 32) {   // one warp: q x q Cholesky, lanes share each column update
+    gram_tiles(Y, Y);
+    if (tid < 32) {   // one warp: Cholesky into W (lower), then L^-1 into T (lower)
       float scale = 0.f;
-      for (int k = tid; k < q; k += 32) scale = fmaxf(scale, T[k * QP + k]);
+      for (int k = tid; k < qn; k += 32) scale = fmaxf(scale, T[k * QP + k]);
       scale = warp_max_f(scale);
-      for (int k = 0; k < q; ++k) {
-        float dkk = T[k * QP + k];
+      for (int e = tid; e < qn * qn; e += 32) W[(e / qn) * QP + e % qn] = T[(e / qn) * QP + e % qn];
+      __syncwarp();
+      for (int k = 0; k < qn; ++k) {
+        const float dkk = W[k * QP + k];
         const bool dead = !(dkk > 1e-12f * fmaxf(scale, 1e-30f));
         const float lkk = dead ? 0.f : sqrtf(dkk);
         __syncwarp();
-        for (int i = k + 1 + tid; i < q; i += 32) T[i * QP + k] = dead ? 0.f : T[i * QP + k] / lkk;
-        if (tid == 0) T[k * QP + k] = lkk;
+        for (int i = k + 1 + tid; i < qn; i += 32) W[i * QP + k] = dead ? 0.f : W[i * QP + k] / lkk;
+        if (tid == 0) W[k * QP + k] = lkk;
         __syncwarp();
-        for (int e = tid; e < (q - k - 1) * (q - k - 1); e += 32) {
-          const int i = k + 1 + e / (q - k - 1), j = k + 1 + e % (q - k - 1);
-          if (j <= i) T[i * QP + j] = fmaf(-T[i * QP + k], T[j * QP + k], T[i * QP + j]);
+        for (int e = tid; e < (qn - k - 1) * (qn - k - 1); e += 32) {
+          const int i = k + 1 + e / (qn - k - 1), j = k + 1 + e % (qn - k - 1);
+          if (j <= i) W[i * QP + j] = fmaf(-W[i * QP + k], W[j * QP + k], W[i * QP + j]);
         }
         __syncwarp();
       }
+      // L^-1, one column per lane (columns of a dead pivot stay zero)
+      for (int c = tid; c < qn; c += 32) {
+        for (int i = 0; i < qn; ++i) {
+          float v = 0.f;
+          if (i >= c) {
+            float sum = (i == c) ? 1.f : 0.f;
+            for (int k = c; k < i; ++k) sum = fmaf(-W[i * QP + k], T[k * QP + c], sum);
+            v = W[i * QP + i] > 0.f ? sum / W[i * QP + i] : 0.f;
+          }
+          T[i * QP + c] = v;   // rows of column c are written in order, reads are rows < i
+        }
+      }
     }
     __syncthreads();
-    for (int i = tid; i < D; i += nt) {   // row i: x L^T = y, forward substitution
-      for (int c = 0; c < q; ++c) {
-        float s = Y[i * QM + c];
-        for (int k = 0; k < c; ++k) s = fmaf(-X[i * QM + k], T[c * QP + k], s);
-        const float lcc = T[c * QP + c];
-        X[i * QM + c] = lcc > 0.f ? s / lcc : 0.f;
+    // X = Y (L^-1)^T: X[i][c] = sum_k Y[i][k] Linv[c][k]
+    for (int t = tid; t < (D / 4) * qb; t += nt) {
+      const int ib = t / qb, cb = t % qb;
+      float acc[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+      for (int k = 0; k < qn; ++k) {
+        float av[4], bv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) av[u] = Y[(4 * ib + u) * QM + k];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) bv[v] = T[(4 * cb + v) * QP + k];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
       }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<float4*>(X + (4 * ib + u) * QM + 4 * cb) =
+            make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
     }
     __syncthreads();
   };
   for (int it = 0; it < SUB_ITERS; ++it) {
-    mul();
+    mul_tiles(S, DS, X, Y);
     orth();
   }
-  mul();   // Y = S X; T = X^T Y
-  for (int e = tid; e < q * q; e += nt) {
-    const int i = e / q, j = e % q;
-    float s = 0.f;
-    for (int k = 0; k < D; ++k) s = fmaf(X[k * QM + i], Y[k * QM + j], s);
-    T[i * QP + j] = s;
+  mul_tiles(S, DS, X, Y);   // Y = S X; T = X^T Y
+  gram_tiles(X, Y);
+  // symmetrise (the pairing of Jacobi needs an even size; qn is a multiple of 8)
+  for (int e = tid; e < qn * qn; e += nt) {
+    const int i = e / qn, j = e % qn;
+    if (i < j) {
+      const float v = 0.5f * (T[i * QP + j] + T[j * QP + i]);
+      T[i * QP + j] = v;
+      T[j * QP + i] = v;
+    }
   }
   __syncthreads();
-  // symmetrise, pad to an even size for the round-robin pairing
-  const int qe = (q + 1) & ~1;
-  for (int e = tid; e < qe * qe; e += nt) {
-    const int i = e / qe, j = e % qe;
-    if (i >= q || j >= q) T[i * QP + j] = (i == j) ? -1.f : 0.f;   // below every Ritz value (>= 0)
-    else if (i < j) { const float v = 0.5f * (T[i * QP + j] + T[j * QP + i]); T[i * QP + j] = v; T[j * QP + i] = v; }
-  }
-  __syncthreads();
-  jacobi_cta(T, W, qe, QP, rc, rs, pq, flag);
+  jacobi_cta(T, W, qn, QP, rc, rs, pq, flag);
   __syncthreads();
   // rank the Ritz values; U[:, k] = X W[:, col of rank k], k < r
-  for (int i = tid; i < qe; i += nt) {
+  for (int i = tid; i < qn; i += nt) {
     const float li = T[i * QP + i];
     int k = 0;
-    for (int j = 0; j < qe; ++j) {
+    for (int j = 0; j < qn; ++j) {
       const float lj = T[j * QP + j];
       k += (lj > li || (lj == li && j < i)) ? 1 : 0;
     }
     rank[i] = k;
   }
   __syncthreads();
-  for (int e = tid; e < D * qe; e += nt) {
-    const int row = e / qe, col = e % qe;
-    if (rank[col] < r && col < q) {
-      float s = 0.f;
-      for (int k = 0; k < q; ++k) s = fmaf(X[row * QM + k], W[k * QP + col], s);
-      U[row * D + rank[col]] = s;
+  for (int e = tid; e < D * qn; e += nt) {
+    const int row = e / qn, col = e % qn;
+    if (rank[col] < r) {
+      float sacc = 0.f;
+      for (int k = 0; k < qn; ++k) sacc = fmaf(X[row * QM + k], W[k * QP + col], sacc);
+      U[row * D + rank[col]] = sacc;
     }
   }
 }
 
 // B P and b P with P = U U^T (U: the first r columns), or P = 0 / I for
-// r = 0 / r >= D; one CTA per head.
+// r = 0 / r >= D; one CTA per head.  B P goes out transposed in bf16 (row n
+// holds column n: the K-major operand of the tensor-core apply; the
+// correction is about a thousandth of the output, so bf16 rounding of it is
+// far below the output's own rounding), b P in fp32.
+template <int D>
+size_t fold_smem_bytes(int r) {
+  const int rr = (r > 0 && r < D) ? r : 0;
+  return ((size_t)(D + 1) * D + (size_t)D * rr + (size_t)(D + 1) * rr) * sizeof(float);
+}
+
 template <int D>
 __global__ void __launch_bounds__(PB_THREADS) probe_fold_kernel(const ProbeArgs a) {
   extern __shared__ __align__(16) float psm[];
   const int bh = blockIdx.x, tid = threadIdx.x;
   const int r = a.r;
-  const float* wfit = a.w + (size_t)bh * (D + 1) * D;   // row 0 = b, rows 1.. = B
-  float* wp = a.wp + (size_t)bh * D * D;
+  float* Ws = psm;                  // [D + 1][D]: row 0 = b, rows 1.. = B
+  const float* wfit = a.w + (size_t)bh * (D + 1) * D;
+  __nv_bfloat16* wt = a.wt + (size_t)bh * D * D;
   float* cp = a.cp + (size_t)bh * D;
+  for (int e = tid; e < (D + 1) * D; e += PB_THREADS) Ws[e] = wfit[e];
+  __syncthreads();
   if (r <= 0 || r >= D) {
     const bool full = r >= D;
-    for (int e = tid; e < D * D; e += PB_THREADS) wp[e] = full ? wfit[D + e] : 0.f;
-    for (int c = tid; c < D; c += PB_THREADS) cp[c] = full ? wfit[c] : 0.f;
+    for (int e = tid; e < D * D; e += PB_THREADS) {
+      const int n = e / D, k = e % D;   // W^T[n][k] = B[k][n]
+      wt[e] = __float2bfloat16_rn(full ? Ws[(k + 1) * D + n] : 0.f);
+    }
+    for (int c = tid; c < D; c += PB_THREADS) cp[c] = full ? Ws[c] : 0.f;
     return;
   }
-  float* Us = psm;                 // [D][r]
-  float* BU = Us + D * r;          // [D + 1][r]: row 0 = b U, rows 1.. = B U
+  float* Us = Ws + (D + 1) * D;     // [D][r]
+  float* BU = Us + D * r;           // [D + 1][r]: row 0 = b U, rows 1.. = B U
   const float* U = a.pu + (size_t)bh * D * D;
   for (int e = tid; e < D * r; e += PB_THREADS) Us[e] = U[(e / r) * D + e % r];
   __syncthreads();
   for (int e = tid; e < (D + 1) * r; e += PB_THREADS) {
     const int i = e / r, k = e % r;
     float s = 0.f;
-    for (int j = 0; j < D; ++j) s = fmaf(wfit[i * D + j], Us[j * r + k], s);
+    for (int j = 0; j < D; ++j) s = fmaf(Ws[i * D + j], Us[j * r + k], s);
     BU[e] = s;
   }
   __syncthreads();
   for (int e = tid; e < (D + 1) * D; e += PB_THREADS) {
-    const int i = e / D, j = e % D;
+    const int i = e / D, j = e % D;   // (B P)[i - 1][j], or (b P)[j] for i = 0
     float s = 0.f;
     for (int k = 0; k < r; ++k) s = fmaf(BU[i * r + k], Us[j * r + k], s);
-    if (i == 0) cp[j] = s; else wp[(i - 1) * D + j] = s;
+    if (i == 0) cp[j] = s; else wt[(size_t)j * D + (i - 1)] = __float2bfloat16_rn(s);
   }
-}
-
-// ---- apply -----------------------------------------------------------------
-
-template <int D>
-size_t apply_smem_bytes() {
-  return ((size_t)D * D + D + (size_t)PA_ROWS * D) * sizeof(float);
-}
-
-template <int D>
-__global__ void __launch_bounds__(PB_THREADS) probe_apply_kernel(const ProbeArgs a) {
-  constexpr int RPT = PA_ROWS * D / PB_THREADS;   // rows per thread (one column each)
-  extern __shared__ float psm[];
-  float* W = psm;                 // [D][D] B P
-  float* cvec = W + D * D;        // [D]    b P
-  float* X = cvec + D;            // [PA_ROWS][D] sparse output rows
-  const int bh = blockIdx.y, n0 = blockIdx.x * PA_ROWS, tid = threadIdx.x;
-  const float* wp = a.wp + (size_t)bh * D * D;
-  for (int e = tid; e < D * D; e += PB_THREADS) W[e] = wp[e];
-  for (int c = tid; c < D; c += PB_THREADS) cvec[c] = a.cp[(size_t)bh * D + c];
-  __nv_bfloat16* orows = a.o + ((size_t)bh * a.N + n0) * D;
-  for (int e = tid; e < PA_ROWS * D; e += PB_THREADS) {
-    const int rr = e / D;
-    X[e] = n0 + rr < a.N ? __bfloat162float(orows[e]) : 0.f;
-  }
-  __syncthreads();
-  const int j = tid % D, r0 = (tid / D) * RPT;
-  float acc[RPT];
-#pragma unroll
-  for (int t = 0; t < RPT; ++t) acc[t] = X[(r0 + t) * D + j] + cvec[j];
-  for (int i = 0; i < D; ++i) {
-    const float w = W[i * D + j];
-#pragma unroll
-    for (int t = 0; t < RPT; ++t) acc[t] = fmaf(X[(r0 + t) * D + i], w, acc[t]);
-  }
-#pragma unroll
-  for (int t = 0; t < RPT; ++t)
-    if (n0 + r0 + t < a.N) orows[(size_t)(r0 + t) * D + j] = __float2bfloat16_rn(acc[t]);
 }
 
 template <int D>
@@ -613,17 +654,11 @@ __global__ void __launch_bounds__(D) probe_set_kernel(const ProbeArgs a) {
 }
 
 template <int D>
-size_t fold_smem_bytes() {
-  return ((size_t)D * (D - 1) + (size_t)(D + 1) * (D - 1)) * sizeof(float);
-}
-
-template <int D>
 cudaError_t launch_probe_d(const Problem& p, const ProbeArgs& a, int m_alloc, __nv_bfloat16* qg,
                            float* gp, cudaStream_t s) {
   cudaError_t e;
   if ((e = ensure_dyn_smem((const void*)probe_solve_kernel<D>, solve_smem_bytes<D>())) != cudaSuccess) return e;
-  if ((e = ensure_dyn_smem((const void*)probe_fold_kernel<D>, fold_smem_bytes<D>())) != cudaSuccess) return e;
-  if ((e = ensure_dyn_smem((const void*)probe_apply_kernel<D>, apply_smem_bytes<D>())) != cudaSuccess) return e;
+  if ((e = ensure_dyn_smem((const void*)probe_fold_kernel<D>, fold_smem_bytes<D>(D - 1))) != cudaSuccess) return e;
   const int gather_blocks = (m_alloc * (D / 8) + PB_THREADS - 1) / PB_THREADS;
   probe_gather_kernel<D><<<dim3(gather_blocks, a.BH), PB_THREADS, 0, s>>>(a, m_alloc, qg);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -633,11 +668,9 @@ cudaError_t launch_probe_d(const Problem& p, const ProbeArgs& a, int m_alloc, __
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   probe_solve_kernel<D><<<dim3(a.BH, 2), SV_THREADS, solve_smem_bytes<D>(), s>>>(a, gp, slabs);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const size_t fold_smem = a.r > 0 && a.r < D ? ((size_t)D * a.r + (size_t)(D + 1) * a.r) * sizeof(float) : 0;
-  probe_fold_kernel<D><<<a.BH, PB_THREADS, fold_smem, s>>>(a);
+  probe_fold_kernel<D><<<a.BH, PB_THREADS, fold_smem_bytes<D>(a.r), s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  probe_apply_kernel<D><<<dim3((a.N + PA_ROWS - 1) / PA_ROWS, a.BH), PB_THREADS, apply_smem_bytes<D>(), s>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_probe_apply_tc(p, a.o, a.wt, a.cp, a.ctrl, s)) != cudaSuccess) return e;
   probe_set_kernel<D><<<dim3(a.M, a.BH), D, 0, s>>>(a);
   return cudaGetLastError();
 }
@@ -673,7 +706,7 @@ cudaError_t launch_probe_correct(const Problem& p, const void* Q, const void* K,
   size_t off = 0;
   a.od = reinterpret_cast<float*>(b + off); off += up(BH * M * d * 4);
   a.w = reinterpret_cast<float*>(b + off);  off += up(BH * (d + 1) * d * 4);
-  a.wp = reinterpret_cast<float*>(b + off); off += up(BH * d * d * 4);
+  a.wt = reinterpret_cast<__nv_bfloat16*>(b + off); off += up(BH * d * d * 4);
   a.cp = reinterpret_cast<float*>(b + off); off += up(BH * d * 4);
   const int m_alloc = probe_rows_alloc(M);
   __nv_bfloat16* qg = reinterpret_cast<__nv_bfloat16*>(b + off); off += up(BH * m_alloc * d * 2);
