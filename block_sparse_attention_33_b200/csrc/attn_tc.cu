@@ -414,17 +414,54 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       // the tile loads are TMA boxes issued by lane 0, or, with a token
       // permutation, row gathers through it issued by all lanes (lane l: tile
       // rows 4l .. 4l + 3; a row past the last token repeats token N - 1).
-      auto gather_tile = [&](uint32_t dst, const CUtensorMap* m, uint32_t fb, int tok0, int tok1) {
-        // tok0: first token (permuted order) of tile rows 0-63, tok1: of rows 64-127
+      // Row gathers: a lane's four rows of a tile (tile rows 4l .. 4l + 3) as
+      // row coordinates of the 2-D map, fetched from perm one task ahead of
+      // their use (tok0: first token, permuted order, of tile rows 0-63; tok1:
+      // of rows 64-127).
+      auto fetch_rows = [&](int tok0, int tok1) -> int4 {
         const int r0 = 4 * lane;
         const int tok = (r0 < 64 ? tok0 : tok1) + (r0 & 63);
-        int rows[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) rows[k] = bh * a.N + __ldg(a.perm + min(tok + k, a.N - 1));
+        const int base = bh * a.N;
+        return make_int4(base + __ldg(a.perm + min(tok, a.N - 1)), base + __ldg(a.perm + min(tok + 1, a.N - 1)),
+                         base + __ldg(a.perm + min(tok + 2, a.N - 1)), base + __ldg(a.perm + min(tok + 3, a.N - 1)));
+      };
+      auto gather_tile = [&](uint32_t dst, const CUtensorMap* m, uint32_t fb, int4 rw) {
 #pragma unroll
         for (int c = 0; c < NCH; ++c)
-          tc::tma_gather4(dst + c * CHUNK_BYTES + r0 * 128, m, fb, c * 64, rows[0], rows[1], rows[2], rows[3]);
+          tc::tma_gather4(dst + c * CHUNK_BYTES + 4 * lane * 128, m, fb, c * 64, rw.x, rw.y, rw.z, rw.w);
       };
+      // first token of the key tile of task t < nkept (and, with b = 64, of its
+      // second block)
+      auto task_rows = [&](int t, int& row, int& row2) {
+        row2 = -1;
+        if (a.b64) {
+          // an absent second block repeats the first (valid data, masked
+          // by the softmax)
+          const int j0 = inf.ublk[2 * t];
+          const int j1 = 2 * t + 1 < inf.nunion ? inf.ublk[2 * t + 1] : j0;
+          row = j0 * 64;
+          row2 = j1 * 64;
+        } else if (a.dense) {
+          row = t * TILE_ROWS;
+        } else if (a.inline_sel) {
+          row = inf.ublk[t] * TILE_ROWS;
+        } else {
+          int j = __ldg(a.col_idx + r_lo + t);
+          if (j < 0 || j >= a.nb) {
+            if (lane == 0) flag_error(a.ctrl, DEV_BAD_INDEX, item);
+            j = 0;  // load something valid; the softmax masks the whole task
+          }
+          row = j * TILE_ROWS;
+        }
+      };
+      auto task_fetch = [&](int t) -> int4 {
+        if (!a.gather || t >= nkept) return make_int4(0, 0, 0, 0);
+        int row, row2;
+        task_rows(t, row, row2);
+        return fetch_rows(row, row2 < 0 ? row + 64 : row2);
+      };
+      int4 qrw = make_int4(0, 0, 0, 0);
+      if (a.gather) qrw = fetch_rows(i * TILE_ROWS, i * TILE_ROWS + 64);   // lands during the wait
       if (lane == 0 && qn > 0)
         ok = tc::mbar_wait_fast(bar(B_QEMPTY), (uint32_t)(qn - 1) & 1u, abort, a.ctrl, 12);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -432,37 +469,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (lane == 0) tc::mbar_expect_tx(bar(B_QFULL), TILE_BYTES);
         if (a.gather) {
           __syncwarp();
-          gather_tile(sQ, &tmQ, bar(B_QFULL), i * TILE_ROWS, i * TILE_ROWS + 64);
+          gather_tile(sQ, &tmQ, bar(B_QFULL), qrw);
         } else if (lane == 0) {
 #pragma unroll
           for (int c = 0; c < NCH; ++c)
             tc::tma_load_3d(sQ + c * CHUNK_BYTES, &tmQ, bar(B_QFULL), c * 64, i * TILE_ROWS, bh);
         }
       }
-      auto issue = [&](int t, bool is_v) -> bool {
+      // rw: the lane's gathered rows of the tile when a.gather and t < nkept
+      auto issue = [&](int t, bool is_v, int4 rw) -> bool {
         const CUtensorMap* m;
-        int row, row2 = -1;   // first token of tile rows 0-.. and, with b = 64, of rows 64-127
+        int row = 0, row2 = -1;
         if (t < nkept) {
           m = is_v ? &tmV : &tmK;
-          if (a.b64) {
-            // an absent second block repeats the first (valid data, masked
-            // by the softmax)
-            const int j0 = inf.ublk[2 * t];
-            const int j1 = 2 * t + 1 < inf.nunion ? inf.ublk[2 * t + 1] : j0;
-            row = j0 * 64;
-            row2 = j1 * 64;
-          } else if (a.dense) {
-            row = t * TILE_ROWS;
-          } else if (a.inline_sel) {
-            row = inf.ublk[t] * TILE_ROWS;
-          } else {
-            int j = __ldg(a.col_idx + r_lo + t);
-            if (j < 0 || j >= a.nb) {
-              if (lane == 0) flag_error(a.ctrl, DEV_BAD_INDEX, item);
-              j = 0;  // load something valid; the softmax masks the whole task
-            }
-            row = j * TILE_ROWS;
-          }
+          if (!a.gather) task_rows(t, row, row2);
         } else {
           m = is_v ? &tmVb : &tmKb;
           row = res_tile(res_tiles, t - nkept) * TILE_ROWS;
@@ -476,7 +496,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint32_t dst = sRing + s * TILE_BYTES;
         if (a.gather && t < nkept) {
           __syncwarp();
-          gather_tile(dst, m, full(s), row, row2 < 0 ? row + 64 : row2);
+          gather_tile(dst, m, full(s), rw);
         } else if (lane == 0) {
           if (row2 < 0) {
 #pragma unroll
@@ -493,11 +513,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         ++li;
         return true;
       };
-      if (ok) ok = issue(0, false);
-      if (ok && T > 1) ok = issue(1, false);
+      // K(0), K(1), then per task t: V(t), K(t + 2); gathered rows of tasks
+      // t, t + 1, t + 2 held in ra, rb, rc, task t + 3's fetched as K(t + 2)
+      // goes out
+      int4 ra = task_fetch(0), rb = task_fetch(1);
+      if (ok) ok = issue(0, false, ra);
+      if (ok && T > 1) ok = issue(1, false, rb);
+      int4 rc = task_fetch(2);
       for (int t = 0; ok && t < T; ++t) {
-        ok = issue(t, true);
-        if (ok && t + 2 < T) ok = issue(t + 2, false);
+        ok = issue(t, true, ra);
+        if (ok && t + 2 < T) ok = issue(t + 2, false, rc);
+        ra = rb;
+        rb = rc;
+        rc = task_fetch(t + 3);
       }
       ++qn;
       if (!ok) break;
