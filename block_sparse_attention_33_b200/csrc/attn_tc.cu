@@ -127,8 +127,6 @@ struct TcArgs {
   const float *qbar, *kbar;  // fp32 means [BH, nb, d]
   float tau;                 // Top-p mass, or the per-block threshold theta
   int threshold, kmin;
-  int gather;      // a token permutation: Q, K and V rows are gathered through perm
-                   // (tmQ, tmK, tmV are then 2-D row maps [BH * N, D], box 64 x 1)
   int b64;         // 64-token blocks: a tile holds two query (key) blocks
   int nq;          // query tiles per (batch, head): nb (b = 128) or ceil(nb / 2) (b = 64)
   int blk;         // block size b
@@ -410,28 +408,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       __syncwarp();
       tc::mbar_arrive(bar(B_INFO_FULL0 + slot));   // every lane: releases its own writes
       if (T == 0) continue;
-      // Loads.  Lane 0 makes every wait and sets every transaction count;
-      // the tile loads are TMA boxes issued by lane 0, or, with a token
-      // permutation, row gathers through it issued by all lanes (lane l: tile
-      // rows 4l .. 4l + 3; a row past the last token repeats token N - 1).
-      // Row gathers: a lane's four rows of a tile (tile rows 4l .. 4l + 3) as
-      // row coordinates of the 2-D map, fetched from perm one task ahead of
-      // their use (tok0: first token, permuted order, of tile rows 0-63; tok1:
-      // of rows 64-127).
-      auto fetch_rows = [&](int tok0, int tok1) -> int4 {
-        const int r0 = 4 * lane;
-        const int tok = (r0 < 64 ? tok0 : tok1) + (r0 & 63);
-        const int base = bh * a.N;
-        return make_int4(base + __ldg(a.perm + min(tok, a.N - 1)), base + __ldg(a.perm + min(tok + 1, a.N - 1)),
-                         base + __ldg(a.perm + min(tok + 2, a.N - 1)), base + __ldg(a.perm + min(tok + 3, a.N - 1)));
-      };
-      auto gather_tile = [&](uint32_t dst, const CUtensorMap* m, uint32_t fb, int4 rw) {
-#pragma unroll
-        for (int c = 0; c < NCH; ++c)
-          tc::tma_gather4(dst + c * CHUNK_BYTES + 4 * lane * 128, m, fb, c * 64, rw.x, rw.y, rw.z, rw.w);
-      };
-      // first token of the key tile of task t < nkept (and, with b = 64, of its
-      // second block)
+      // Loads: lane 0 makes every wait, sets every transaction count and
+      // issues the TMA boxes; the other lanes follow its verdicts.
+      // task_rows: first token of the key tile of task t < nkept (and, with
+      // b = 64, of its second block)
       auto task_rows = [&](int t, int& row, int& row2) {
         row2 = -1;
         if (a.b64) {
@@ -454,35 +434,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           row = j * TILE_ROWS;
         }
       };
-      auto task_fetch = [&](int t) -> int4 {
-        if (!a.gather || t >= nkept) return make_int4(0, 0, 0, 0);
-        int row, row2;
-        task_rows(t, row, row2);
-        return fetch_rows(row, row2 < 0 ? row + 64 : row2);
-      };
-      int4 qrw = make_int4(0, 0, 0, 0);
-      if (a.gather) qrw = fetch_rows(i * TILE_ROWS, i * TILE_ROWS + 64);   // lands during the wait
       if (lane == 0 && qn > 0)
         ok = tc::mbar_wait_fast(bar(B_QEMPTY), (uint32_t)(qn - 1) & 1u, abort, a.ctrl, 12);
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (ok) {
-        if (lane == 0) tc::mbar_expect_tx(bar(B_QFULL), TILE_BYTES);
-        if (a.gather) {
-          __syncwarp();
-          gather_tile(sQ, &tmQ, bar(B_QFULL), qrw);
-        } else if (lane == 0) {
+      if (ok && lane == 0) {
+        tc::mbar_expect_tx(bar(B_QFULL), TILE_BYTES);
 #pragma unroll
-          for (int c = 0; c < NCH; ++c)
-            tc::tma_load_3d(sQ + c * CHUNK_BYTES, &tmQ, bar(B_QFULL), c * 64, i * TILE_ROWS, bh);
-        }
+        for (int c = 0; c < NCH; ++c)
+          tc::tma_load_3d(sQ + c * CHUNK_BYTES, &tmQ, bar(B_QFULL), c * 64, i * TILE_ROWS, bh);
       }
-      // rw: the lane's gathered rows of the tile when a.gather and t < nkept
-      auto issue = [&](int t, bool is_v, int4 rw) -> bool {
+      auto issue = [&](int t, bool is_v) -> bool {
         const CUtensorMap* m;
         int row = 0, row2 = -1;
         if (t < nkept) {
           m = is_v ? &tmV : &tmK;
-          if (!a.gather) task_rows(t, row, row2);
+          task_rows(t, row, row2);
         } else {
           m = is_v ? &tmVb : &tmKb;
           row = res_tile(res_tiles, t - nkept) * TILE_ROWS;
@@ -492,12 +458,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (lane == 0)
           free_slot = tc::mbar_wait_fast(empty(s), ((uint32_t)(li / STAGES) & 1u) ^ 1u, abort, a.ctrl, 1);
         if (!__shfl_sync(0xffffffffu, free_slot, 0)) return false;
-        if (lane == 0) tc::mbar_expect_tx(full(s), TILE_BYTES);
-        const uint32_t dst = sRing + s * TILE_BYTES;
-        if (a.gather && t < nkept) {
-          __syncwarp();
-          gather_tile(dst, m, full(s), rw);
-        } else if (lane == 0) {
+        if (lane == 0) {
+          tc::mbar_expect_tx(full(s), TILE_BYTES);
+          const uint32_t dst = sRing + s * TILE_BYTES;
           if (row2 < 0) {
 #pragma unroll
             for (int c = 0; c < NCH; ++c) tc::tma_load_3d(dst + c * CHUNK_BYTES, m, full(s), c * 64, row, bh);
@@ -513,19 +476,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         ++li;
         return true;
       };
-      // K(0), K(1), then per task t: V(t), K(t + 2); gathered rows of tasks
-      // t, t + 1, t + 2 held in ra, rb, rc, task t + 3's fetched as K(t + 2)
-      // goes out
-      int4 ra = task_fetch(0), rb = task_fetch(1);
-      if (ok) ok = issue(0, false, ra);
-      if (ok && T > 1) ok = issue(1, false, rb);
-      int4 rc = task_fetch(2);
+      if (ok) ok = issue(0, false);
+      if (ok && T > 1) ok = issue(1, false);
       for (int t = 0; ok && t < T; ++t) {
-        ok = issue(t, true, ra);
-        if (ok && t + 2 < T) ok = issue(t + 2, false, rc);
-        ra = rb;
-        rb = rc;
-        rc = task_fetch(t + 3);
+        ok = issue(t, true);
+        if (ok && t + 2 < T) ok = issue(t + 2, false);
       }
       ++qn;
       if (!ok) break;
@@ -934,20 +889,6 @@ bool encode_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH, int bo
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [rows, D] bf16 matrix as a 2-D map for row gathers: box = 64 channels x 1
-// row, 128-byte swizzle (rows land as consecutive 128-byte box rows).
-bool encode_rows_map(CUtensorMap* m, const void* ptr, int D, long long rows) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // A tensor map depends only on (pointer, D, rows, BH, box rows): the last few
 // encoded maps of each host thread are kept so repeated calls on the same
 // buffers skip the driver's encode.
@@ -961,7 +902,6 @@ struct MapEntry {
   bool used;
 };
 
-// box = 0 asks for the 2-D row-gather map of [BH * rows, D].
 bool make_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH, int box = TILE_ROWS) {
   constexpr int SLOTS = 16;
   thread_local MapEntry cache[SLOTS] = {};
@@ -974,8 +914,7 @@ bool make_map(CUtensorMap* m, const void* ptr, int D, int rows, int BH, int box 
       return true;
     }
   }
-  if (!(box == 0 ? encode_rows_map(m, ptr, D, (long long)rows * BH) : encode_map(m, ptr, D, rows, BH, box)))
-    return false;
+  if (!encode_map(m, ptr, D, rows, BH, box)) return false;
   MapEntry& e = cache[next];
   next = (next + 1) % SLOTS;
   e.k = MapKey{ptr, D, rows, BH, box};
@@ -1021,18 +960,16 @@ bool attend_tc_supported(const Problem& p) {
 cudaError_t launch_attend_tc(const Problem& p, const void* Q, const void* K, const void* V,
                              const int32_t* row_ptr, const int32_t* col_idx, void* O,
                              const Work& w, cudaStream_t s) {
+  // with a permutation, the workspace's permuted copies (blocked order)
+  const void* q = w.qp ? (const void*)w.qp : Q;
+  const void* k = w.kp ? (const void*)w.kp : K;
+  const void* v = w.vp ? (const void*)w.vp : V;
   // K and V tiles: one 128-row box, or two 64-row boxes (one per block) with
-  // 64-token blocks; with a permutation, rows gathered through it from the
-  // caller's tensors (no permuted copies)
+  // 64-token blocks
   const bool b64 = p.b == TILE_ROWS / 2;
-  const bool gather = p.perm != nullptr;
   CUtensorMap maps[5];
-  const bool ok_maps =
-      gather ? (make_map(&maps[0], Q, p.d, p.N, p.BH, 0) && make_map(&maps[1], K, p.d, p.N, p.BH, 0) &&
-                make_map(&maps[2], V, p.d, p.N, p.BH, 0))
-             : (make_map(&maps[0], Q, p.d, p.N, p.BH) && make_map(&maps[1], K, p.d, p.N, p.BH, p.b) &&
-                make_map(&maps[2], V, p.d, p.N, p.BH, p.b));
-  if (!ok_maps || !make_map(&maps[3], w.kbar16, p.d, p.nb, p.BH) ||
+  if (!make_map(&maps[0], q, p.d, p.N, p.BH) || !make_map(&maps[1], k, p.d, p.N, p.BH, p.b) ||
+      !make_map(&maps[2], v, p.d, p.N, p.BH, p.b) || !make_map(&maps[3], w.kbar16, p.d, p.nb, p.BH) ||
       !make_map(&maps[4], w.vbar16, p.d, p.nb, p.BH))
     return cudaErrorInvalidValue;
   TcArgs a;
@@ -1054,7 +991,6 @@ cudaError_t launch_attend_tc(const Problem& p, const void* Q, const void* K, con
     a.order = nullptr;
   }
   a.perm = p.perm;
-  a.gather = gather ? 1 : 0;
   a.o = static_cast<__nv_bfloat16*>(O);
   a.o32 = nullptr;
   a.q_rows = p.N;

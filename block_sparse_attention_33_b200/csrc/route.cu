@@ -124,88 +124,6 @@ __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
   }
 }
 
-// Rows of at least 256 blocks (one thread per key block and logit, the
-// channels summed in order): Kbar is staged through shared memory in chunks
-// of RB_CHUNK blocks with coalesced loads, and each thread keeps a register
-// tile of ROWS / 4 query rows x 2 key blocks, so a value read from shared
-// memory feeds several logits.  Every logit is the same ordered sum over the
-// channels as in route_kernel (and in the attention's inline selection), so
-// the selections agree bit for bit.  ROWS = 32, or 16 when nb > 1024 (the
-// probability tile S must fit beside the chunk).
-constexpr int RB_CHUNK = 128;
-
-template <int D, int ROWS>
-size_t route_big_smem_bytes(int nb) {
-  const int nbp = (nb + 31) & ~31;
-  return ((size_t)ROWS * D + (size_t)RB_CHUNK * (D + 4) + (size_t)ROWS * nbp) * sizeof(float);
-}
-
-template <int D, int ROWS>
-__global__ void __launch_bounds__(RT_THREADS) route_big_kernel(RouteArgs a) {
-  constexpr int KS = D + 4;             // padded Kbar row (float4-aligned, spreads the banks)
-  constexpr int RPT = ROWS / 4;         // query rows per thread
-  extern __shared__ __align__(16) float sm[];
-  const int nbp = (a.nb + 31) & ~31;
-  float* Qs = sm;                       // [ROWS][D]
-  float* Ks = Qs + ROWS * D;            // [RB_CHUNK][KS]
-  float* S = Ks + RB_CHUNK * KS;        // [ROWS][nbp]
-  const int bh = blockIdx.y, i0 = blockIdx.x * ROWS, tid = threadIdx.x;
-  const int rows = min(ROWS, a.nb - i0);
-  const float* qbar = a.qbar + ((size_t)bh * a.nb + i0) * D;
-  const float* kbar = a.kbar + (size_t)bh * a.nb * D;
-  for (int e = tid; e < ROWS * D; e += RT_THREADS) Qs[e] = (e / D < rows) ? qbar[e] : 0.f;
-
-  const float inv_sqrt_d = 1.0f / sqrtf((float)D);
-  const int jj = tid % 64, rg = tid / 64;   // key blocks jj, jj + 64 of a chunk; rows rg*RPT ..
-  for (int c0 = 0; c0 < a.nb; c0 += RB_CHUNK) {
-    __syncthreads();   // the previous chunk is no longer read
-    for (int e = tid; e < RB_CHUNK * (D / 4); e += RT_THREADS) {
-      const int jr = e / (D / 4), k4 = e % (D / 4), j = c0 + jr;
-      const float4 v = j < a.nb ? __ldg(reinterpret_cast<const float4*>(kbar + (size_t)j * D) + k4)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-      *reinterpret_cast<float4*>(Ks + jr * KS + 4 * k4) = v;
-    }
-    __syncthreads();
-    float acc[RPT][2];
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) acc[r][0] = acc[r][1] = 0.f;
-#pragma unroll 4
-    for (int k4 = 0; k4 < D / 4; ++k4) {
-      const float4 k0 = *reinterpret_cast<const float4*>(Ks + jj * KS + 4 * k4);
-      const float4 k1 = *reinterpret_cast<const float4*>(Ks + (jj + 64) * KS + 4 * k4);
-#pragma unroll
-      for (int r = 0; r < RPT; ++r) {
-        const float4 q = *reinterpret_cast<const float4*>(Qs + (rg * RPT + r) * D + 4 * k4);
-        acc[r][0] = fmaf(q.x, k0.x, acc[r][0]);
-        acc[r][0] = fmaf(q.y, k0.y, acc[r][0]);
-        acc[r][0] = fmaf(q.z, k0.z, acc[r][0]);
-        acc[r][0] = fmaf(q.w, k0.w, acc[r][0]);
-        acc[r][1] = fmaf(q.x, k1.x, acc[r][1]);
-        acc[r][1] = fmaf(q.y, k1.y, acc[r][1]);
-        acc[r][1] = fmaf(q.z, k1.z, acc[r][1]);
-        acc[r][1] = fmaf(q.w, k1.w, acc[r][1]);
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int j = c0 + jj + 64 * h;
-      if (j < a.nb) {
-        const int nj = (j == a.nb - 1) ? a.n_last : a.b;
-        const float lnn = logf((float)nj);
-#pragma unroll
-        for (int r = 0; r < RPT; ++r) S[(rg * RPT + r) * nbp + j] = fmaf(acc[r][h], inv_sqrt_d, lnn);
-      }
-    }
-  }
-  __syncthreads();
-  const int warp = tid >> 5;
-  for (int r = warp; r < rows; r += RT_THREADS / 32) {
-    float* p = S + r * nbp;
-    sel::softmax_row(p, a.nb);
-    select_emit(p, a, bh * a.nb + i0 + r);
-  }
-}
-
 // PAMA block importance (PARK page 5.1): every query token of block i keeps
 // its own softmax over the key blocks of the centroid logit
 // q . Kbar_j / sqrt(d) + ln n_j, and p_i is the mean of the n_i tokens'
@@ -511,22 +429,8 @@ cudaError_t launch_route_rows(const RouteArgs& a, int nb, int BH, cudaStream_t s
   return cudaGetLastError();
 }
 
-template <int D, int ROWS>
-cudaError_t launch_route_big(const RouteArgs& a, int nb, int BH, cudaStream_t s) {
-  const size_t smem = route_big_smem_bytes<D, ROWS>(nb);
-  cudaError_t e = ensure_dyn_smem((const void*)route_big_kernel<D, ROWS>, smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid((nb + ROWS - 1) / ROWS, BH);
-  route_big_kernel<D, ROWS><<<grid, RT_THREADS, smem, s>>>(a);
-  return cudaGetLastError();
-}
-
 template <int D>
 cudaError_t launch_route_d(const RouteArgs& a, int nb, int BH, cudaStream_t s) {
-  // one thread per key block and logit (rows of 256 blocks and more): the
-  // Kbar-staging kernel, with the same per-logit arithmetic
-  if (sel::proxy_threads_per_block(nb) == 1)
-    return nb <= 1024 ? launch_route_big<D, 32>(a, nb, BH, s) : launch_route_big<D, 16>(a, nb, BH, s);
   switch (route_rows_per_cta(nb)) {
     case 4: return launch_route_rows<D, 4>(a, nb, BH, s);
     case 8: return launch_route_rows<D, 8>(a, nb, BH, s);

@@ -104,19 +104,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Row gather (TMA tile::gather4, no multicast): rows r0..r3 of a 2-D tensor
-// map whose box is `box columns x 1 row`, starting at column c0 (its byte
-// offset a multiple of 16), land as four consecutive box rows at dst,
-// completing on mbarrier `bar`.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int c0, int r0, int r1, int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];\n" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
-}
-
 // ---- shared-memory matrix descriptor (sm100 format) ----
 // start address, leading/stride byte offsets (16-byte units), version 1 in
 // bits 46-47, layout type in bits 61-63 (2 = 128-byte swizzle).

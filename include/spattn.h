@@ -47,8 +47,7 @@
  *     spattn_route_static call on a device are not capturable.
  *   - Supported: d in {64, 128}; b in {64, 128}; 1 <= N; nb <= 2048;
  *     1 <= kmin <= kmax (kmax > nb is clamped to nb); tau finite;
- *     B*H <= 65535; B*H*nb*min(kmax, nb) <= 2^31 - 1 (int32 CSR offsets);
- *     with a permutation, B*H*N <= 2^31 - 1 (int32 row indices).
+ *     B*H <= 65535; B*H*nb*min(kmax, nb) <= 2^31 - 1 (int32 CSR offsets).
  */
 #ifndef SPATTN_H_
 #define SPATTN_H_
@@ -154,11 +153,10 @@ spattn_status_t spattn_plan_destroy(spattn_plan_t plan);
  * caller-provided col_idx buffer must have. */
 spattn_status_t spattn_plan_info(spattn_plan_t plan, int* nb, int64_t* col_capacity);
 
-/* Block means: writes the fp32 block means Qbar, Kbar, Vbar (and bf16
- * copies of Kbar, Vbar for the residual tiles) into the workspace, the
- * tokens read through the plan's permutation when it has one (the attention
- * gathers its rows through the permutation as well: no permuted copies of Q,
- * K, V are made).  Q, K, V: bf16 [B, H, N, d] device. */
+/* Gather (if the plan has a permutation) and pool.  Writes the permuted
+ * copies of Q, K, V (read by the attention as whole tiles) and the fp32 block
+ * means Qbar, Kbar, Vbar (with bf16 copies of Kbar, Vbar for the residual
+ * tiles) into the workspace.  Q, K, V: bf16 [B, H, N, d] device. */
 spattn_status_t spattn_pool(spattn_plan_t plan, const void* Q, const void* K, const void* V,
                             void* workspace, void* stream);
 
