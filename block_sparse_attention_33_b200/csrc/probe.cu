@@ -112,7 +112,7 @@ constexpr int GR_ROWS = 128;      // probe rows per Gram CTA
 constexpr int GR_THREADS = 768;
 constexpr int GR_CHUNK = 32;      // rows staged at a time
 constexpr int SV_THREADS = 1024;  // solve kernel
-constexpr int SUB_ITERS = 24;     // subspace iterations
+constexpr int SUB_ITERS = 16;     // subspace iterations
 constexpr int SUB_EXTRA = 16;     // subspace columns beyond r
 constexpr int SUB_MAXQ = 64;      // subspace iteration for r + SUB_EXTRA <= 64, else Jacobi
 
@@ -265,7 +265,10 @@ __device__ void jacobi_cta(float* S, float* V, int n, int ld, float* rc, float* 
       }
       off = warp_sum_f(off);
       dia = warp_sum_f(dia);
-      if (tid == 0) *flag = off <= 1e-12f * dia ? 1 : 0;
+      // 1e-9: the off-diagonal elements are then about 3e-5 of the diagonal's
+      // scale; fp32 rounding alone keeps a converged matrix near 1e-11, so a
+      // tighter test would never stop before the sweep limit
+      if (tid == 0) *flag = off <= 1e-9f * dia ? 1 : 0;
     }
     __syncthreads();
     if (*flag) break;
