@@ -58,6 +58,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstddef>
 #include <type_traits>
 
@@ -117,6 +118,11 @@ struct TcArgs {
   float* o32;                 // or, when set, fp32 output [BH, q_rows, D] in tile order
   int q_rows;                 // query (and output) rows per (batch, head)
   int dense;                  // every key tile of the N keys, no residual (exact rows)
+  // dense rows only: the key tiles cut into `splits` ranges, one item each
+  // (item = tile item * splits + range); range c writes its normalised rows
+  // to o32 + c * BH * q_rows * D and their log2 mass to lse[c][BH][q_rows]
+  int splits;
+  float* lse;
   int32_t* ctrl;
   int N, nb, n_last, residual, items;
   // inline selection (Sol-Attn abstract: blocks chosen inside the attention
@@ -306,8 +312,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       const int item = a.order ? __ldg(a.order + ticket) : ticket;
-      const int bh = item / a.nq, i = item % a.nq;
-      int r_lo = 0, nkept = 0;
+      const int tile_item = item / a.splits, range = item % a.splits;
+      const int bh = tile_item / a.nq, i = tile_item % a.nq;
+      int r_lo = 0, nkept = 0, t0 = 0;
       inf.kept[0][lane] = 0u;
       inf.kept[0][lane + 32] = 0u;
       inf.kept[1][lane] = 0u;
@@ -318,9 +325,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       __syncwarp();
       const bool pair2 = a.b64 && 2 * i + 1 < a.nb;   // the tile holds a second query block
       if (a.dense) {
-        // exact rows: every key tile, in order
-        nkept = a.nb;
-        if (lane == 0 && a.n_last < TILE_ROWS) inf.tail_task = a.nb - 1;
+        // exact rows: every key tile of this item's range, in order
+        const int per = (a.nb + a.splits - 1) / a.splits;
+        t0 = range * per;
+        const int t1 = min(a.nb, t0 + per);
+        nkept = max(0, t1 - t0);
+        if (lane == 0 && t1 == a.nb && nkept > 0 && a.n_last < TILE_ROWS) inf.tail_task = nkept - 1;
         __syncwarp();
       } else if (a.inline_sel) {
         const SelArgs sa{a.qbar, a.kbar, a.nb, a.n_last, a.blk, a.threshold, a.kmin, a.kcap, a.tau};
@@ -422,7 +432,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           row = j0 * 64;
           row2 = j1 * 64;
         } else if (a.dense) {
-          row = t * TILE_ROWS;
+          row = (t0 + t) * TILE_ROWS;
         } else if (a.inline_sel) {
           row = inf.ublk[t] * TILE_ROWS;
         } else {
@@ -620,7 +630,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (item < 0) break;
       const int T = inf.T, nkept = inf.nkept, tail_task = inf.tail_task;
       const uint32_t res_tiles = inf.res_tiles;
-      const int bh = item / a.nq, i = item % a.nq;
       // m: reference maximum of this row's key half (log2 units); l: sum of
       // p at that reference; owe: factor O_h owes once PV(g-1) is done.
       float m = -INFINITY, l = 0.f, owe = 1.f;
@@ -797,11 +806,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const float a0 = m0 == -INFINITY ? 0.f : tc::ex2(m0 - M);
         const float a1 = m1 == -INFINITY ? 0.f : tc::ex2(m1 - M);
         const float L = a0 * cs->xl[slot][0][r] + a1 * cs->xl[slot][1][r];
-        const int tok = i * TILE_ROWS + r;
+        // query tile and output head (key range c of a split dense item
+        // writes its own copy, c * (batch, head) pairs further on)
+        const int it = item / a.splits;
+        const int obh = (item % a.splits) * (a.items / (a.splits * a.nq)) + it / a.nq;
+        const int tok = (it % a.nq) * TILE_ROWS + r;
         const bool store = tok < a.q_rows;   // rows past the last query are padding
         const int dst = store ? (a.perm ? __ldg(a.perm + tok) : tok) : 0;
-        const size_t obase = ((size_t)bh * a.q_rows + dst) * D + half * (D / 2);
+        const size_t obase = ((size_t)obh * a.q_rows + dst) * D + half * (D / 2);
         const float inv = L > 0.f ? 1.f / L : 0.f;
+        if (a.lse && store && half == 0)   // log2 of the row's mass: sum of 2^(s sl2) = 2^M L
+          a.lse[(size_t)obh * a.q_rows + dst] =
+              L > 0.f ? M + __log2f(L) : -INFINITY;
         const float w0 = a0 * inv, w1 = a1 * inv;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
@@ -995,6 +1011,8 @@ cudaError_t launch_attend_tc(const Problem& p, const void* Q, const void* K, con
   a.o32 = nullptr;
   a.q_rows = p.N;
   a.dense = 0;
+  a.splits = 1;
+  a.lse = nullptr;
   a.ctrl = w.ctrl;
   a.N = p.N; a.nb = p.nb; a.n_last = p.n_last; a.residual = p.residual;
   a.b64 = b64 ? 1 : 0;
@@ -1149,13 +1167,59 @@ cudaError_t launch_apply_tc_d(const Problem& p, void* O, const void* Wt, const f
   return cudaGetLastError();
 }
 
+// Rows of split key ranges put together: range c holds each row normalised
+// over its own keys plus the log2 of its mass, so the full row is the
+// mass-weighted mean of the ranges.  One warp per row, a float4 per lane.
+__global__ void __launch_bounds__(256) dense_combine_kernel(const float* part, const float* lse,
+                                                            float* out, int rows, int splits, int d) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float mx = -INFINITY;
+  for (int c = 0; c < splits; ++c) mx = fmaxf(mx, lse[(size_t)c * rows + row]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float wsum = 0.f;
+  const int d4 = d / 4;
+  for (int c = 0; c < splits; ++c) {
+    const float lc = lse[(size_t)c * rows + row];
+    const float w = lc == -INFINITY ? 0.f : exp2f(lc - mx);
+    wsum += w;
+    if (lane < d4) {
+      const float4 v = reinterpret_cast<const float4*>(part + ((size_t)c * rows + row) * d)[lane];
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  if (lane < d4)
+    reinterpret_cast<float4*>(out + (size_t)row * d)[lane] =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+}
+
+// Key ranges per dense tile item: the count (at most DENSE_MAX_SPLITS, at
+// most one range per key tile) whose waves of items over the SMs finish
+// soonest, in units of one unsplit item; the fewest ranges on a tie.
+static int dense_splits(int items, int nb, int sms) {
+  int best = 1;
+  double best_t = std::ceil((double)items / sms);
+  for (int s = 2; s <= std::min(DENSE_MAX_SPLITS, nb); ++s) {
+    const double tm = std::ceil((double)items * s / sms) / s;
+    if (tm < best_t) { best_t = tm; best = s; }
+  }
+  return best;
+}
+
 // Exact (dense) softmax attention of gathered query rows, fp32 out: Qg holds
 // q_alloc rows per (batch, head) (a multiple of 128, zero past q_rows), every
 // one of the N keys of K and V is attended, and rows [0, q_rows) of each head
 // are written to out [BH, q_rows, d].  The probe correction's exact rows.
+// When there are too few 128-row tiles to fill the GPU, each tile's keys are
+// cut into ranges (part: DENSE_MAX_SPLITS x [BH, q_rows, d] fp32, lse:
+// DENSE_MAX_SPLITS x [BH, q_rows]) put together by dense_combine_kernel.
 cudaError_t launch_dense_rows_tc(const Problem& p, const void* Qg, int q_alloc, int q_rows,
-                                 const void* K, const void* V, float* out, int32_t* ctrl,
-                                 cudaStream_t s) {
+                                 const void* K, const void* V, float* out, float* part, float* lse,
+                                 int32_t* ctrl, cudaStream_t s) {
   const int nb = (p.N + TILE_ROWS - 1) / TILE_ROWS;
   CUtensorMap maps[5];
   if (!make_map(&maps[0], Qg, p.d, q_alloc, p.BH) || !make_map(&maps[1], K, p.d, p.N, p.BH) ||
@@ -1163,10 +1227,13 @@ cudaError_t launch_dense_rows_tc(const Problem& p, const void* Qg, int q_alloc, 
     return cudaErrorInvalidValue;
   maps[3] = maps[1];   // no residual tiles: the centroid maps are never read
   maps[4] = maps[2];
+  int dev = 0, sms = 148;
+  cudaError_t e;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   TcArgs a{};
   a.dense = 1;
   a.o = nullptr;
-  a.o32 = out;
   a.q_rows = q_rows;
   a.ctrl = ctrl;
   a.N = p.N; a.nb = nb; a.n_last = p.N - (nb - 1) * TILE_ROWS; a.residual = 0;
@@ -1175,13 +1242,19 @@ cudaError_t launch_dense_rows_tc(const Problem& p, const void* Qg, int q_alloc, 
   a.nq = q_alloc / TILE_ROWS;
   a.kcap = nb;
   a.sl2 = 1.4426950408889634f / sqrtf((float)p.d);
-  a.items = p.BH * a.nq;
+  a.splits = (part && lse) ? dense_splits(p.BH * a.nq, nb, sms) : 1;
+  a.o32 = a.splits > 1 ? part : out;
+  a.lse = a.splits > 1 ? lse : nullptr;
+  a.items = p.BH * a.nq * a.splits;
   // the work ticket and retirement count start from zero (the workspace may
   // never have run an attention); the error word is left as it is
   static_assert(CTRL_DONE == CTRL_WORK + 1, "ticket words cleared together");
-  cudaError_t e = cudaMemsetAsync(ctrl + CTRL_WORK, 0, 2 * sizeof(int32_t), s);
-  if (e != cudaSuccess) return e;
-  return p.d == 128 ? launch_tc<128>(maps, a, s) : launch_tc<64>(maps, a, s);
+  if ((e = cudaMemsetAsync(ctrl + CTRL_WORK, 0, 2 * sizeof(int32_t), s)) != cudaSuccess) return e;
+  if ((e = p.d == 128 ? launch_tc<128>(maps, a, s) : launch_tc<64>(maps, a, s)) != cudaSuccess) return e;
+  if (a.splits == 1) return cudaSuccess;
+  const int rows = p.BH * q_rows;
+  dense_combine_kernel<<<(rows + 7) / 8, 256, 0, s>>>(part, lse, out, rows, a.splits, p.d);
+  return cudaGetLastError();
 }
 
 // O <- O + O W + c per head on the tensor cores (the probe correction's

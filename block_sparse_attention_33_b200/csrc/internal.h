@@ -59,8 +59,11 @@ cudaError_t launch_attend(const Problem& p, const void* Q, const void* K, const 
 // q_alloc a multiple of 128) over all N keys of K and V, fp32 output rows
 // [BH, q_rows, d]; the tcgen05 attention kernel in its dense mode.
 cudaError_t launch_dense_rows_tc(const Problem& p, const void* Qg, int q_alloc, int q_rows,
-                                 const void* K, const void* V, float* out, int32_t* ctrl,
-                                 cudaStream_t s);
+                                 const void* K, const void* V, float* out, float* part, float* lse,
+                                 int32_t* ctrl, cudaStream_t s);
+// key ranges a dense tile item may be cut into (part / lse buffers of the
+// dense rows hold this many copies)
+constexpr int DENSE_MAX_SPLITS = 8;
 
 // O <- O + O W + c for every row of every head, on the tensor cores: Wt is
 // bf16 [BH, d, d] holding W transposed (row n = column n of W), c fp32 [BH, d].

@@ -268,9 +268,10 @@ spattn_status_t spattn_probe_scratch_bytes(spattn_plan_t plan, int M, size_t* by
  * The exact probe rows run on the tensor cores, as the attention does (bf16
  * operands, fp32 accumulation), with an fp32 output.  The fit is fp32: one
  * Gram pass over the probe rows [1, x, R] gives the (d+1) x (d+1) normal
- * equations (solved by Cholesky factorisation) and R^T R, whose r leading
+ * equations (inverted by Gauss-Jordan elimination) and R^T R, whose r leading
  * eigenvectors come from block subspace iteration with a Rayleigh-Ritz step
- * (r + 16 <= 64; cyclic Jacobi on the whole matrix otherwise).  The pass
+ * (r + 16 <= 64 and < d; cyclic Jacobi on the whole matrix otherwise).  The
+ * pass
  * O += O (B P) + b P runs on the tensor cores with B P in bf16 (the
  * correction is a small fraction of the output) and fp32 accumulation.  Normal
  * equations that are not positive definite (lam = 0 with fewer than d + 1

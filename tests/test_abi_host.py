@@ -232,21 +232,24 @@ def test_binding_checks_host_tensors_of_the_host_forward(L):
 
 def test_probe_correct_argument_checks(L):
     """spattn_probe_scratch_bytes sizes the exact rows, the fit, B P, b P, the
-    gathered probe queries (whole 128-row tiles), the subspace basis and the
-    per-slab Gram matrices of [1, x, R] (slabs of 128 probe rows, width
-    1 + 2 d padded to a multiple of 4); spattn_probe_correct refuses bad
-    arguments before any CUDA call."""
+    gathered probe queries (whole 128-row tiles), the subspace basis, one
+    Gram matrix of [1, x, R] per head (width 1 + 2 d padded to a multiple of
+    4, whatever the number of probes), and up to 8 key ranges of the exact
+    rows with their log2 masses; spattn_probe_correct refuses bad arguments
+    before any CUDA call."""
     B, H, N, d = 1, 3, 1000, 64
     st, h, ws = plan_status(B, H, N, d, 64, 0.9, 1, 4, 1)
     assert st == sp.OK
     up = lambda x: (x + 255) // 256 * 256
     n = ctypes.c_size_t()
-    M = 48
-    assert L.spattn_probe_scratch_bytes(h, M, ctypes.byref(n)) == sp.OK
     zw = (1 + 2 * d + 3) // 4 * 4
-    assert n.value == (up(B * H * M * d * 4) + up(B * H * (d + 1) * d * 4) + up(B * H * d * d * 4)
-                       + up(B * H * d * 4) + up(B * H * 128 * d * 2) + up(B * H * d * d * 4)
-                       + up(B * H * 1 * zw * zw * 4))
+    for M in (300, 48):
+        assert L.spattn_probe_scratch_bytes(h, M, ctypes.byref(n)) == sp.OK
+        assert n.value == (up(B * H * M * d * 4) + up(B * H * (d + 1) * d * 4)
+                           + up(B * H * d * d * 4) + up(B * H * d * 4)
+                           + up(B * H * ((M + 127) // 128 * 128) * d * 2) + up(B * H * d * d * 4)
+                           + up(B * H * zw * zw * 4)
+                           + up(8 * B * H * M * d * 4) + up(8 * B * H * M * 4))
     assert L.spattn_probe_scratch_bytes(h, 0, ctypes.byref(n)) == sp.ERR_INVALID_ARG
     f = L.spattn_probe_correct
     ok = dict(Q=16, K=16, V=16, O=16, probes=16, M=M, lam=100.0, r=8, ws=256, scratch=256)
