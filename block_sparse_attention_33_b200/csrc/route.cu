@@ -60,26 +60,13 @@ __device__ void select_emit(const float* p, const RouteArgs& a, int row) {
 }
 
 
+// Proxy logits S[r][j] = Qbar_r . Kbar_j / sqrt(d) + ln n_j of a routing
+// CTA's rows.  Split form: a group of TPJ threads owns key block j (all
+// rows), each thread a strided share of the channels, reduced with shuffles;
+// TPJ = 256 / nb (at most 32) keeps every thread busy when nb is small.
 template <int D, int RT_ROWS>
-__global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
-  extern __shared__ __align__(16) float sm[];
-  const int nbp = (a.nb + 31) & ~31;
-  float* Qs = sm;                       // [RT_ROWS][D]
-  float* S = sm + RT_ROWS * D;          // [RT_ROWS][nbp]
-  const int bh = blockIdx.y, i0 = blockIdx.x * RT_ROWS;
-  const int rows = min(RT_ROWS, a.nb - i0);
-  const float* qbar = a.qbar + ((size_t)bh * a.nb + i0) * D;
-  const float* kbar = a.kbar + (size_t)bh * a.nb * D;
-
-  for (int e = threadIdx.x; e < RT_ROWS * D; e += RT_THREADS)
-    Qs[e] = (e / D < rows) ? qbar[e] : 0.f;
-  __syncthreads();
-
-  // ---- proxy logits: a group of TPJ threads owns key block j (all rows),
-  // each thread a strided share of the channels, reduced with shuffles;
-  // TPJ = 256 / nb (at most 32) keeps every thread busy when nb is small
-  const float inv_sqrt_d = 1.0f / sqrtf((float)D);
-  const int tpj = sel::proxy_threads_per_block(a.nb);
+__device__ __forceinline__ void proxy_split(const float* Qs, const float* kbar, float* S, int nbp,
+                                            const RouteArgs& a, float inv_sqrt_d, int tpj) {
   const int sub = threadIdx.x % tpj, grp = threadIdx.x / tpj, ngrp = RT_THREADS / tpj;
   for (int j0 = 0; j0 < a.nb; j0 += ngrp) {
     const int j = j0 + grp;
@@ -112,6 +99,86 @@ __global__ void __launch_bounds__(RT_THREADS) route_kernel(RouteArgs a) {
 #pragma unroll
       for (int r = 0; r < RT_ROWS; ++r) S[r * nbp + j] = fmaf(acc[r], inv_sqrt_d, lnn);
     }
+  }
+}
+
+// Tiled form, one thread per block (nb >= 256): a thread takes JT blocks, so
+// that each mean row of Q read from shared memory feeds JT dot products;
+// every dot product is still one fma chain over the channels in order, the
+// arithmetic of the split form with TPJ = 1.  (Spreading a warp's quarters
+// over different rows instead, so that each shared-memory read serves one
+// quarter, measured slower on B200: the key rows' global reads then feed
+// too few FMAs each.)
+template <int D, int RT_ROWS>
+__device__ __forceinline__ void proxy_tiled(const float* Qs, const float* kbar, float* S, int nbp,
+                                            const RouteArgs& a, float inv_sqrt_d) {
+  constexpr int JT = RT_ROWS >= 16 ? 2 : 4;   // 32 accumulators a thread
+  for (int j0 = 0; j0 < a.nb; j0 += JT * RT_THREADS) {
+    float acc[JT][RT_ROWS];
+    const float4* kr[JT];
+    bool live[JT];
+#pragma unroll
+    for (int u = 0; u < JT; ++u) {
+      const int j = j0 + u * RT_THREADS + threadIdx.x;
+      live[u] = j < a.nb;
+      kr[u] = reinterpret_cast<const float4*>(kbar + (size_t)(live[u] ? j : 0) * D);
+#pragma unroll
+      for (int r = 0; r < RT_ROWS; ++r) acc[u][r] = 0.f;
+    }
+#pragma unroll 2
+    for (int k4 = 0; k4 < D / 4; ++k4) {
+      float4 kv[JT];
+#pragma unroll
+      for (int u = 0; u < JT; ++u) kv[u] = live[u] ? __ldg(kr[u] + k4) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int r = 0; r < RT_ROWS; ++r) {
+        const float4 q = reinterpret_cast<const float4*>(Qs + r * D)[k4];
+#pragma unroll
+        for (int u = 0; u < JT; ++u) {
+          acc[u][r] = fmaf(q.x, kv[u].x, acc[u][r]);
+          acc[u][r] = fmaf(q.y, kv[u].y, acc[u][r]);
+          acc[u][r] = fmaf(q.z, kv[u].z, acc[u][r]);
+          acc[u][r] = fmaf(q.w, kv[u].w, acc[u][r]);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < JT; ++u) {
+      const int j = j0 + u * RT_THREADS + threadIdx.x;
+      if (live[u]) {
+        const int nj = (j == a.nb - 1) ? a.n_last : a.b;
+        const float lnn = logf((float)nj);
+#pragma unroll
+        for (int r = 0; r < RT_ROWS; ++r) S[r * nbp + j] = fmaf(acc[u][r], inv_sqrt_d, lnn);
+      }
+    }
+  }
+}
+
+template <int D, int RT_ROWS>
+__global__ void __launch_bounds__(RT_THREADS, RT_ROWS >= 8 ? 2 : 1) route_kernel(RouteArgs a) {
+  extern __shared__ __align__(16) float sm[];
+  const int nbp = (a.nb + 31) & ~31;
+  float* Qs = sm;                       // [RT_ROWS][D]
+  float* S = sm + RT_ROWS * D;          // [RT_ROWS][nbp]
+  const int bh = blockIdx.y, i0 = blockIdx.x * RT_ROWS;
+  const int rows = min(RT_ROWS, a.nb - i0);
+  const float* qbar = a.qbar + ((size_t)bh * a.nb + i0) * D;
+  const float* kbar = a.kbar + (size_t)bh * a.nb * D;
+
+  for (int e = threadIdx.x; e < RT_ROWS * D; e += RT_THREADS)
+    Qs[e] = (e / D < rows) ? qbar[e] : 0.f;
+  __syncthreads();
+
+  // ---- proxy logits (nb >= 256 means at least 8 rows a CTA: only those
+  // instantiations carry the tiled form) ----
+  const float inv_sqrt_d = 1.0f / sqrtf((float)D);
+  const int tpj = sel::proxy_threads_per_block(a.nb);
+  if constexpr (RT_ROWS >= 8) {
+    if (tpj == 1) proxy_tiled<D, RT_ROWS>(Qs, kbar, S, nbp, a, inv_sqrt_d);
+    else proxy_split<D, RT_ROWS>(Qs, kbar, S, nbp, a, inv_sqrt_d, tpj);
+  } else {
+    proxy_split<D, RT_ROWS>(Qs, kbar, S, nbp, a, inv_sqrt_d, tpj);
   }
   __syncthreads();
 
@@ -319,6 +386,7 @@ cudaError_t launch_pama_d(const RouteArgs& a, const void* Q, const int32_t* perm
 // group.  The order is a counting sort on the key
 // group * (kcap + 1) + (kcap - count).
 constexpr int SCAN_THREADS = 1024;
+constexpr size_t SCAN_SMEM_MAX = 200 * 1024;   // histogram plus staged counts
 
 // Exclusive prefix sum over the CTA's threads (SCAN_THREADS = 32 warps):
 // shuffle scans inside each warp, one warp scans the warp totals.  `part`
@@ -350,14 +418,23 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* part) {
   return ex;
 }
 
-__global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(const int32_t* counts, int rows,
-                                                            int kcap, int group_rows,
+__global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(const int32_t* counts_g, int rows,
+                                                            int kcap, int group_rows, int stage,
                                                             int32_t* row_ptr, int32_t* order,
                                                             int32_t* ctrl) {
   __shared__ int part[32];
-  extern __shared__ int hist[];  // [ngroups * (kcap + 1)]
+  extern __shared__ int hist[];  // [ngroups * (kcap + 1)], then the counts when staged
   const int ngroups = (rows + group_rows - 1) / group_rows;
   const int nbins = ngroups * (kcap + 1);
+  // every thread reads a contiguous range of counts three times: from shared
+  // memory when they fit (one coalesced pass over global memory)
+  const int32_t* counts = counts_g;
+  if (stage) {
+    int* cs = hist + nbins;
+    for (int q = threadIdx.x; q < rows; q += SCAN_THREADS) cs[q] = counts_g[q];
+    counts = cs;
+    __syncthreads();   // (stage is the same for every thread)
+  }
   auto key = [&](int q) { return (q / group_rows) * (kcap + 1) + (kcap - min(counts[q], kcap)); };
   const int per = (rows + SCAN_THREADS - 1) / SCAN_THREADS;
   const int lo = threadIdx.x * per, hi = min(rows, lo + per);
@@ -487,9 +564,12 @@ cudaError_t launch_route(const Problem& p, const Work& w, const void* Q, int32_t
   const int group_rows = scan_group_rows(p);
   const size_t hist_bytes =
       (size_t)((rows + group_rows - 1) / group_rows) * (p.kcap + 1) * sizeof(int);
-  if ((e = ensure_dyn_smem((const void*)scan_kernel, hist_bytes)) != cudaSuccess) return e;
-  scan_kernel<<<1, SCAN_THREADS, hist_bytes, s>>>(w.counts, rows, p.kcap, group_rows, w.row_ptr,
-                                                  w.order, w.ctrl);
+  const size_t staged = hist_bytes + (size_t)rows * sizeof(int);
+  const int stage = staged <= SCAN_SMEM_MAX ? 1 : 0;
+  const size_t smem = stage ? staged : hist_bytes;
+  if ((e = ensure_dyn_smem((const void*)scan_kernel, smem)) != cudaSuccess) return e;
+  scan_kernel<<<1, SCAN_THREADS, smem, s>>>(w.counts, rows, p.kcap, group_rows, stage, w.row_ptr,
+                                            w.order, w.ctrl);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (!need_csr && !row_ptr_out && !col_idx_out) return cudaSuccess;
   compact_kernel<<<(rows + 7) / 8, 256, 0, s>>>(w.counts, w.lists, w.row_ptr, rows, p.kcap,

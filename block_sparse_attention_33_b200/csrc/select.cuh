@@ -17,7 +17,8 @@
 // where v is the smallest value whose strictly-larger mass is < tau.  A
 // search over the bit patterns finds v: 32-way for rows of at most 128
 // blocks (each lane evaluates one candidate over the whole row), binary with
-// one warp reduction per step otherwise.  The same search on the count
+// one warp reduction per step otherwise (the row held in registers up to 1024
+// blocks).  The same search on the count
 // #{p_j > u} yields the top-k set when the clamp binds.  Kept blocks are then
 // walked in ascending j with warp ballots.
 #pragma once
@@ -110,6 +111,34 @@ __device__ __forceinline__ int count_above_1(const float* p, int nb, uint32_t u)
 
 // rows with at most this many blocks use the 32-way search
 constexpr int SEARCH32_MAX_NB = 128;
+// longer rows up to this many blocks run the binary search on registers
+constexpr int REG_MAX_NB = 1024;
+
+// A row in registers: lane l holds p[l + 32 i] in pv[i], +0 past the row
+// (bits 0: never above any u, so the mass and count below skip it).  The
+// sums run in the order of mass_above / count_above (i ascending per lane,
+// then the same xor tree), so they are the same numbers.
+__device__ __forceinline__ void row_to_regs(const float* p, int nb, float (&pv)[REG_MAX_NB / 32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < REG_MAX_NB / 32; ++i) {
+    const int j = lane + 32 * i;
+    pv[i] = j < nb ? p[j] : 0.f;
+  }
+}
+__device__ __forceinline__ float mass_above_r(const float (&pv)[REG_MAX_NB / 32], uint32_t u) {
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < REG_MAX_NB / 32; ++i)
+    if (__float_as_uint(pv[i]) > u) s += pv[i];
+  return warp_sum(s);
+}
+__device__ __forceinline__ int count_above_r(const float (&pv)[REG_MAX_NB / 32], uint32_t u) {
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < REG_MAX_NB / 32; ++i) c += (__float_as_uint(pv[i]) > u) ? 1 : 0;
+  return warp_sum_i(c);
+}
 
 // The cut of one probability row: keep {bits(p) > thr} plus the first `ties`
 // blocks (ascending j) with bits(p) == thr, or every block when `all`; k is
@@ -144,8 +173,17 @@ __device__ __forceinline__ Cut cut_row(const float* p, int nb, float tau, int th
   } else if (tau > 0.0f) {
     if (nb <= SEARCH32_MAX_NB) {
       thr = search32(0u, 0x3F800000u, [&](uint32_t u) { return mass_above_1(p, nb, u) < tau; });
-    } else {
+    } else if (nb <= REG_MAX_NB) {
+      float pv[REG_MAX_NB / 32];
+      row_to_regs(p, nb, pv);
       uint32_t lo = 0, hi = 0x3F800000u;  // p <= 1, so nothing is above hi
+      while (lo < hi) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (mass_above_r(pv, mid) < tau) hi = mid; else lo = mid + 1;
+      }
+      thr = lo;
+    } else {
+      uint32_t lo = 0, hi = 0x3F800000u;
       while (lo < hi) {
         const uint32_t mid = lo + ((hi - lo) >> 1);
         if (mass_above(p, nb, mid) < tau) hi = mid; else lo = mid + 1;
@@ -170,6 +208,15 @@ __device__ __forceinline__ Cut cut_row(const float* p, int nb, float tau, int th
     // the clamp binds (or tau <= 0): top-k in (p desc, j asc) order
     if (nb <= SEARCH32_MAX_NB) {
       thr = search32(0u, 0x3F800000u, [&](uint32_t u) { return count_above_1(p, nb, u) < k; });
+    } else if (nb <= REG_MAX_NB) {
+      float pv[REG_MAX_NB / 32];
+      row_to_regs(p, nb, pv);
+      uint32_t lo = 0, hi = 0x3F800000u;
+      while (lo < hi) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (count_above_r(pv, mid) < k) hi = mid; else lo = mid + 1;
+      }
+      thr = lo;
     } else {
       uint32_t lo = 0, hi = 0x3F800000u;
       while (lo < hi) {
