@@ -41,17 +41,19 @@ L2_NOTE = "flushed (256 MiB write between timed steps)"
 # ncu capture of the bench command for that workload, keyed by kernel and
 # (workload, heads, tau, residual).  Valid only while the kernel's sources are
 # the ones captured: each entry carries a hash of them, and the bench reports
-# null when the hash no longer matches.
+# null when the hash no longer matches.  The HunyuanVideo-like entries (24
+# heads) are 3 x the capture of the same layer with 8 heads: the heads are
+# independent and every head's key and value tiles are read the same way, so
+# the bytes grow with the head count.
 MEASURED_TRAFFIC = {
-    "attention": {"sources": ["attn_tc.cu", "tc.cuh", "common.cuh"],
-                  "sha": "dad78e858eb2aed2",
-                  "bytes": {("medium", 8, 0.9, 1): 51736832, ("wan", 8, 0.9, 1): 279409664,
-                            ("stress", 8, 0.7, 1): 245197056}},
-    # medium / wan: pool_kernel (contiguous blocks); stress: pool_gather_kernel
+    "attention": {"sources": ["attn_tc.cu", "tc.cuh", "common.cuh", "select.cuh"],
+                  "sha": "857b37df0d5c2d2f",
+                  "bytes": {("hunyuan", 24, 0.95, 1): 3 * 2727366144}},
+    # wan / hunyuan: pool_kernel (contiguous blocks); stress: pool_gather_kernel
     "pool": {"sources": ["pool.cu", "tc.cuh", "common.cuh"],
-             "sha": "45cb4400ecca3a58",
-             "bytes": {("medium", 8, 0.9, 1): 50362112, ("wan", 8, 0.9, 1): 206082304,
-                       ("stress", 8, 0.7, 1): 356619008}},
+             "sha": "da762629b964bc69",
+             "bytes": {("wan", 8, 0.9, 1): 206850048, ("stress", 8, 0.7, 1): 357913344,
+                       ("hunyuan", 24, 0.95, 1): 3 * 746453248}},
 }
 
 
