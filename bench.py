@@ -105,7 +105,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-chunk", type=int, default=0,
                     help="heads per chunk of spattn_forward_host in the e2e figure (host "
-                         "tensors, copies overlapped over chunks); 0: a quarter of the heads")
+                         "tensors, copies overlapped over chunks); 0: the binding's default")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the compact timing of every seeded configuration")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -619,7 +619,7 @@ def run_ours(args):
         qh, kh, vh = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
                       for x in (Qh, Kh, Vh))
         oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
-        chunk = args.e2e_chunk if args.e2e_chunk > 0 else max(1, (B * H + 3) // 4)
+        chunk = args.e2e_chunk if args.e2e_chunk > 0 else sp.default_chunk_heads(B * H)
 
         def pipe_step():
             plan.forward_host(qh, kh, vh, oh, chunk_heads=chunk)

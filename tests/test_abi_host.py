@@ -361,3 +361,12 @@ def test_build_stamp_tells_variant_builds_apart(L):
     assert not build.up_to_date(("-DSPATTN_EXP_EMU=2",))
     with open(build.STAMP) as f:
         assert f.read() == ""
+
+
+def test_default_chunk_heads():
+    """The host pipeline's default chunk balances the exposed first/last
+    copies against the last attention wave of every chunk: about
+    sqrt(BH / 5) heads, at least 1 and at most BH."""
+    f = sp.default_chunk_heads
+    assert [f(x) for x in (1, 2, 8, 24, 40, 80)] == [1, 1, 1, 2, 3, 4]
+    assert all(1 <= f(x) <= x for x in range(1, 200))
