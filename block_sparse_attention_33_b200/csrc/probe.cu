@@ -300,8 +300,13 @@ __device__ __forceinline__ void jacobi_rot(const float* S, int ld, int p, int q,
   s = 0.f;
   if (fabsf(apq) > 1e-30f) {
     const float theta = __fdividef(aqq - app, 2.f * apq);
-    const float h2 = fmaf(theta, theta, 1.f);            // sqrt(h2) = h2 rsqrt(h2)
-    const float tt = __fdividef(copysignf(1.f, theta), fabsf(theta) + h2 * rsqrtf(h2));
+    float tt;
+    if (fabsf(theta) > 1e18f) {
+      tt = __fdividef(0.5f, theta);   // theta^2 would overflow: t = 1 / (2 theta) to first order
+    } else {
+      const float h2 = fmaf(theta, theta, 1.f);   // sqrt(h2) = h2 rsqrt(h2), h2 < 1e37
+      tt = __fdividef(copysignf(1.f, theta), fabsf(theta) + h2 * rsqrtf(h2));
+    }
     c = rsqrtf(fmaf(tt, tt, 1.f));
     s = tt * c;
   }
@@ -695,7 +700,7 @@ __device__ void subspace_role(const float* gh, int r, float* U, float* sm) {
         // broadcast float4 reads
         float* colk = Pp + (k & 1) * QN;
         const float dkk = __shfl_sync(0xffffffffu, c[k >> 5][k], k & 31);
-        const bool dead = !(dkk > tiny);
+        const bool dead = !(dkk > tiny && dkk < INFINITY);
         const float rk = dead ? 0.f : rsqrtf(dkk);   // approximate: the next step re-orthonormalises
         const float lkk = dkk * rk;
 #pragma unroll
@@ -726,7 +731,7 @@ __device__ void subspace_role(const float* gh, int r, float* U, float* sm) {
 #pragma unroll
       for (int k = 0; k < QN; ++k) {   // QN = 64: columns of L passed by shuffles
         const float dkk = __shfl_sync(0xffffffffu, c[k >> 5][k], k & 31);
-        const bool dead = !(dkk > tiny);
+        const bool dead = !(dkk > tiny && dkk < INFINITY);
         const float rk = dead ? 0.f : rsqrtf(dkk);
         const float lkk = dkk * rk;
 #pragma unroll
@@ -901,17 +906,37 @@ __global__ void __launch_bounds__(PB_THREADS) probe_fold_kernel(const ProbeArgs 
   const float* U = a.pu + (size_t)bh * D * D;
   for (int e = tid; e < D * r; e += PB_THREADS) Us[(e / r) * rp + e % r] = U[(e / r) * D + e % r];
   __syncthreads();
+  // four interleaved partial sums (channels j mod 4), added in a fixed order:
+  // short dependent chains for a latency-bound loop
+  int nonfinite = 0;
   for (int e = tid; e < (D + 1) * r; e += PB_THREADS) {
     const int i = e / r, k = e % r;
-    float s = 0.f;
-    for (int j = 0; j < D; ++j) s = fmaf(Ws[i * D + j], Us[j * rp + k], s);
-    BU[i * rp + k] = s;
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int j = 0; j < D; j += 4)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) s[q] = fmaf(Ws[i * D + j + q], Us[(j + q) * rp + k], s[q]);
+    const float v = (s[0] + s[1]) + (s[2] + s[3]);
+    nonfinite |= !isfinite(v);
+    BU[i * rp + k] = v;
   }
-  __syncthreads();
+  // a fit or subspace that is not finite leaves the head uncorrected, flagged
+  if (__syncthreads_or(nonfinite)) {
+    if (tid == 0) flag_error(a.ctrl, DEV_NUMERIC, bh);
+    for (int e = tid; e < D * D; e += PB_THREADS) wt[e] = __float2bfloat16_rn(0.f);
+    for (int c = tid; c < D; c += PB_THREADS) cp[c] = 0.f;
+    return;
+  }
   for (int e = tid; e < (D + 1) * D; e += PB_THREADS) {
     const int j = e / (D + 1), i = e % (D + 1);   // (B P)[i - 1][j], or (b P)[j] for i = 0
-    float s = 0.f;
-    for (int k = 0; k < r; ++k) s = fmaf(BU[i * rp + k], Us[j * rp + k], s);
+    float s0 = 0.f, s1 = 0.f;
+    int k = 0;
+    for (; k + 1 < r; k += 2) {
+      s0 = fmaf(BU[i * rp + k], Us[j * rp + k], s0);
+      s1 = fmaf(BU[i * rp + k + 1], Us[j * rp + k + 1], s1);
+    }
+    if (k < r) s0 = fmaf(BU[i * rp + k], Us[j * rp + k], s0);
+    const float s = s0 + s1;
     if (i == 0) cp[j] = s; else wt[(size_t)j * D + (i - 1)] = __float2bfloat16_rn(s);
   }
 }

@@ -71,6 +71,47 @@ def test_probe_correction_against_oracle(desc, name, ov, per_block, lam, r):
                     <= 2.0 ** -8 * np.abs(dense).max() + 1e-5)
 
 
+PATH_CASES = [
+    # heavier sparsity (tau 0.5, 1-2 kept blocks) so the correction stands well above the
+    # bf16 rounding of the output; r picks the device's subspace path
+    ("tiny r=16: 32-column subspace", "tiny", dict(kmax=1, tau=0.5), 16, 16),
+    ("tiny r=24: whole-matrix Jacobi (d=64)", "tiny", dict(kmax=1, tau=0.5), 16, 24),
+    ("medium r=16: 32-column subspace", "medium", dict(H=2, tau=0.5, kmax=2), 4, 16),
+    ("medium r=40: 64-column subspace", "medium", dict(H=2, tau=0.5, kmax=2), 4, 40),
+    ("medium r=64: whole-matrix Jacobi", "medium", dict(H=2, tau=0.5, kmax=2), 4, 64),
+    ("medium r=d: P = I", "medium", dict(H=2, tau=0.5, kmax=2), 4, 128),
+]
+
+
+@pytest.mark.parametrize("desc,name,ov,per_block,r", PATH_CASES, ids=[c[0] for c in PATH_CASES])
+def test_probe_correction_itself_on_every_subspace_path(desc, name, ov, per_block, r):
+    """The correction o_corr - o_sparse (rows other than the probes) against the oracle's
+    want - o_sparse.  The device output is one bf16 rounding of the corrected value, an
+    error of at most 2^-9 |o| per element, about |o| 2^-9 / sqrt(3) in rms, while the
+    oracle's is exact: the bound is three times that noise relative to the correction, plus
+    2 % for the fp32 fit, the bf16 B P of the tensor-core apply and the iterative subspace.
+    A wrong subspace or fit is off by order one, a non-finite one fails outright."""
+    import block_sparse_attention_33_b200 as sp
+    w = get_config(name, **ov)
+    Q, K, V, probes, o_sparse, o_corr, status = _run(w, per_block, 100.0, r)
+    assert status == sp.OK
+    for hi in range(w.H):
+        q, k, v = (R.decode_bf16(X[0, hi]) for X in (Q, K, V))
+        rows = probes[0, hi].astype(np.int64)
+        dense = P.dense_rows(q, k, v, rows)
+        want = P.correct(o_sparse[0, hi], dense, rows, 100.0, r)
+        keep = np.ones(w.N, bool)
+        keep[rows] = False
+        got_c = (o_corr[0, hi] - o_sparse[0, hi])[keep]
+        want_c = (want - o_sparse[0, hi])[keep]
+        assert np.all(np.isfinite(got_c)), hi
+        noise = 2.0 ** -9 * np.linalg.norm(o_sparse[0, hi][keep]) / np.sqrt(3.0)
+        scale = np.linalg.norm(want_c)
+        assert scale > 10 * noise, (hi, scale, noise)   # the case measures something
+        rel = np.linalg.norm(got_c - want_c) / scale
+        assert rel < 3 * noise / scale + 0.02, (hi, rel, noise / scale)
+
+
 def test_probe_index_out_of_range_is_flagged():
     import block_sparse_attention_33_b200 as sp
     w = get_config("tiny", kmax=2)
