@@ -270,13 +270,13 @@ spattn_status_t spattn_probe_scratch_bytes(spattn_plan_t plan, int M, size_t* by
  * Gram pass over the probe rows [1, x, R] gives the (d+1) x (d+1) normal
  * equations (inverted by Gauss-Jordan elimination) and R^T R, whose r leading
  * eigenvectors come from block subspace iteration with a Rayleigh-Ritz step
- * (r + 16 <= 64 and < d; cyclic Jacobi on the whole matrix otherwise).  The
- * pass
+ * (r + 16 <= d / 2; cyclic Jacobi on the whole matrix otherwise).  The pass
  * O += O (B P) + b P runs on the tensor cores with B P in bf16 (the
  * correction is a small fraction of the output) and fp32 accumulation.  Normal
  * equations that are not positive definite (lam = 0 with fewer than d + 1
- * independent probe rows, for instance) leave that head uncorrected and are
- * flagged (spattn_check: SPATTN_ERR_DEVICE).  B*H <= 65535. */
+ * independent probe rows, for instance), or a fit or subspace that is not
+ * finite, leave that head uncorrected and are flagged (spattn_check:
+ * SPATTN_ERR_DEVICE).  B*H <= 65535. */
 spattn_status_t spattn_probe_correct(spattn_plan_t plan, const void* Q, const void* K,
                                      const void* V, void* O, const int32_t* probes, int M,
                                      float lam, int r, void* workspace, void* scratch,
