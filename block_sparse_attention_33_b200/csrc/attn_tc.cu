@@ -758,15 +758,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tc::tmem_st32(scol, pk);   // P(g) over this warp's own, already read, columns
         l += lt;
         // O_h owes `owe` once PV(g-1) is done (factor 1 on rows owing
-        // nothing); only a warp with a row that owes waits for it.  The
-        // parity names that one PV: S(g), whose completion this warp has
-        // waited for, was issued after PV(g-2) and the tensor core runs in
-        // issue order, so every earlier PV is complete, and PV(g) cannot
-        // start before this warp's P(g) is ready.
-        if (t > 0 && __any_sync(0xffffffffu, owe != 1.f)) {
+        // nothing).  Every phase of the PV barrier inside an item is waited
+        // for, and the item's first task follows the previous item's OFULL,
+        // so the parity always names the one PV in question.
+        if (t > 0) {
           if (!(ok = wait_warp(bar(B_PVDONE), (uint32_t)(g - 1) & 1u, 10))) break;
-          tc::tc_fence_after();
-          rescale_o(owe);
+          if (__any_sync(0xffffffffu, owe != 1.f)) {
+            tc::tc_fence_after();
+            rescale_o(owe);
+          }
         }
         owe = 1.f;
         // keep p moderate: when this tile's sum passes 2^16 the reference
