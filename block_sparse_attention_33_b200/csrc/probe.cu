@@ -440,6 +440,17 @@ __device__ void rank_values(const float* S, int n, int ld, int* rank) {
   __syncthreads();
 }
 
+// A residual basis that is not finite: the head's correction is left out
+// (its first r columns of U zeroed, so B P = 0) and flagged.  Every thread
+// of the CTA calls this after writing its share of U.
+template <int D>
+__device__ void basis_check(float* U, int r, int nonfinite, int32_t* ctrl, int bh) {
+  if (__syncthreads_or(nonfinite)) {
+    if (threadIdx.x == 0) flag_error(ctrl, DEV_NUMERIC, bh);
+    for (int e = threadIdx.x; e < D * r; e += blockDim.x) U[(e / r) * D + e % r] = 0.f;
+  }
+}
+
 // role 0: W = (G + lam diag(0, 1, ..., 1))^-1 C.  The inverse is taken in
 // place by Gauss-Jordan elimination without pivoting (the matrix is
 // symmetric positive definite), the matrix held in registers: thread
@@ -518,15 +529,19 @@ __device__ void fit_role(const ProbeArgs& a, const float* gh, int bh, float* sm)
 #pragma unroll
       for (int b = 0; b < NS; ++b) A[s][b] = fmaf(-u[s], v[b], A[s][b]);
   }
+  int nonfinite = 0;
 #pragma unroll
   for (int s = 0; s < NS; ++s)
 #pragma unroll
     for (int b = 0; b < NS; ++b) {
       const int i = ty + GJ_G * s, j = tx + GJ_G * b;
       if (i < N && j < LDA) Ai[i * LDA + j] = j < N ? A[s][b] : 0.f;
+      nonfinite |= !isfinite(A[s][b]);
     }
-  __syncthreads();
-  const bool failed = *badp != 0;
+  for (int e = tid; e < N * D; e += SV_THREADS) nonfinite |= !isfinite(Cm[e]);
+  // a pivot that was not positive, or an inverse or right-hand side that is
+  // not finite: the head is left uncorrected (W = 0) and flagged
+  const bool failed = __syncthreads_or(nonfinite) || *badp != 0;
   if (failed && tid == 0) flag_error(a.ctrl, DEV_NUMERIC, bh);
   float* w = a.w + (size_t)bh * N * D;
   // W = Ai C on 4 x 4 tiles; the inverse is symmetric, so its row j serves as
@@ -569,7 +584,7 @@ __device__ void fit_role(const ProbeArgs& a, const float* gh, int bh, float* sm)
 // in the registers of one warp (QN / 32 rows per lane, columns of L passed
 // by shuffles); the triangular solve one thread per row of Y.
 template <int D, int QN>
-__device__ void subspace_role(const float* gh, int r, float* U, float* sm) {
+__device__ void subspace_role(const float* gh, int r, float* U, float* sm, int32_t* ctrl, int bh) {
   constexpr int DS = D + 4, TP = QN + 1, QB = QN / 4, ZW = gram_w<D>();
   constexpr int TILES = QB * QB, SL = SV_THREADS / TILES > 1 ? SV_THREADS / TILES : 1;
   static_assert(QN % 32 == 0 && QN < D, "subspace width");
@@ -798,19 +813,22 @@ __device__ void subspace_role(const float* gh, int r, float* U, float* sm) {
   if constexpr (QN == 32) Td = jacobi32(T, Y, L, TP, red);   // Y is free: its second buffer
   else jacobi_cta(T, L, QN, TP, rc, rs, pq, red);
   rank_values(Td, QN, TP, rank);
+  int nonfinite = 0;
   for (int e = tid; e < D * QN; e += SV_THREADS) {
     const int row = e / QN, col = e % QN;
     if (rank[col] < r) {
       float acc = 0.f;
       for (int k = 0; k < QN; ++k) acc = fmaf(X[row * QN + k], L[k * TP + col], acc);
       U[row * D + rank[col]] = acc;
+      nonfinite |= !isfinite(acc);
     }
   }
+  basis_check<D>(U, r, nonfinite, ctrl, bh);
 }
 
 // role 1 without room for the extra columns: Jacobi on the whole D x D matrix.
 template <int D>
-__device__ void eigen_role(const float* gh, int r, float* U, float* sm) {
+__device__ void eigen_role(const float* gh, int r, float* U, float* sm, int32_t* ctrl, int bh) {
   constexpr int DP = D + 1, ZW = gram_w<D>();
   float* S = sm;                  // [D][DP]
   float* V = S + D * DP;          // [D][DP]
@@ -826,10 +844,15 @@ __device__ void eigen_role(const float* gh, int r, float* U, float* sm) {
   __syncthreads();
   jacobi_cta(S, V, D, DP, rc, rs, pq, red);
   rank_values(S, D, DP, rank);
+  int nonfinite = 0;
   for (int e = tid; e < D * D; e += SV_THREADS) {
     const int row = e / D, col = e % D;
-    if (rank[col] < r) U[row * D + rank[col]] = V[row * DP + col];
+    if (rank[col] < r) {
+      U[row * D + rank[col]] = V[row * DP + col];
+      nonfinite |= !isfinite(V[row * DP + col]);
+    }
   }
+  basis_check<D>(U, r, nonfinite, ctrl, bh);
 }
 
 // One instantiation per subspace width QN = sub_cols(r, D) (0: the whole-
@@ -847,8 +870,8 @@ __global__ void __launch_bounds__(SV_THREADS) probe_solve_kernel(const ProbeArgs
   }
   if (r >= D) return;   // P = I: the fold needs no U
   float* U = a.pu + (size_t)bh * D * D;
-  if constexpr (QN > 0) subspace_role<D, QN>(gh, r, U, psm);
-  else eigen_role<D>(gh, r, U, psm);
+  if constexpr (QN > 0) subspace_role<D, QN>(gh, r, U, psm, a.ctrl, bh);
+  else eigen_role<D>(gh, r, U, psm, a.ctrl, bh);
 }
 
 template <int D, int QN>
@@ -863,81 +886,77 @@ cudaError_t launch_solve(const ProbeArgs& a, const float* gp, cudaStream_t s) {
 }
 
 // B P and b P with P = U U^T (U: the first r columns), or P = 0 / I for
-// r = 0 / r >= D; one CTA per head.  B P goes out transposed in bf16 (row n
-// holds column n: the K-major operand of the tensor-core apply; the
-// correction is about a thousandth of the output, so bf16 rounding of it is
-// far below the output's own rounding), b P in fp32.  WU = W U first (one
-// thread per (row, k), k across lanes), then (W U) U^T with the output
-// column i across lanes, so that the transposed bf16 rows are written whole.
+// r = 0 / r >= D.  B P goes out transposed in bf16 (row n holds column n: the
+// K-major operand of the tensor-core apply; the correction is about a
+// thousandth of the output, so bf16 rounding of it is far below the output's
+// own rounding), b P in fp32.  FOLD_SPLIT CTAs per head, each taking a range
+// of rows of W = [b; B]: W U for its rows (one thread per (row, k)), then
+// (W U) U^T with the output row across lanes.  The solve kernel has already
+// zeroed W or U where the fit or the basis was not finite.
+constexpr int FOLD_SPLIT = 8;
+
+template <int D>
+constexpr int fold_rows() { return (D + 1 + FOLD_SPLIT - 1) / FOLD_SPLIT; }
+
 template <int D>
 size_t fold_smem_bytes(int r) {
   const int rr = (r > 0 && r < D) ? r : 0;
-  return ((size_t)(D + 1) * D + (size_t)D * (rr + 1) + (size_t)(D + 1) * (rr + 1)) * sizeof(float);
+  return ((size_t)fold_rows<D>() * D + (size_t)D * (rr + 1) + (size_t)fold_rows<D>() * (rr + 1)) *
+         sizeof(float);
 }
 
 template <int D>
 __global__ void __launch_bounds__(PB_THREADS) probe_fold_kernel(const ProbeArgs a) {
   extern __shared__ __align__(16) float psm[];
+  constexpr int RW = fold_rows<D>();
   const int bh = blockIdx.x, tid = threadIdx.x;
+  const int i0 = blockIdx.y * RW, i1 = min(D + 1, i0 + RW), nr = i1 - i0;   // rows of W
+  if (nr <= 0) return;
   const int r = a.r;
-  float* Ws = psm;                  // [D + 1][D]: row 0 = b, rows 1.. = B
+  float* Ws = psm;                  // [nr][D]: rows i0 .. i1 - 1 of W (row 0 = b, rows 1.. = B)
   const float* wfit = a.w + (size_t)bh * (D + 1) * D;
   __nv_bfloat16* wt = a.wt + (size_t)bh * D * D;
   float* cp = a.cp + (size_t)bh * D;
+  // output element (j, row i) of B P (i >= 1: W^T row j, column i - 1) or b P (i = 0)
+  auto put = [&](int j, int i, float v) {
+    if (i == 0) cp[j] = v; else wt[(size_t)j * D + (i - 1)] = __float2bfloat16_rn(v);
+  };
   if (r <= 0) {
-    for (int e = tid; e < D * D; e += PB_THREADS) wt[e] = __float2bfloat16_rn(0.f);
-    for (int c = tid; c < D; c += PB_THREADS) cp[c] = 0.f;
+    for (int e = tid; e < D * nr; e += PB_THREADS) put(e / nr, i0 + e % nr, 0.f);
     return;
   }
-  for (int e = tid; e < (D + 1) * D / 4; e += PB_THREADS)
-    reinterpret_cast<float4*>(Ws)[e] = reinterpret_cast<const float4*>(wfit)[e];
+  for (int e = tid; e < nr * D / 4; e += PB_THREADS)
+    reinterpret_cast<float4*>(Ws)[e] = reinterpret_cast<const float4*>(wfit + (size_t)i0 * D)[e];
   __syncthreads();
   if (r >= D) {
-    for (int e = tid; e < D * D; e += PB_THREADS) {
-      const int n = e / D, k = e % D;   // W^T[n][k] = B[k][n]
-      wt[e] = __float2bfloat16_rn(Ws[(k + 1) * D + n]);
+    for (int e = tid; e < D * nr; e += PB_THREADS) {
+      const int j = e / nr, q = e % nr;   // (B P)[i - 1][j] = B[i - 1][j]
+      put(j, i0 + q, Ws[q * D + j]);
     }
-    for (int c = tid; c < D; c += PB_THREADS) cp[c] = Ws[c];
     return;
   }
   const int rp = r + 1;
-  float* Us = Ws + (D + 1) * D;     // [D][r + 1]
-  float* BU = Us + D * rp;          // [D + 1][r + 1]: row 0 = b U, rows 1.. = B U
+  float* Us = Ws + RW * D;          // [D][r + 1]
+  float* BU = Us + D * rp;          // [nr][r + 1]
   const float* U = a.pu + (size_t)bh * D * D;
   for (int e = tid; e < D * r; e += PB_THREADS) Us[(e / r) * rp + e % r] = U[(e / r) * D + e % r];
   __syncthreads();
-  // four interleaved partial sums (channels j mod 4), added in a fixed order:
-  // short dependent chains for a latency-bound loop
-  int nonfinite = 0;
-  for (int e = tid; e < (D + 1) * r; e += PB_THREADS) {
-    const int i = e / r, k = e % r;
+  // four interleaved partial sums (channels j mod 4), added in a fixed order
+  for (int e = tid; e < nr * r; e += PB_THREADS) {
+    const int q = e / r, k = e % r;
     float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
     for (int j = 0; j < D; j += 4)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) s[q] = fmaf(Ws[i * D + j + q], Us[(j + q) * rp + k], s[q]);
-    const float v = (s[0] + s[1]) + (s[2] + s[3]);
-    nonfinite |= !isfinite(v);
-    BU[i * rp + k] = v;
+      for (int c = 0; c < 4; ++c) s[c] = fmaf(Ws[q * D + j + c], Us[(j + c) * rp + k], s[c]);
+    BU[q * rp + k] = (s[0] + s[1]) + (s[2] + s[3]);
   }
-  // a fit or subspace that is not finite leaves the head uncorrected, flagged
-  if (__syncthreads_or(nonfinite)) {
-    if (tid == 0) flag_error(a.ctrl, DEV_NUMERIC, bh);
-    for (int e = tid; e < D * D; e += PB_THREADS) wt[e] = __float2bfloat16_rn(0.f);
-    for (int c = tid; c < D; c += PB_THREADS) cp[c] = 0.f;
-    return;
-  }
-  for (int e = tid; e < (D + 1) * D; e += PB_THREADS) {
-    const int j = e / (D + 1), i = e % (D + 1);   // (B P)[i - 1][j], or (b P)[j] for i = 0
-    float s0 = 0.f, s1 = 0.f;
-    int k = 0;
-    for (; k + 1 < r; k += 2) {
-      s0 = fmaf(BU[i * rp + k], Us[j * rp + k], s0);
-      s1 = fmaf(BU[i * rp + k + 1], Us[j * rp + k + 1], s1);
-    }
-    if (k < r) s0 = fmaf(BU[i * rp + k], Us[j * rp + k], s0);
-    const float s = s0 + s1;
-    if (i == 0) cp[j] = s; else wt[(size_t)j * D + (i - 1)] = __float2bfloat16_rn(s);
+  __syncthreads();
+  for (int e = tid; e < D * nr; e += PB_THREADS) {
+    const int j = e / nr, q = e % nr;
+    float s = 0.f;
+    for (int k = 0; k < r; ++k) s = fmaf(BU[q * rp + k], Us[j * rp + k], s);
+    put(j, i0 + q, s);
   }
 }
 
@@ -966,7 +985,7 @@ cudaError_t launch_probe_d(const Problem& p, const ProbeArgs& a, int m_alloc, __
   else if (qn == 64) e = launch_solve<D, (64 < D ? 64 : 0)>(a, gp, s);
   else e = launch_solve<D, 0>(a, gp, s);
   if (e != cudaSuccess) return e;
-  probe_fold_kernel<D><<<a.BH, PB_THREADS, fold_smem_bytes<D>(a.r), s>>>(a);
+  probe_fold_kernel<D><<<dim3(a.BH, FOLD_SPLIT), PB_THREADS, fold_smem_bytes<D>(a.r), s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = launch_probe_apply_tc(p, a.o, a.wt, a.cp, a.ctrl, s)) != cudaSuccess) return e;
   probe_set_kernel<D><<<dim3(a.M, a.BH), D, 0, s>>>(a);
