@@ -13,7 +13,9 @@
 //                       tcgen05 attention kernel in its dense mode: exact
 //                       softmax attention of those rows over all N keys, fp32
 //                       output (bf16 operands, fp32 accumulation, as every
-//                       attention row of this library);
+//                       attention row of this library), the keys cut into
+//                       ranges put together afterwards when the tiles are
+//                       too few to fill the GPU;
 //   probe_gram_kernel   the Gram matrix of the probe rows [1, x, R] (one CTA
 //                       per pair of 64-column blocks and head, all probe rows
 //                       in order): its blocks are A^T A, A^T R and R^T R for
@@ -25,7 +27,7 @@
 //                       singular vectors of R) by block subspace iteration
 //                       with a Rayleigh-Ritz step, or cyclic Jacobi on the
 //                       whole matrix for large r;
-//   probe_fold_kernel   B P and b P with P = U U^T;
+//   probe_fold_kernel   B P and b P with P = U U^T (eight CTAs per head);
 //   then the tcgen05 apply (launch_probe_apply_tc): O <- O + O (B P) + b P
 //                       for every row, bf16 out;
 //   probe_set_kernel    probe rows <- their exact output.
@@ -33,8 +35,8 @@
 // The fit and the subspace are fp32; B P enters the tensor-core apply in
 // bf16 (the correction it makes is about a thousandth of the output).  A
 // probe index outside [0, N) is skipped and flagged (DEV_BAD_INDEX); normal
-// equations that are not positive definite leave that head uncorrected and
-// are flagged (DEV_NUMERIC).
+// equations that are not positive definite, or a fit or residual basis that
+// is not finite, leave that head uncorrected and are flagged (DEV_NUMERIC).
 #include <math.h>
 
 #include "common.cuh"
