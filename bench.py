@@ -101,6 +101,9 @@ def parse_args(argv=None):
                     help="skip the extra timing of threshold selection at --theta")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the number of heads (smaller profiling captures)")
+    ap.add_argument("--block", type=int, default=None, choices=[64, 128],
+                    help="override the block size b (64-token blocks: two query blocks per "
+                         "128-row tile of the attention)")
     ap.add_argument("--no-dense", action="store_true", help="skip the tau = 1 comparison run")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-chunk", type=int, default=0,
@@ -137,6 +140,13 @@ def workload_from_args(args, rank=0):
         ov["residual"] = args.residual
     if args.heads is not None:
         ov["H"] = args.heads
+    if args.block is not None:
+        ov["b"] = args.block
+        # the budget cap is a block count: keep it the same share of the blocks
+        base = get_config(args.workload)
+        nb_base = -(-base.N // base.b)
+        nb_new = -(-base.N // args.block)
+        ov["kmax"] = max(1, min(nb_new, -(-base.kmax * nb_new // nb_base)))
     w = get_config(args.workload, **ov)
     if rank:
         w = w.with_(seed=w.seed + 1000 * rank)   # independent replica per rank
