@@ -121,3 +121,17 @@ def test_default_arguments_are_one_gpu_and_a_short_run():
     assert a.gpus == 1 and a.impl == "ours" and a.workload == "hunyuan"
     assert a.warmup >= 3 and 1 <= a.steps <= 100
     assert a.selection == "top_p" and a.routing == "centroid"
+
+
+def test_block_override_keeps_the_budget_share():
+    """--block 64 doubles the block count of a layer and scales the budget cap with it, so
+    the cap keeps the same share of the blocks (never above nb)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    for name in ("medium", "wan", "hunyuan", "stress"):
+        base = bench.workload_from_args(bench.parse_args(["--workload", name]))
+        w = bench.workload_from_args(bench.parse_args(["--workload", name, "--block", "64"]))
+        nb0, nb1 = -(-base.N // base.b), -(-w.N // 64)
+        assert w.b == 64 and w.N == base.N and w.tau == base.tau
+        assert w.kmax == min(nb1, -(-base.kmax * nb1 // nb0))
+    assert bench.workload_from_args(bench.parse_args(["--block", "128"])).b == 128
